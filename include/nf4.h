@@ -1,0 +1,182 @@
+/*
+ * nf4.h -- C ABI of libnf4.so: QLoRA NF4 blockwise weight quantization with
+ * double quantization, dequantization and the fused frozen-base LoRA linear,
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages, cited by title and section):
+ *   [MF]  "QLoRA: Mathematical Foundations of 4-Bit NormalFloat Quantization,
+ *         Double Quantization, and Paged Optimizers" (llms.blog)
+ *   [L15] "Lesson 15. NF4 and Double Quantisation" (tokencemetery)
+ *   [AD]  "QLoRA: quantising the part you are not training" (addaly.com)
+ *   [QP]  "QLoRA in Production: 4-bit NormalFloat & Double Quantization Deep
+ *         Dive" (devtechtools.org)
+ *
+ * Conventions for every entry point
+ *   - Device buffers are allocated and owned by the caller; the library never
+ *     allocates or frees device memory.  Pointers marked "device" must point
+ *     to memory of the current CUDA device; "host" pointers to host memory.
+ *   - Device pointers must be 16-byte aligned (NF4_ERR_INVALID otherwise).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls only enqueue work: they return once the kernels are
+ *     launched, and results are valid after the stream is synchronized.
+ *   - Sizes are element counts unless named *_bytes.
+ *   - Inputs must be finite (not checked).
+ *   - Return value: NF4_OK, NF4_ERR_INVALID (bad pointer, size or alignment;
+ *     nothing was launched), NF4_ERR_UNSUPPORTED (a block size or rank this
+ *     build does not implement; nothing was launched), NF4_ERR_CUDA (a CUDA
+ *     launch or runtime error; see nf4_last_cuda_error), NF4_ERR_TIMEOUT
+ *     (reported only by nf4_device_status: a bounded wait inside a kernel
+ *     expired and the kernel returned early; its outputs are invalid).
+ *
+ * Data layout (READINGS of what the pages leave open are marked):
+ *   - A weight W[N, K] (PyTorch Linear layout, row n = output feature n) is
+ *     flattened row-major, n = N*K elements, and cut into contiguous blocks of
+ *     64 ([MF] "Block-Wise Quantization Mechanics"; the last block may be
+ *     shorter).  nblocks = ceil(n / 64).
+ *   - packed: uint8[n/2]; READING: element 2j in the high nibble of byte j,
+ *     element 2j+1 in the low nibble.  Codes index the NF4 table.
+ *   - absmax: fp32[nblocks], c1 = max |w| of each block.
+ *   - Double quantization ([MF] "Double Quantization (DQ)"): absmax_q
+ *     uint8[nblocks] holds OCP FP8 E4M3 codes (READING of "FP8") of
+ *     (c1 - mu) / c2; absmax2 fp32[ceil(nblocks / 256)] holds c2 per run of
+ *     256 constants; offset fp32[1] holds mu, one per tensor (READING of the
+ *     "bias/mean subtraction"; NULL offset = no centring, mu = 0).
+ *   - Storage per parameter: 0.5 + 1/64 + 4/16384 bytes ([L15] "Double
+ *     quantisation"), plus 4 bytes of offset per tensor.
+ */
+#ifndef NF4_H_
+#define NF4_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NF4_OK = 0,
+    NF4_ERR_INVALID = 1,
+    NF4_ERR_UNSUPPORTED = 2,
+    NF4_ERR_CUDA = 3,
+    NF4_ERR_TIMEOUT = 4
+} nf4_status;
+
+typedef enum { NF4_F32 = 0, NF4_BF16 = 1 } nf4_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char *nf4_status_string(nf4_status s);
+
+/* The last CUDA error code (cudaError_t as int) seen by a call that
+ * returned NF4_ERR_CUDA in this process; 0 if none. */
+int nf4_last_cuda_error(void);
+
+/* nf4_codebook -- the sixteen NF4 levels q_0..q_15 ([MF] section "4-Bit
+ * NormalFloat (NF4)", the printed list: q_0 = -1, q_7 = 0, q_15 = 1).
+ * out_host: host float[16], written in index order.  NF4_ERR_INVALID if
+ * NULL.  Pure host call; no device work. */
+nf4_status nf4_codebook(float *out_host);
+
+/* nf4_quantize -- blockwise NF4 quantization ([MF] "Block-Wise Quantization
+ * Mechanics": c1 = max_j |w_j| per contiguous block of 64, code_j = arg-min_i
+ * |w_j / c1 - q_i|).  The quotient w_j / c1 is the IEEE binary32 quotient;
+ * READING: exact ties go to the lower index; an all-zero block gives c1 = 0
+ * and code 7 (the exact zero) for every element.
+ *   w        device, n elements of w_dtype (NF4_F32 or NF4_BF16)
+ *   n        element count, even, >= 0
+ *   blocksize must be 64 (else NF4_ERR_UNSUPPORTED)
+ *   packed   device uint8[n/2]  (output)
+ *   absmax   device fp32[ceil(n/64)]  (output)
+ * One kernel launch. */
+nf4_status nf4_quantize(const void *w, nf4_dtype w_dtype, int64_t n, int blocksize,
+                        uint8_t *packed, float *absmax, void *stream);
+
+/* Bytes of device workspace nf4_double_quantize needs for nblocks first-level
+ * constants with centring (0 when nblocks == 0). */
+int64_t nf4_double_quantize_workspace_size(int64_t nblocks, int dq_blocksize);
+
+/* nf4_double_quantize -- quantize the fp32 block constants to 8 bits in runs
+ * of 256, each run with an fp32 second-level scale ([MF] "Double Quantization
+ * (DQ)": c2 = max |c1| per run, c1_FP8 = quantize_FP8(c1 / c2)).
+ * READINGS: the 8-bit format is OCP FP8 E4M3, round to nearest even,
+ * saturating; with `offset` non-NULL one per-tensor mean mu is subtracted
+ * first (c2 = max |c1 - mu|, code = E4M3((c1 - mu) / c2), each step one
+ * binary32 rounding), where mu = RN_f32(S / nblocks) and S is a fixed-order
+ * binary64 sum: each run of 256 summed in index order, then the run sums
+ * combined pairwise level by level (an odd last element carried up).  A run
+ * with c2 = 0 stores code 0.
+ *   absmax     device fp32[nblocks]   (input, from nf4_quantize)
+ *   nblocks    >= 0
+ *   dq_blocksize must be 256 (else NF4_ERR_UNSUPPORTED)
+ *   absmax_q   device uint8[nblocks]  (output)
+ *   absmax2    device fp32[ceil(nblocks/256)]  (output)
+ *   offset     device fp32[1] (output mu) or NULL (no centring)
+ *   workspace  device scratch of workspace_bytes >=
+ *              nf4_double_quantize_workspace_size(); may be NULL when offset
+ *              is NULL.  Contents on entry are ignored; the caller keeps
+ *              ownership; it must not be used by other work until the
+ *              stream passes this call.
+ * Two kernel launches with centring, one without. */
+nf4_status nf4_double_quantize(const float *absmax, int64_t nblocks, int dq_blocksize,
+                               uint8_t *absmax_q, float *absmax2, float *offset,
+                               void *workspace, int64_t workspace_bytes, void *stream);
+
+/* nf4_dequantize -- w~_j = c1' * q[code_j] in binary32 ([MF] "Block-Wise
+ * Quantization Mechanics", dequantization equation), with the block constant
+ *   c1' = fma(E4M3(absmax_q[b]), absmax2[b/256], *offset)   (one rounding;
+ *         READING), or E4M3(absmax_q[b]) * absmax2[b/256] when offset is NULL,
+ *   or, when absmax_q is NULL (no double quantization), c1' = absmax2[b]
+ *   taken as the fp32 first-level constants absmax[nblocks].
+ * NF4_BF16 output is the binary32 value rounded to nearest-even bfloat16 (the
+ * compute dtype of [MF] "Forward Pass Computation").
+ *   packed     device uint8[n/2]
+ *   absmax_q   device uint8[nblocks] or NULL
+ *   absmax2    device fp32[ceil(nblocks/256)] (or fp32[nblocks] if absmax_q
+ *              is NULL)
+ *   offset     device fp32[1] or NULL
+ *   n          even, >= 0; blocksize 64; dq_blocksize 256
+ *   out        device, n elements of out_dtype (output)
+ * One kernel launch. */
+nf4_status nf4_dequantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2,
+                          const float *offset, int64_t n, int blocksize, int dq_blocksize,
+                          void *out, nf4_dtype out_dtype, void *stream);
+
+/* Bytes of device workspace nf4_lora_linear_fwd needs for M rows of x and
+ * rank r (0 when r == 0). */
+int64_t nf4_lora_linear_workspace_size(int64_t M, int r);
+
+/* nf4_lora_linear_fwd -- the frozen-base LoRA linear of [MF] "Forward Pass
+ * Computation", Y = X dequant(c1, c2, W) + (alpha/r)(X L1) L2, in weight
+ * layout:  y = x W~^T + s (x A^T) B^T,  with W~ the bf16-rounded dequantized
+ * weight (dequantized on the fly, never written to memory: [MF] "The
+ * dequantization operation does not materialize ..."), bf16 inputs, fp32
+ * accumulation, bf16 output.  Internally t = s x A^T is formed first in fp32
+ * and kept as a bf16 hi/lo pair (t ~ t_hi + t_lo) in the workspace.
+ *   x          device bf16[M, K] row-major
+ *   M >= 1, K % 64 == 0, N >= 1
+ *   packed, absmax_q, absmax2, offset: the quantized W[N, K] (as for
+ *              nf4_dequantize; absmax_q NULL = fp32 first-level constants)
+ *   A          device bf16[r, K] or NULL;  B  device bf16[N, r] or NULL
+ *   r          0, 16, 32 or 64 (0 or NULL A/B: no low-rank term)
+ *   scaling    s = alpha / r
+ *   y          device bf16[M, N] (output)
+ *   workspace  device scratch, workspace_bytes >=
+ *              nf4_lora_linear_workspace_size(M, r); NULL allowed when r == 0
+ * M <= 16 runs the streaming GEMV kernel, larger M the tensor-core GEMM
+ * kernel; the LoRA pre-step is one extra launch when r > 0. */
+nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N,
+                               const uint8_t *packed, const uint8_t *absmax_q,
+                               const float *absmax2, const float *offset,
+                               const void *A, const void *B, int r, float scaling,
+                               void *y, void *workspace, int64_t workspace_bytes, void *stream);
+
+/* nf4_device_status -- synchronize `stream`, then read and clear the
+ * library's device error word on the current device.  Returns
+ * NF4_ERR_TIMEOUT if a bounded wait in a kernel expired since the last call,
+ * NF4_ERR_CUDA on a CUDA error, NF4_OK otherwise. */
+nf4_status nf4_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NF4_H_ */
