@@ -49,6 +49,12 @@
 
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define NF4_API __attribute__((visibility("default")))
+#else
+#define NF4_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -64,17 +70,17 @@ typedef enum {
 typedef enum { NF4_F32 = 0, NF4_BF16 = 1 } nf4_dtype;
 
 /* Human-readable name of a status code (static string). */
-const char *nf4_status_string(nf4_status s);
+NF4_API const char *nf4_status_string(nf4_status s);
 
 /* The last CUDA error code (cudaError_t as int) seen by a call that
  * returned NF4_ERR_CUDA in this process; 0 if none. */
-int nf4_last_cuda_error(void);
+NF4_API int nf4_last_cuda_error(void);
 
 /* nf4_codebook -- the sixteen NF4 levels q_0..q_15 ([MF] section "4-Bit
  * NormalFloat (NF4)", the printed list: q_0 = -1, q_7 = 0, q_15 = 1).
  * out_host: host float[16], written in index order.  NF4_ERR_INVALID if
  * NULL.  Pure host call; no device work. */
-nf4_status nf4_codebook(float *out_host);
+NF4_API nf4_status nf4_codebook(float *out_host);
 
 /* nf4_quantize -- blockwise NF4 quantization ([MF] "Block-Wise Quantization
  * Mechanics": c1 = max_j |w_j| per contiguous block of 64, code_j = arg-min_i
@@ -87,12 +93,12 @@ nf4_status nf4_codebook(float *out_host);
  *   packed   device uint8[n/2]  (output)
  *   absmax   device fp32[ceil(n/64)]  (output)
  * One kernel launch. */
-nf4_status nf4_quantize(const void *w, nf4_dtype w_dtype, int64_t n, int blocksize,
+NF4_API nf4_status nf4_quantize(const void *w, nf4_dtype w_dtype, int64_t n, int blocksize,
                         uint8_t *packed, float *absmax, void *stream);
 
 /* Bytes of device workspace nf4_double_quantize needs for nblocks first-level
  * constants with centring (0 when nblocks == 0). */
-int64_t nf4_double_quantize_workspace_size(int64_t nblocks, int dq_blocksize);
+NF4_API int64_t nf4_double_quantize_workspace_size(int64_t nblocks, int dq_blocksize);
 
 /* nf4_double_quantize -- quantize the fp32 block constants to 8 bits in runs
  * of 256, each run with an fp32 second-level scale ([MF] "Double Quantization
@@ -116,7 +122,7 @@ int64_t nf4_double_quantize_workspace_size(int64_t nblocks, int dq_blocksize);
  *              ownership; it must not be used by other work until the
  *              stream passes this call.
  * Two kernel launches with centring, one without. */
-nf4_status nf4_double_quantize(const float *absmax, int64_t nblocks, int dq_blocksize,
+NF4_API nf4_status nf4_double_quantize(const float *absmax, int64_t nblocks, int dq_blocksize,
                                uint8_t *absmax_q, float *absmax2, float *offset,
                                void *workspace, int64_t workspace_bytes, void *stream);
 
@@ -136,13 +142,13 @@ nf4_status nf4_double_quantize(const float *absmax, int64_t nblocks, int dq_bloc
  *   n          even, >= 0; blocksize 64; dq_blocksize 256
  *   out        device, n elements of out_dtype (output)
  * One kernel launch. */
-nf4_status nf4_dequantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2,
+NF4_API nf4_status nf4_dequantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2,
                           const float *offset, int64_t n, int blocksize, int dq_blocksize,
                           void *out, nf4_dtype out_dtype, void *stream);
 
 /* Bytes of device workspace nf4_lora_linear_fwd needs for M rows of x and
  * rank r (0 when r == 0). */
-int64_t nf4_lora_linear_workspace_size(int64_t M, int r);
+NF4_API int64_t nf4_lora_linear_workspace_size(int64_t M, int r);
 
 /* nf4_lora_linear_fwd -- the frozen-base LoRA linear of [MF] "Forward Pass
  * Computation", Y = X dequant(c1, c2, W) + (alpha/r)(X L1) L2, in weight
@@ -163,7 +169,7 @@ int64_t nf4_lora_linear_workspace_size(int64_t M, int r);
  *              nf4_lora_linear_workspace_size(M, r); NULL allowed when r == 0
  * M <= 16 runs the streaming GEMV kernel, larger M the tensor-core GEMM
  * kernel; the LoRA pre-step is one extra launch when r > 0. */
-nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N,
+NF4_API nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N,
                                const uint8_t *packed, const uint8_t *absmax_q,
                                const float *absmax2, const float *offset,
                                const void *A, const void *B, int r, float scaling,
@@ -173,7 +179,7 @@ nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N,
  * library's device error word on the current device.  Returns
  * NF4_ERR_TIMEOUT if a bounded wait in a kernel expired since the last call,
  * NF4_ERR_CUDA on a CUDA error, NF4_OK otherwise. */
-nf4_status nf4_device_status(void *stream);
+NF4_API nf4_status nf4_device_status(void *stream);
 
 #ifdef __cplusplus
 }

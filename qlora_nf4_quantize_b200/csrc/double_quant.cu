@@ -1,0 +1,199 @@
+// double_quant.cu -- K2: double quantization of the fp32 block constants.
+//
+// "QLoRA: Mathematical Foundations ..." (llms.blog), section "Double
+// Quantization (DQ)": the first-level constants are grouped in runs of 256,
+// each run gets c2 = max |.| and every constant is stored as an 8-bit float
+// code of (constant / c2).  Readings (see nf4.h): E4M3 round-to-nearest-even;
+// with centring a per-tensor mean mu is subtracted first,
+//   mu = RN_f32( RN_f64( S / nblocks ) ),
+// S = fixed-order fp64 sum: each run summed sequentially in index order, then
+// the run sums combined pairwise level by level, an odd last element carried
+// up unchanged.
+//
+// Kernels
+//   k_dq_chunk_sums  one warp per run: the run's fp64 sum, then one CTA
+//                    combines 32 consecutive run sums (a level-5 node of the
+//                    pairwise tree) into the workspace.
+//   k_dq_quantize    every CTA rebuilds mu from the chunk sums (the same
+//                    tree, continued); then one warp per run computes c2 and
+//                    the E4M3 codes.
+// The pairwise tree restricted to an aligned group of 2^L leaves is the
+// perfect tree of that group, and the last partial group follows the same
+// level-by-level rule on its own leaves, so splitting the tree at level 5
+// reproduces the single-pass order exactly.
+//
+// Run sums in parallel: the sequential fp64 sum of one run equals its exact
+// sum whenever every partial sum is representable.  The constants are >= 0
+// and multiples of 2^(emin - 150) (emin = smallest biased exponent among the
+// non-zero ones, 1 for subnormals), and the total is below
+// 256 * 2^(emax - 126); if emax - emin <= 21 every subset sum is exact in
+// fp64, so any summation order gives the sequential result.  Otherwise lane 0
+// sums the run sequentially.
+#include "nf4_device.cuh"
+
+namespace nf4 {
+namespace {
+
+constexpr int kRunsPerChunk = 32;
+
+__device__ __forceinline__ int biased_exp(float v) {
+    int e = (int)((__float_as_uint(v) >> 23) & 0xFF);
+    return e == 0 ? 1 : e;
+}
+
+__global__ void __launch_bounds__(1024) k_dq_chunk_sums(const float *__restrict__ c1, int64_t nb,
+                                                         double *__restrict__ chunk_sums) {
+    __shared__ double s_run[kRunsPerChunk];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
+    const int64_t d = (int64_t)blockIdx.x * kRunsPerChunk + warp;
+    if (d < nd) {
+        const int64_t lo = d * kDqBlock;
+        const int64_t cnt = (nb - lo) < kDqBlock ? (nb - lo) : kDqBlock;
+        double sum = 0.0;
+        int emin = 255, emax = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            int64_t k = lane + 32 * i;
+            if (k < cnt) {
+                float v = __ldg(c1 + lo + k);
+                sum += (double)v;
+                if (v != 0.0f) {
+                    int e = biased_exp(v);
+                    emin = min(emin, e);
+                    emax = max(emax, e);
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+            emin = min(emin, __shfl_xor_sync(0xFFFFFFFFu, emin, o));
+            emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
+        }
+        if (emax != 0 && emax - emin > 21) {  // rare: reproduce the sequential order
+            if (lane == 0) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < cnt; ++k) acc += (double)c1[lo + k];
+                sum = acc;
+            }
+        }
+        if (lane == 0) s_run[warp] = sum;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int64_t len = nd - (int64_t)blockIdx.x * kRunsPerChunk;
+        if (len > kRunsPerChunk) len = kRunsPerChunk;
+        while (len > 1) {
+            int64_t half = len >> 1;
+            for (int64_t j = 0; j < half; ++j) s_run[j] = s_run[2 * j] + s_run[2 * j + 1];
+            if (len & 1) s_run[half] = s_run[len - 1];
+            len = half + (len & 1);
+        }
+        chunk_sums[blockIdx.x] = s_run[0];
+    }
+}
+
+// Level-by-level pairwise combination of s[0..len) in shared memory (two
+// buffers, so no element is overwritten while another thread still reads it).
+__device__ double tree_reduce(double *a, double *b, int64_t len) {
+    while (len > 1) {
+        const int64_t half = len >> 1;
+        for (int64_t j = threadIdx.x; j < half; j += blockDim.x) b[j] = a[2 * j] + a[2 * j + 1];
+        if ((len & 1) && threadIdx.x == 0) b[half] = a[len - 1];
+        __syncthreads();
+        double *t = a; a = b; b = t;
+        len = half + (len & 1);
+    }
+    return a[0];
+}
+
+__global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c1, int64_t nb,
+                                                      const double *__restrict__ chunk_sums, int64_t nchunks,
+                                                      uint8_t *__restrict__ codes, float *__restrict__ absmax2,
+                                                      float *__restrict__ offset) {
+    extern __shared__ double s_tree[];  // 2 * nchunks doubles when centring
+    __shared__ float s_mu;
+    if (offset != nullptr) {
+        for (int64_t j = threadIdx.x; j < nchunks; j += blockDim.x) s_tree[j] = chunk_sums[j];
+        __syncthreads();
+        double S = tree_reduce(s_tree, s_tree + nchunks, nchunks);
+        if (threadIdx.x == 0) {
+            float mu = (float)(S / (double)nb);
+            s_mu = mu;
+            if (blockIdx.x == 0) *offset = mu;
+        }
+    } else if (threadIdx.x == 0) {
+        s_mu = 0.0f;
+    }
+    __syncthreads();
+    const float mu = s_mu;
+
+    const int lane = threadIdx.x & 31;
+    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t d = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); d < nd; d += warps_total) {
+        const int64_t lo = d * kDqBlock;
+        const int64_t cnt = (nb - lo) < kDqBlock ? (nb - lo) : kDqBlock;
+        // lane owns constants lo + 8 lane .. lo + 8 lane + 7
+        float v[8];
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            int64_t k = 8 * lane + i;
+            v[i] = (k < cnt) ? __fsub_rn(__ldg(c1 + lo + k), mu) : 0.0f;
+            m = fmaxf(m, fabsf(v[i]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        const float c2 = m;
+        uint8_t q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = (c2 == 0.0f) ? (uint8_t)0 : f32_to_e4m3(__fdiv_rn(v[i], c2));
+        if (8 * lane + 8 <= cnt) {
+            uint2 pk;
+            pk.x = (uint32_t)q[0] | ((uint32_t)q[1] << 8) | ((uint32_t)q[2] << 16) | ((uint32_t)q[3] << 24);
+            pk.y = (uint32_t)q[4] | ((uint32_t)q[5] << 8) | ((uint32_t)q[6] << 16) | ((uint32_t)q[7] << 24);
+            *reinterpret_cast<uint2 *>(codes + lo + 8 * lane) = pk;
+        } else {
+            for (int i = 0; i < 8; ++i)
+                if (8 * lane + i < cnt) codes[lo + 8 * lane + i] = q[i];
+        }
+        if (lane == 0) absmax2[d] = c2;
+    }
+}
+
+}  // namespace
+
+int64_t dq_chunk_count(int64_t nblocks) {
+    int64_t nd = (nblocks + kDqBlock - 1) / kDqBlock;
+    return (nd + kRunsPerChunk - 1) / kRunsPerChunk;
+}
+
+// Largest chunk count whose tree fits in shared memory (2 buffers of doubles).
+int64_t dq_max_chunks() { return (200 * 1024) / (2 * (int64_t)sizeof(double)); }
+
+cudaError_t launch_double_quantize(const float *absmax, int64_t nb, uint8_t *codes, float *absmax2,
+                                   float *offset, double *chunk_sums, cudaStream_t stream, int num_sms) {
+    if (nb == 0) return cudaSuccess;
+    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
+    const int64_t nchunks = dq_chunk_count(nb);
+    size_t smem = 0;
+    if (offset != nullptr) {
+        k_dq_chunk_sums<<<(unsigned)nchunks, 1024, 0, stream>>>(absmax, nb, chunk_sums);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        smem = (size_t)(2 * nchunks) * sizeof(double);
+        if (smem > 48 * 1024) {
+            e = cudaFuncSetAttribute(k_dq_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+    }
+    int64_t want = (nd + 7) / 8;
+    int64_t cap = (int64_t)num_sms * 4;
+    int grid = (int)(want < cap ? want : cap);
+    k_dq_quantize<<<grid, 256, smem, stream>>>(absmax, nb, chunk_sums, nchunks, codes, absmax2, offset);
+    return cudaGetLastError();
+}
+
+}  // namespace nf4

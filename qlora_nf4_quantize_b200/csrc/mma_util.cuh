@@ -1,0 +1,57 @@
+// mma_util.cuh -- warp-level bf16 MMA and the NF4 register lookup table.
+#pragma once
+
+#include "nf4_device.cuh"
+
+namespace nf4 {
+
+// D = A * B + D for one m16n8k16 bf16 tile with fp32 accumulators.
+// a: 4 registers (bf16x2) of the 16x16 row-major A fragment, b: 2 registers
+// of the 16x8 column-major B fragment, d: 4 fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Per-block lookup table of the 16 dequantized bf16 weights
+//   e_i = RNE_bf16( RN_f32( q_i * c ) ),  i = 0..15,
+// held as byte planes: L0..L3 carry the low bytes of e_0..e_15 (four per
+// register), H0..H3 the high bytes.  Built once per 64-block from its
+// reconstructed constant c (16 binary32 multiplies, 8 bf16x2 conversions,
+// 8 byte permutes).
+struct Lut {
+    uint32_t L0, L1, L2, L3, H0, H1, H2, H3;
+};
+
+__device__ __forceinline__ Lut make_lut(float c) {
+    uint32_t P[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) P[j] = pack_bf16x2(__fmul_rn(c_levels[2 * j], c), __fmul_rn(c_levels[2 * j + 1], c));
+    Lut t;
+    t.L0 = __byte_perm(P[0], P[1], 0x6420); t.H0 = __byte_perm(P[0], P[1], 0x7531);
+    t.L1 = __byte_perm(P[2], P[3], 0x6420); t.H1 = __byte_perm(P[2], P[3], 0x7531);
+    t.L2 = __byte_perm(P[4], P[5], 0x6420); t.H2 = __byte_perm(P[4], P[5], 0x7531);
+    t.L3 = __byte_perm(P[6], P[7], 0x6420); t.H3 = __byte_perm(P[6], P[7], 0x7531);
+    return t;
+}
+
+// Look up four codes held in the low 16 bits of p16 (two packed bytes:
+// byte 0 = e0 << 4 | e1, byte 1 = e2 << 4 | e3, so the nibbles from bit 0 up
+// are e1, e0, e3, e2).  Returns the bf16 weights as two bf16x2 words:
+// lo01 = (e0 in the low half, e1 in the high half), lo23 = (e2, e3).
+// Each byte permute selects within 8 bytes, so codes 0-7 and 8-15 are looked
+// up separately and merged on bit 3 of each code.
+__device__ __forceinline__ void lut_lookup4(const Lut &t, uint32_t p16, uint32_t &w01, uint32_t &w23) {
+    const uint32_t s = p16 & 0x7777u;
+    const uint32_t s2 = ((p16 >> 1) & 0x4444u) | 0x3210u;
+    const uint32_t loA = __byte_perm(t.L0, t.L1, s), loB = __byte_perm(t.L2, t.L3, s);
+    const uint32_t hiA = __byte_perm(t.H0, t.H1, s), hiB = __byte_perm(t.H2, t.H3, s);
+    const uint32_t lo = __byte_perm(loA, loB, s2), hi = __byte_perm(hiA, hiB, s2);
+    w01 = __byte_perm(lo, hi, 0x4051);
+    w23 = __byte_perm(lo, hi, 0x6273);
+}
+
+}  // namespace nf4

@@ -1,0 +1,67 @@
+// nf4_device.cuh -- device-side definitions shared by the NF4 kernels.
+//
+// The NF4 table is the list printed on "QLoRA: Mathematical Foundations of
+// 4-Bit NormalFloat Quantization, Double Quantization, and Paged Optimizers"
+// (llms.blog), section "4-Bit NormalFloat (NF4): Information-Theoretic
+// Quantile Quantization"; every printed decimal is an exact binary32 value.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace nf4 {
+
+constexpr int kBlock = 64;      // first-level block ("B_1 = 64")
+constexpr int kDqBlock = 256;   // second-level block ("B_2 = 256")
+
+// Host copy (used to fill device tables and by nf4_codebook()).
+static const float kLevelsHost[16] = {
+    -1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
+    -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,
+    0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f, 0.33791524171829224f,
+    0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, 1.0f};
+
+// Device copy in constant memory (broadcast reads only; kernels that index it
+// per element first copy it to shared memory).
+static __constant__ float c_levels[16] = {
+    -1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
+    -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,
+    0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f, 0.33791524171829224f,
+    0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, 1.0f};
+
+// OCP FP8 E4M3 byte -> fp32 (exact: every E4M3 value is an fp16 value).
+__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
+    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+// fp32 -> E4M3, round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint8_t f32_to_e4m3(float y) {
+    return (uint8_t)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Reconstructed first-level constant of block b (see nf4_dequantize in nf4.h).
+//   kMode 0: double quantization with centring  c = fma(E4M3(q8), c2, mu)
+//   kMode 1: double quantization, no centring   c = E4M3(q8) * c2
+//   kMode 2: no double quantization            c = scales[b] (fp32 c1)
+template <int kMode>
+__device__ __forceinline__ float block_scale(const uint8_t *__restrict__ q8, const float *__restrict__ scales,
+                                             float mu, int64_t b) {
+    if constexpr (kMode == 2) {
+        return __ldg(scales + b);
+    } else {
+        float d = e4m3_to_f32(__ldg(q8 + b));
+        float c2 = __ldg(scales + (b >> 8));
+        if constexpr (kMode == 0) return __fmaf_rn(d, c2, mu);
+        else return __fmul_rn(d, c2);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+}  // namespace nf4

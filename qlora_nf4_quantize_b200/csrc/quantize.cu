@@ -1,0 +1,176 @@
+// quantize.cu -- K1: blockwise NF4 quantization.
+//
+// "QLoRA: Mathematical Foundations ..." (llms.blog), section "Block-Wise
+// Quantization Mechanics": c1 = max_j |w_j| over each contiguous block of 64,
+// code_j = arg-min_i |w_j / c1 - q_i|.  The quotient is the IEEE binary32
+// quotient; ties go to the lower index, i.e. code = #{i : x > t_i} with
+// t_i = RD_f32((q_i + q_{i+1}) / 2) (the exact midpoint rounded down).
+//
+// Layout of the work: one thread owns 8 consecutive elements, so the 8 lanes
+// l..l+7 (l a multiple of 8) of a warp own one 64-block; c1 is a 3-step
+// xor-shuffle max inside that lane group.  Each thread writes its 8 codes as
+// one 32-bit word (4 packed bytes), a warp 128 contiguous bytes.
+//
+// Division-free exact code selection: instead of the per-element IEEE
+// division, each element uses q = RN(w * RN(1 / c1)), which is within 2^-22
+// of x = RN(w / c1).  A 129-cell table indexed by round(64 q) gives the code
+// below the cell and the (at most one) threshold inside the cell widened by
+// 2^-18; code = base + (q > t).  When |q - t| <= 2^-18 the decision could
+// differ from the exact one and the element falls back to __fdiv_rn and a
+// full threshold count.  Each table word stores the threshold's bits with the
+// low 4 mantissa bits replaced by the base code (a perturbation below 2^-20,
+// covered by the 2^-18 margin).
+#include "nf4_device.cuh"
+
+namespace nf4 {
+namespace {
+
+constexpr float kAmbiguity = 0x1p-18f;
+constexpr int kCells = 129;
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ int exact_code(float w, float c1, const float *s_t) {
+    float x = __fdiv_rn(w, c1);
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < 15; ++i) c += (x > s_t[i]) ? 1 : 0;
+    return c;
+}
+
+// Fill the thresholds and the cell table in shared memory (once per CTA).
+__device__ void build_tables(float *s_t, uint32_t *s_cell) {
+    int tid = threadIdx.x;
+    if (tid < 15) {
+        double m = ((double)c_levels[tid] + (double)c_levels[tid + 1]) * 0.5;  // exact
+        s_t[tid] = __double2float_rd(m);
+    }
+    __syncthreads();
+    if (tid < kCells) {
+        // cell tid holds q with RN(64 q) = tid - 64, i.e. q in [lo, hi]
+        float lo = ((float)tid - 64.5f) * 0.015625f;
+        float hi = ((float)tid - 63.5f) * 0.015625f;
+        int base = 0;
+        uint32_t word = 0x40800000u;  // 4.0f: no threshold near this cell
+        for (int i = 0; i < 15; ++i) {
+            float t = s_t[i];
+            if (t < lo - kAmbiguity) ++base;
+            else if (t <= hi + kAmbiguity) word = __float_as_uint(t);
+        }
+        s_cell[tid] = (word & ~15u) | (uint32_t)base;
+    }
+    __syncthreads();
+}
+
+template <bool kBf16>
+__device__ __forceinline__ void load8(const void *w, int64_t e0, int64_t n, float v[8]) {
+    if (e0 + 8 <= n) {
+        if constexpr (kBf16) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(w) + e0));
+            uint32_t p[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                v[2 * i] = __uint_as_float(p[i] << 16);
+                v[2 * i + 1] = __uint_as_float(p[i] & 0xFFFF0000u);
+            }
+        } else {
+            const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(w) + e0);
+            float4 a = __ldg(src), b = __ldg(src + 1);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            int64_t e = e0 + i;
+            float x = 0.0f;
+            if (e < n) {
+                if constexpr (kBf16) {
+                    uint16_t h = __ldg(reinterpret_cast<const unsigned short *>(w) + e);
+                    x = __uint_as_float((uint32_t)h << 16);
+                } else {
+                    x = __ldg(static_cast<const float *>(w) + e);
+                }
+            }
+            v[i] = x;
+        }
+    }
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restrict__ w, int64_t n,
+                                                             uint8_t *__restrict__ packed,
+                                                             float *__restrict__ absmax) {
+    __shared__ float s_t[16];
+    __shared__ uint32_t s_cell[kCells + 3];
+    build_tables(s_t, s_cell);
+
+    const int lane = threadIdx.x & 31;
+    const int64_t ngroups = (n + 7) >> 3;
+    // the trip count depends only on blockIdx, so whole warps stay converged
+    for (int64_t base = (int64_t)blockIdx.x * kQuantThreads; base < ngroups;
+         base += (int64_t)gridDim.x * kQuantThreads) {
+        const int64_t g = base + threadIdx.x;
+        const int64_t e0 = g << 3;
+        float v[8];
+        load8<kBf16>(w, e0, n, v);
+
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 4));
+        const float c1 = a;
+        if (e0 >= n) continue;
+        if ((lane & 7) == 0) absmax[g >> 3] = c1;
+
+        int code[8];
+        if (c1 == 0.0f) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) code[i] = 7;
+        } else if (c1 < 0x1p-125f || c1 >= 0x1p125f) {
+            // c1 < 2^-125 or >= 2^125: 1/c1 may overflow or be subnormal, so
+            // the 2^-22 error bound of the fast path would not hold
+#pragma unroll
+            for (int i = 0; i < 8; ++i) code[i] = exact_code(v[i], c1, s_t);
+        } else {
+            const float rc = __frcp_rn(c1);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float q = __fmul_rn(v[i], rc);
+                float f = __fmaf_rn(q, 64.0f, 12582976.0f);  // 1.5 * 2^23 + 64: RN(64 q) + 64 in the low bits
+                // in [0, 128] for finite inputs; the clamp keeps a non-finite
+                // input from indexing outside the table
+                uint32_t e = s_cell[min(__float_as_uint(f) - 0x4B400000u, 128u)];
+                float t = __uint_as_float(e);
+                int c = (int)(e & 15u) + ((q > t) ? 1 : 0);
+                if (fabsf(q - t) <= kAmbiguity) c = exact_code(v[i], c1, s_t);
+                code[i] = c;
+            }
+        }
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) word |= (uint32_t)((code[2 * j] << 4) | code[2 * j + 1]) << (8 * j);
+        if (e0 + 8 <= n) {
+            reinterpret_cast<uint32_t *>(packed)[g] = word;
+        } else {
+            for (int j = 0; 2 * j < (int)(n - e0); ++j) packed[(e0 >> 1) + j] = (uint8_t)(word >> (8 * j));
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed, float *absmax,
+                            cudaStream_t stream, int num_sms) {
+    if (n == 0) return cudaSuccess;
+    int64_t ngroups = (n + 7) / 8;
+    int64_t want = (ngroups + kQuantThreads - 1) / kQuantThreads;
+    int64_t cap = (int64_t)num_sms * 8;
+    int grid = (int)(want < cap ? want : cap);
+    if (bf16) k_quantize<true><<<grid, kQuantThreads, 0, stream>>>(w, n, packed, absmax);
+    else k_quantize<false><<<grid, kQuantThreads, 0, stream>>>(w, n, packed, absmax);
+    return cudaGetLastError();
+}
+
+}  // namespace nf4

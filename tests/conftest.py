@@ -46,3 +46,40 @@ def read_golden_kv(name):
                 k, v = line.split("=")
                 out[k.strip()] = float(v)
     return out
+
+
+@pytest.fixture(scope="session")
+def nf4lib():
+    """The CUDA library, built in-tree for sm_100a (nvcc cross-compiles on a
+    machine without a GPU as well)."""
+    from qlora_nf4_quantize_b200 import build as b
+    b.build()
+    import qlora_nf4_quantize_b200 as q
+    q.lib()
+    return q
+
+
+@pytest.fixture(scope="session")
+def cuda_device():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("gpu test needs a CUDA device")
+    return torch.device("cuda:0")
+
+
+def rel_error_stats(y, ref):
+    """Max and mean relative error with the denominator floored at 1e-2 of
+    the reference's rms (so outputs near zero are judged on an absolute
+    scale), plus the Frobenius relative error."""
+    import numpy as np
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    den = np.maximum(np.abs(ref), 1e-2 * rms)
+    rel = np.abs(y - ref) / den
+    fro = float(np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300))
+    return float(rel.max()) if rel.size else 0.0, float(rel.mean()) if rel.size else 0.0, fro
+
+
+MATMUL_MAX_REL = 1e-2
+MATMUL_MEAN_REL = 2e-3

@@ -1,0 +1,75 @@
+"""GPU parity of nf4_lora_linear_fwd (the fused frozen-base LoRA linear)
+through the C ABI against the CPU oracle (fp64), within the matmul tolerance:
+max relative error <= 1e-2 and mean relative error < 2e-3, the denominator
+floored at 1e-2 of the reference's rms.  Special cases reduce to library
+routines: with no LoRA term the result equals torch.matmul on the bf16 output
+of nf4_dequantize."""
+import numpy as np
+import pytest
+import torch
+
+import nf4_workloads as wl
+from conftest import MATMUL_MAX_REL, MATMUL_MEAN_REL, rel_error_stats
+
+pytestmark = pytest.mark.gpu
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def quantize_on_gpu(q, W: torch.Tensor, dev, dq=True):
+    return q.quantize_weight(W.to(dev), double_quant=dq)
+
+
+def oracle_linear(oracle_mod, st, x, A, B, r, s, rows=None):
+    K = x.shape[1]
+    N = st.shape[0]
+    packed = st.packed.cpu().numpy()
+    scales = st.absmax2.cpu().numpy()
+    q8 = None if st.absmax_q is None else st.absmax_q.cpu().numpy()
+    mu = None if st.offset is None else np.float32(st.offset.cpu().numpy()[0])
+    return oracle_mod.lora_linear(u16(x), K, N, packed, q8, scales, mu,
+                                  None if A is None else u16(A), None if B is None else u16(B), r, s, rows=rows)
+
+
+def check(y: torch.Tensor, ref: np.ndarray):
+    mx, mean, fro = rel_error_stats(y.float().cpu().numpy(), ref)
+    assert mx <= MATMUL_MAX_REL and mean < MATMUL_MEAN_REL, (mx, mean, fro)
+    return mx, mean, fro
+
+
+@pytest.mark.parametrize("case", wl.GEMV_CASES, ids=lambda c: f"T{c.M}")
+def test_decode_gemv_full_size(nf4lib, oracle_mod, cuda_device, case):
+    W, x, A, B = wl.linear_inputs(case)
+    st = quantize_on_gpu(nf4lib, W, cuda_device)
+    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, case.N,
+                                   A.to(cuda_device), B.to(cuda_device), case.scaling)
+    torch.cuda.synchronize()
+    check(y, oracle_linear(oracle_mod, st, x, A, B, case.r, case.scaling))
+
+
+@pytest.mark.parametrize("M,K,N,r,dq", [(1, 192, 200, 16, True), (7, 64, 40, 32, True), (16, 320, 96, 64, False),
+                                        (9, 1024, 8, 16, True), (16, 4096, 1000, 0, True)])
+def test_gemv_ragged_shapes(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
+    c = wl.LinearCase("ragged", M, K, N, r, 1.5, 31 + M + K + N)
+    W, x, A, B = wl.linear_inputs(c, with_lora=r > 0)
+    st = quantize_on_gpu(nf4lib, W, cuda_device, dq)
+    dA = None if A is None else A.to(cuda_device)
+    dB = None if B is None else B.to(cuda_device)
+    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, N, dA, dB,
+                                   c.scaling)
+    torch.cuda.synchronize()
+    check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
+
+
+def test_gemv_without_lora_equals_matmul_on_dequantized(nf4lib, cuda_device):
+    c = wl.GEMV_CASES[2]
+    W, x, _, _ = wl.linear_inputs(c, with_lora=False)
+    st = quantize_on_gpu(nf4lib, W, cuda_device)
+    xd = x.to(cuda_device)
+    y = nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N)
+    wb = nf4lib.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N * c.K).view(c.N, c.K)
+    ref = torch.matmul(xd.float(), wb.float().t())
+    torch.cuda.synchronize()
+    check(y, ref.cpu().numpy())

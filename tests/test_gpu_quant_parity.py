@@ -1,0 +1,177 @@
+"""GPU parity: nf4_quantize, nf4_double_quantize and nf4_dequantize through the
+C ABI against the CPU oracle, bit-exact (codes, packed bytes, absmax, 8-bit
+scales, c2, mu, dequantized fp32 and bf16 values, signed zeros included)."""
+import numpy as np
+import pytest
+import torch
+
+import nf4_workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def f32bits(a) -> np.ndarray:
+    return np.ascontiguousarray(a, np.float32).view(np.uint32)
+
+
+def oracle_input(w_cpu: torch.Tensor) -> np.ndarray:
+    return u16(w_cpu).ravel() if w_cpu.dtype == torch.bfloat16 else w_cpu.contiguous().numpy().ravel()
+
+
+def run_round_trip(q, oracle_mod, w_cpu: torch.Tensor, centre=True):
+    dev = torch.device("cuda:0")
+    w = w_cpu.to(dev)
+    n = w.numel()
+    packed, absmax = q.nf4_quantize(w.reshape(-1))
+    q8, c2, off = q.nf4_double_quantize(absmax, centre=centre)
+    f32 = q.nf4_dequantize(packed, q8, c2, off, n, torch.float32)
+    b16 = q.nf4_dequantize(packed, q8, c2, off, n, torch.bfloat16)
+    nodq = q.nf4_dequantize(packed, None, absmax, None, n, torch.float32)
+    torch.cuda.synchronize()
+
+    op, oa = oracle_mod.quantize(oracle_input(w_cpu))
+    assert np.array_equal(packed.cpu().numpy(), op), "packed codes differ"
+    assert np.array_equal(f32bits(absmax.cpu().numpy()), f32bits(oa)), "absmax differs"
+    oq8, oc2, omu = oracle_mod.double_quantize(oa, centre=centre)
+    assert np.array_equal(q8.cpu().numpy(), oq8), "8-bit scale codes differ"
+    assert np.array_equal(f32bits(c2.cpu().numpy()), f32bits(oc2)), "c2 differs"
+    if centre:
+        assert f32bits(off.cpu().numpy())[0] == f32bits([omu])[0], "mean differs"
+    of = oracle_mod.dequantize(op, oq8, oc2, omu if centre else None, n, "f32")
+    ob = oracle_mod.dequantize(op, oq8, oc2, omu if centre else None, n, "bf16")
+    assert np.array_equal(f32bits(f32.cpu().numpy()), f32bits(of)), "fp32 dequant differs"
+    assert np.array_equal(u16(b16), ob), "bf16 dequant differs"
+    on = oracle_mod.dequantize(op, None, oa, None, n, "f32")
+    assert np.array_equal(f32bits(nodq.cpu().numpy()), f32bits(on)), "no-DQ dequant differs"
+
+
+def test_tiny_round_trip(nf4lib, oracle_mod, cuda_device):
+    run_round_trip(nf4lib, oracle_mod, wl.weight_case(wl.TINY))
+
+
+def test_projection_round_trip(nf4lib, oracle_mod, cuda_device):
+    run_round_trip(nf4lib, oracle_mod, wl.weight_case(wl.PROJECTION))
+
+
+def test_projection_without_centring(nf4lib, oracle_mod, cuda_device):
+    run_round_trip(nf4lib, oracle_mod, wl.weight_case(wl.PROJECTION), centre=False)
+
+
+@pytest.mark.parametrize("n", [2, 62, 64, 66, 130, 64 * 37 + 18, 16384 * 3 + 64 * 5 + 6])
+def test_ragged_sizes(nf4lib, oracle_mod, cuda_device, n):
+    w = wl.weight((n,), 0.02, 100 + n, "f32")
+    run_round_trip(nf4lib, oracle_mod, w)
+    run_round_trip(nf4lib, oracle_mod, w.to(torch.bfloat16))
+
+
+def test_empty_input(nf4lib, cuda_device):
+    w = torch.empty(0, device=cuda_device)
+    packed, absmax = nf4lib.nf4_quantize(w)
+    assert packed.numel() == 0 and absmax.numel() == 0
+
+
+def tie_and_edge_tensor(oracle_mod) -> torch.Tensor:
+    """Blocks built to hit exact ties, near-threshold quotients, zero and
+    signed-zero elements, subnormal and huge scales."""
+    q = oracle_mod.codebook().astype(np.float64)
+    mids = (q[:-1] + q[1:]) / 2
+    blocks = []
+    # ties: c1 = 1, elements exactly at representable midpoints
+    b = np.zeros(64, np.float32)
+    b[0] = 1.0
+    for i, m in enumerate(mids):
+        b[1 + i] = np.float32(m)
+        b[17 + i] = np.nextafter(np.float32(m), np.float32(2))
+        b[33 + i] = np.nextafter(np.float32(m), np.float32(-2))
+    b[48] = -0.0
+    blocks.append(b)
+    # the same with a non-power-of-two scale
+    blocks.append((b * np.float32(0.0371)).astype(np.float32))
+    # all zeros / negative zeros
+    blocks.append(np.full(64, -0.0, np.float32))
+    # subnormal-scale block and huge-scale block
+    rng = np.random.default_rng(9)
+    blocks.append((rng.standard_normal(64) * 1e-41).astype(np.float32))
+    blocks.append((rng.standard_normal(64) * 1e37).astype(np.float32))
+    blocks.append((rng.standard_normal(64) * 2.0 ** -126).astype(np.float32))
+    # quotients a few ulps either side of every threshold, for several scales
+    for c in (1.0, 0.7, 3.3e-3, 1.7e5):
+        b = np.zeros(64, np.float32)
+        b[0] = np.float32(c)
+        k = 1
+        for m in mids[:12]:
+            t = np.float32(m * c)
+            for d in (-2, 0, 2):
+                v = t
+                for _ in range(abs(d)):
+                    v = np.nextafter(v, np.float32(np.sign(d) * np.inf))
+                if k < 64:
+                    b[k] = v
+                    k += 1
+        blocks.append(b)
+    mixed = wl.random_bits_f32(64 * 40, 12).numpy()
+    return torch.from_numpy(np.concatenate(blocks + [mixed]).astype(np.float32))
+
+
+def test_ties_and_edge_values(nf4lib, oracle_mod, cuda_device):
+    w = tie_and_edge_tensor(oracle_mod)
+    dev = cuda_device
+    packed, absmax = nf4lib.nf4_quantize(w.to(dev))
+    op, oa = oracle_mod.quantize(w.numpy())
+    assert np.array_equal(packed.cpu().numpy(), op)
+    assert np.array_equal(f32bits(absmax.cpu().numpy()), f32bits(oa))
+    # dequantize without DQ: exact including signed zeros
+    out = nf4lib.nf4_dequantize(packed, None, absmax, None, w.numel(), torch.float32)
+    ref = oracle_mod.dequantize(op, None, oa, None, w.numel(), "f32")
+    assert np.array_equal(f32bits(out.cpu().numpy()), f32bits(ref))
+
+
+def test_dq_sequential_fallback_and_zero_runs(nf4lib, oracle_mod, cuda_device):
+    """Runs whose constants span more than 2^21 in magnitude take the
+    sequential fp64 sum; runs of equal constants give c2 = 0."""
+    rng = np.random.default_rng(13)
+    c1 = rng.uniform(0.01, 0.1, 256 * 70 + 17).astype(np.float32)
+    c1[256 * 3: 256 * 4] = (rng.uniform(0, 1, 256) * 2.0 ** rng.integers(-60, 0, 256)).astype(np.float32)
+    c1[256 * 5: 256 * 6] = np.float32(1e-40)
+    c1[256 * 7] = np.float32(3e30)
+    c1[256 * 9: 256 * 10] = 0.0
+    dev = cuda_device
+    for centre in (True, False):
+        q8, c2, off = nf4lib.nf4_double_quantize(torch.from_numpy(c1).to(dev), centre=centre)
+        oq8, oc2, omu = oracle_mod.double_quantize(c1, centre=centre)
+        assert np.array_equal(q8.cpu().numpy(), oq8)
+        assert np.array_equal(f32bits(c2.cpu().numpy()), f32bits(oc2))
+        if centre:
+            assert f32bits(off.cpu().numpy())[0] == f32bits([omu])[0]
+    # every constant equal to the mean: c2 = 0 and code 0
+    c1 = np.full(1000, 0.0625, np.float32)
+    q8, c2, off = nf4lib.nf4_double_quantize(torch.from_numpy(c1).to(dev))
+    assert float(off.item()) == 0.0625 and torch.all(c2 == 0) and torch.all(q8 == 0)
+
+
+def test_many_chunks_mean(nf4lib, oracle_mod, cuda_device):
+    """More than one chunk of 32 runs, ragged last chunk (tree across chunks)."""
+    rng = np.random.default_rng(14)
+    c1 = (rng.standard_normal(256 * 1000 + 100) ** 2 * 0.01).astype(np.float32)
+    q8, c2, off = nf4lib.nf4_double_quantize(torch.from_numpy(c1).to(cuda_device))
+    oq8, oc2, omu = oracle_mod.double_quantize(c1)
+    assert f32bits(off.cpu().numpy())[0] == f32bits([omu])[0]
+    assert np.array_equal(q8.cpu().numpy(), oq8)
+    assert np.array_equal(f32bits(c2.cpu().numpy()), f32bits(oc2))
+
+
+def test_stream_ordering_on_side_stream(nf4lib, oracle_mod, cuda_device):
+    w = wl.weight((512, 512), 0.02, 21, "bf16")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        wd = w.to(cuda_device, non_blocking=False)
+        packed, absmax = nf4lib.nf4_quantize(wd.reshape(-1), stream=s)
+        out = nf4lib.nf4_dequantize(packed, None, absmax, None, w.numel(), torch.bfloat16, stream=s)
+    s.synchronize()
+    op, oa = oracle_mod.quantize(u16(w).ravel())
+    assert np.array_equal(packed.cpu().numpy(), op)
+    assert np.array_equal(u16(out), oracle_mod.dequantize(op, None, oa, None, w.numel(), "bf16"))
