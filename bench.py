@@ -1,0 +1,410 @@
+"""Benchmark of the NF4 hot path on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path on per-GPU synthetic inputs:
+  1. nf4_quantize        projection weight 4096x4096 bf16 (0.1% x10 outliers)
+  2. nf4_double_quantize its 262,144 block constants (E4M3, centred)
+  3. nf4_dequantize      back to bf16
+  4. nf4_lora_linear_fwd decode GEMV: x[16, 4096], W 11008x4096, r=16, s=2
+  5. nf4_lora_linear_fwd training GEMM: x[4096, 4096], W 14336x4096, r=64, s=0.25
+Inputs are resident in HBM before timing; every buffer of steps 1-4 rotates
+between two copies and one step touches ~0.27 GB, more than the 126 MB L2, so
+no timed call reads its inputs from a warm L2.  Each call is bracketed by CUDA
+events on the launching stream; the JSON line reports the headline metric
+(NF4 dequant GB/s, the call of step 3), the tensor-core GEMM (the kernel that
+dominates the step) against the tensor roofline, and every call's own rate.
+
+With N > 1 (torchrun) every rank runs the same per-GPU workload on its own
+data (independent problems, no data-path collective: weak scaling); times are
+the maximum over ranks.  --impl reference times the CPU oracle (the method's
+plain C restatement) on the same workload and metric on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NF4 dequant GB/s; fused NF4+LoRA linear TFLOP/s; % of HBM/tensor roofline"
+BLOCK, DQ_BLOCK = 64, 256
+BYTES_PER_PARAM_DQ = 0.5 + 1 / 64 + 4 / 16384
+WORKLOAD = ("projection 4096x4096 bf16 (0.1% x10 outliers): quantize + double-quantize + dequantize(bf16); "
+            "decode GEMV x[16,4096] W 11008x4096 r=16; training GEMM x[4096,4096] W 14336x4096 r=64")
+
+
+# ------------------------------------------------------------------ algorithmic work per call
+def quantize_bytes(n):   # read bf16 weight, write codes and fp32 absmax
+    return n * 2 + n // 2 + (n // BLOCK) * 4
+
+
+def dq_bytes(nb):        # read fp32 constants, write 8-bit codes, c2 and the mean
+    return nb * 4 + nb + -(-nb // DQ_BLOCK) * 4 + 4
+
+
+def dequant_bytes(n, out_bytes=2):  # read the quantized state once, write the weight
+    nb = -(-n // BLOCK)
+    return n // 2 + nb + -(-nb // DQ_BLOCK) * 4 + 4 + n * out_bytes
+
+
+def linear_bytes(M, K, N, r):
+    n = N * K
+    nb = n // BLOCK
+    return n // 2 + nb + -(-nb // DQ_BLOCK) * 4 + 4 + M * K * 2 + r * K * 2 + N * r * 2 + M * N * 2
+
+
+def linear_flops(M, K, N, r):
+    return 2 * M * N * K + 2 * M * r * (K + N)
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def dist_init(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(values, world, device=None):
+    """Element-wise maximum of a list of floats over all ranks."""
+    import torch
+    if world == 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def rank_seed(base, rank):
+    """Each rank draws its own independent problem."""
+    return base + 100_003 * rank
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"nf4_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "50"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": float(np.median(loaded)) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def recorded_traffic(kernel_file):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, "qlora_nf4_quantize_b200", "csrc", kernel_file), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+        e = rec.get(kernel_file)
+        if e and e.get("source_sha256_16") == digest:
+            return e.get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    import nf4_workloads as wl
+    import qlora_nf4_quantize_b200 as q
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = dist_init(world, "nccl")
+    q.lib()  # fails loudly if the CUDA library is missing
+
+    # -------- inputs (generated on the CPU, then resident in HBM)
+    wp = wl.weight((4096, 4096), 0.02, rank_seed(wl.PROJECTION["seed"], rank), "bf16", outliers=True)
+    n = wp.numel()
+    nb = n // BLOCK
+    W2 = [wp.to(dev).reshape(-1), wp.to(dev).reshape(-1)]
+    packed2 = [torch.empty(n // 2, dtype=torch.uint8, device=dev) for _ in range(2)]
+    absmax2 = [torch.empty(nb, dtype=torch.float32, device=dev) for _ in range(2)]
+    q8 = [torch.empty(nb, dtype=torch.uint8, device=dev) for _ in range(2)]
+    c2 = [torch.empty(-(-nb // DQ_BLOCK), dtype=torch.float32, device=dev) for _ in range(2)]
+    mu = [torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2)]
+    dq_ws = torch.empty(q.nf4_double_quantize_workspace_size(nb), dtype=torch.uint8, device=dev)
+    deq = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+
+    c3 = wl.GEMV_CASES[2]
+    c3 = wl.LinearCase(c3.name, c3.M, c3.K, c3.N, c3.r, c3.scaling, rank_seed(c3.seed, rank))
+    W3, x3, A3, B3 = wl.linear_inputs(c3)
+    st3 = [q.quantize_weight(W3.to(dev)) for _ in range(2)]
+    x3d = [x3.to(dev), x3.to(dev)]
+    A3d, B3d = A3.to(dev), B3.to(dev)
+    y3 = [torch.empty(c3.M, c3.N, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    ws3 = torch.empty(q.nf4_lora_linear_workspace_size(c3.M, c3.r), dtype=torch.uint8, device=dev)
+
+    c4 = wl.GEMM_TRAIN
+    c4 = wl.LinearCase(c4.name, c4.M, c4.K, c4.N, c4.r, c4.scaling, rank_seed(c4.seed, rank))
+    W4, x4, A4, B4 = wl.linear_inputs(c4)
+    st4 = q.quantize_weight(W4.to(dev))
+    del W4
+    x4d, A4d, B4d = x4.to(dev), A4.to(dev), B4.to(dev)
+    y4 = torch.empty(c4.M, c4.N, dtype=torch.bfloat16, device=dev)
+    ws4 = torch.empty(q.nf4_lora_linear_workspace_size(c4.M, c4.r), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    calls = ["quantize", "double_quantize", "dequantize", "gemv_T16", "gemm_M4096"]
+    launches_per_step = 1 + 2 + 1 + 2 + 2
+
+    def step(i, ev=None):
+        k = i & 1
+        def mark(j):
+            if ev is not None:
+                ev[j].record()
+        mark(0)
+        q.nf4_quantize(W2[k], packed=packed2[k], absmax=absmax2[k])
+        mark(1)
+        q.nf4_double_quantize(absmax2[k], absmax_q=q8[k], absmax2=c2[k], offset=mu[k], workspace=dq_ws)
+        mark(2)
+        q.nf4_dequantize(packed2[k], q8[k], c2[k], mu[k], n, torch.bfloat16, out=deq[k])
+        mark(3)
+        s3 = st3[k]
+        q.nf4_lora_linear_fwd(x3d[k], s3.packed, s3.absmax_q, s3.absmax2, s3.offset, c3.N, A3d, B3d, c3.scaling,
+                              y=y3[k], workspace=ws3)
+        mark(4)
+        q.nf4_lora_linear_fwd(x4d, st4.packed, st4.absmax_q, st4.absmax2, st4.offset, c4.N, A4d, B4d, c4.scaling,
+                              y=y4, workspace=ws4)
+        mark(5)
+
+    for i in range(args.warmup):
+        step(i)
+    q.nf4_device_status()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record()
+    for i in range(args.steps):
+        step(i, events[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    q.nf4_device_status()
+
+    total_ms = t_start.elapsed_time(t_end)
+    per_call_ms = [sum(events[i][j].elapsed_time(events[i][j + 1]) for i in range(args.steps)) for j in range(5)]
+    red = reduce_max([total_ms] + per_call_ms, world, dev)
+    total_ms, per_call_ms = red[0], red[1:]
+    K = args.steps
+
+    # -------- end to end through host buffers (rank-local dequant call)
+    st_host = [packed2[0].cpu().pin_memory(), q8[0].cpu().pin_memory(), c2[0].cpu().pin_memory(),
+               mu[0].cpu().pin_memory()]
+    out_host = torch.empty(n, dtype=torch.bfloat16).pin_memory()
+    dev_in = [torch.empty_like(t, device=dev) for t in st_host]
+    e2e_iters = max(10, min(K, 100))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for it in range(e2e_iters + 3):
+        if it == 3:
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            e0.record()
+        for d, h in zip(dev_in, st_host):
+            d.copy_(h, non_blocking=True)
+        q.nf4_dequantize(dev_in[0], dev_in[1], dev_in[2], dev_in[3], n, torch.bfloat16, out=deq[0])
+        out_host.copy_(deq[0], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max([e0.elapsed_time(e1) / e2e_iters], world, dev)[0]
+    h2d = sum(t.numel() * t.element_size() for t in st_host)
+    d2h = out_host.numel() * 2
+
+    peaks = measured_peaks()
+    deq_b = dequant_bytes(n)
+    value = world * K * deq_b / (per_call_ms[2] * 1e-3) / 1e9
+    gemm_flops = linear_flops(c4.M, c4.K, c4.N, c4.r)
+    gemm_tflops = gemm_flops / (per_call_ms[4] / K * 1e-3) / 1e12
+    kernels = []
+    algo = [("quantize", quantize_bytes(n), "GB/s"), ("double_quantize", dq_bytes(nb), "GB/s"),
+            ("dequantize", deq_b, "GB/s"), ("gemv_T16", linear_bytes(c3.M, c3.K, c3.N, c3.r), "GB/s"),
+            ("gemm_M4096", gemm_flops, "TFLOP/s")]
+    for j, (name, work, unit) in enumerate(algo):
+        us = per_call_ms[j] / K * 1e3
+        if unit == "GB/s":
+            ach = work / (us * 1e-6) / 1e9
+            peak = peaks["hbm_gbs"]
+        else:
+            ach = work / (us * 1e-6) / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+        kernels.append({"call": name, "us": round(us, 3), "achieved": round(ach, 2), "unit": unit,
+                        "peak": peak, "frac": round(ach / peak, 4), "work_per_call": work})
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "quant": "NF4 block 64 + double quant block 256 (E4M3, centred)",
+                   "arith": "quantize/dequantize fp32 -> bf16; linear bf16 x bf16 tensor cores, fp32 accumulate",
+                   "l2": "inputs rotate over 2 copies, 0.27 GB touched per step (> 126 MB L2)",
+                   "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_tc (nf4_lora_linear_fwd, M=4096)",
+                     "achieved": round(gemm_tflops, 2), "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / peaks["bf16_tflops_sustained"], 4),
+                     "traffic": recorded_traffic("gemm_tc.cu"),
+                     "peak_source": peaks["source"] + " bf16 sustained (kernel timed inside a long step)"},
+        "kernels": kernels,
+        "e2e": {"value": round(world * deq_b / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "call": "nf4_dequantize with pinned host inputs and output"},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wp)
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_dequant_rate(wp, budget_s):
+    """The oracle's NF4 dequant (bf16 output) on the projection weight,
+    repeated for about budget_s seconds; returns (GB/s, repetitions)."""
+    import torch
+    import oracle
+    bits = wp.contiguous().view(torch.int16).numpy().view(np.uint16).ravel()
+    packed, c1 = oracle.quantize(bits)
+    codes, c2, mu = oracle.double_quantize(c1)
+    n = bits.size
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.dequantize(packed, codes, c2, mu, n, "bf16")
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return reps * dequant_bytes(n) / el / 1e9, reps, el
+
+
+def cpu_baseline(wp, budget_s=10.0):
+    gbs, reps, el = oracle_dequant_rate(wp, budget_s)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"oracle nf4 dequantize (bf16 out) of the full 4096x4096 projection weight, {reps} passes "
+                      f"in {el:.1f} s, single thread"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import nf4_workloads as wl
+    wp = wl.weight((4096, 4096), 0.02, wl.PROJECTION["seed"], "bf16", outliers=True)
+    for _ in range(args.warmup):
+        oracle_dequant_rate(wp, 0.0)
+    t0 = time.perf_counter()
+    gbs = []
+    for _ in range(args.steps):
+        g, _, _ = oracle_dequant_rate(wp, 0.0)
+        gbs.append(g)
+    el = time.perf_counter() - t0
+    n = wp.numel()
+    value = args.steps * dequant_bytes(n) / el / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "projection 4096x4096 bf16 (0.1% x10 outliers): NF4 dequantize (bf16 out), "
+                                   "CPU oracle (plain C, single thread)", "parallelism": "rank 0 only"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} full dequantize passes of the projection weight"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    run_ours(args)
+    rank, world, _ = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

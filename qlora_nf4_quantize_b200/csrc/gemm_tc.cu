@@ -1,13 +1,431 @@
-// gemm_tc.cu -- K5: fused NF4-dequantizing tensor-core GEMM (tcgen05) for
-// large token counts.  (Implementation in progress.)
-#include "nf4_device.cuh"
+// gemm_tc.cu -- K5: fused NF4-dequantizing tensor-core GEMM for large token
+// counts (tcgen05 / TMEM / TMA, sm_100a).
+//
+//   y[M, N] = x[M, K] W~[N, K]^T + [t_hi | t_lo | 0][M, RP] [B | B | 0][N, RP]^T
+//
+// "QLoRA: Mathematical Foundations ...", section "Forward Pass Computation":
+// the NF4 weight is dequantized on the fly into on-chip tiles and never
+// written to global memory; bf16 operands, fp32 accumulation, bf16 output.
+// W~ is bit-identical to the bf16 output of nf4_dequantize.
+//
+// One CTA computes a 128 (weight rows) x 256 (tokens) tile of y^T:
+//   MMA  D[n, m] += A[n, k] * X[m, k],   M_mma = 128, N_mma = 256, K = 16
+//   A = W~ (bf16) lives in tensor memory: two dequant warpgroups turn the
+//       packed nibbles of a 64-wide k-step into bf16 in registers (one scale
+//       and one register lookup table per 64-block per thread, see
+//       mma_util.cuh) and store them with tcgen05.st; no shared memory is
+//       used for the weight.
+//   X = x tile (256 tokens x 64 k, bf16) brought in by TMA with 128-byte
+//       swizzle into a 4-stage shared-memory ring.
+//   D = fp32 accumulators in tensor memory (256 columns).
+// After the K/64 weight steps the same pipeline runs RP/64 extension steps in
+// which the warpgroups copy rows of [B | B | 0] into tensor memory and TMA
+// brings tiles of the [t_hi | t_lo | 0] workspace: the LoRA term is summed by
+// the same MMAs into the same accumulators.
+//
+// Warp roles (12 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
+// MMA issuer (one elected thread), warps 4..11 = two dequant warpgroups
+// (warpgroup h produces the k-steps with index = h mod 2) and, at the end,
+// the epilogue (tcgen05.ld, bf16 conversion, stores of y).
+//
+// Every mbarrier wait is bounded (about one second of %globaltimer): on
+// expiry the waiter raises a CTA-wide abort flag and the device error word,
+// every role leaves its loop, the MMA issuer drains its own MMAs, the TMA
+// producer drains its own loads, and tensor memory is released before the
+// CTA exits.  nf4_device_status() reports the expiry as NF4_ERR_TIMEOUT.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "mma_util.cuh"
 
 namespace nf4 {
+namespace {
 
-cudaError_t launch_gemm_tc(const void *, int64_t, int64_t, int64_t, const uint8_t *, const uint8_t *,
-                           const float *, const float *, const void *, int, const void *, int, void *,
-                           cudaStream_t, int, unsigned *) {
-    return cudaErrorNotSupported;
+constexpr int kBN = 128;                   // weight rows per CTA (MMA M)
+constexpr int kBT = 256;                   // tokens per CTA (MMA N)
+constexpr int kBK = 64;                    // k per pipeline step
+constexpr int kStages = 4;
+constexpr int kThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 0;            // accumulator: columns [0, 256)
+constexpr uint32_t kACol = 256;            // A stages: columns [256 + 32 s, +32)
+constexpr uint32_t kXStageBytes = kBT * kBK * 2;
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+
+// UMMA instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBT >> 3) << 17) |
+                            ((uint32_t)(kBN >> 4) << 24);
+
+struct __align__(1024) SmemLayout {
+    uint8_t x[kStages][kXStageBytes];
+    uint64_t x_full[kStages];
+    uint64_t x_empty[kStages];
+    uint64_t a_full[kStages];
+    uint64_t a_empty[kStages];
+    uint64_t acc_full;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: true when the phase completed; false after the time limit
+// (abort raised) or when another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicOr(err, 1u);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+            "r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand tile written by TMA with
+// 128-byte swizzle (rows of 128 bytes, 8-row groups 1024 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void *p) {
+    const uint64_t addr = smem_addr(p);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;          // start address
+    d |= (uint64_t)1 << 16;                // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;      // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                // descriptor version for tcgen05
+    d |= (uint64_t)2 << 61;                // SWIZZLE_128B
+    return d;
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_store32(uint32_t taddr, const uint32_t v[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_load32(uint32_t taddr, uint32_t v[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
+          "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+          "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 64 bf16 weights (one k-step) of weight row n as 32 bf16x2 words, word j =
+// (element 2j low half, element 2j+1 high half).
+template <int kMode>
+__device__ __forceinline__ void dequant_step(const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
+                                             const float *__restrict__ scales, float mu, int64_t n, int64_t K,
+                                             int64_t kt, bool valid, uint32_t out[32]) {
+    uint32_t w[8];
+    float c = 0.0f;
+    if (valid) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(packed + n * (K >> 1) + kt * 32);
+        const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
+        w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
+        w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
+        c = block_scale<kMode>(q8, scales, mu, n * (K >> 6) + kt);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = 0x77777777u;
+    }
+    const Lut lut = make_lut(c);
+#pragma unroll
+    for (int s = 0; s < 16; ++s) lut_lookup4(lut, w[s >> 1] >> ((s & 1) * 16), out[2 * s], out[2 * s + 1]);
+}
+
+// 64 columns [64 e, 64 e + 64) of the row n of [B | B | 0] (bf16 pairs).
+__device__ __forceinline__ void lora_step(const __nv_bfloat16 *__restrict__ Bl, int r, int64_t n, bool valid,
+                                          int e, uint32_t out[32]) {
+    const uint32_t *row = reinterpret_cast<const uint32_t *>(Bl + (valid ? n : 0) * r);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const int j = 64 * e + 2 * c;
+        out[c] = (valid && j < 2 * r) ? __ldg(row + ((j % r) >> 1)) : 0u;
+    }
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_t, int64_t M,
+              int64_t K, int64_t N, const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
+              const float *__restrict__ scales, const float *__restrict__ offset,
+              const __nv_bfloat16 *__restrict__ Bl, int r, int rp, __nv_bfloat16 *__restrict__ y, unsigned *err) {
+    extern __shared__ uint8_t smem_raw[];
+    SmemLayout &S = *reinterpret_cast<SmemLayout *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    volatile int *abort = &S.abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n0 = (int64_t)blockIdx.x * kBN;
+    const int64_t m0 = (int64_t)blockIdx.y * kBT;
+    const int kw_steps = (int)(K / kBK);
+    const int kt_total = kw_steps + (r > 0 ? rp / kBK : 0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&S.x_full[s], 1);
+            mbar_init(&S.x_empty[s], 1);
+            mbar_init(&S.a_full[s], 128);
+            mbar_init(&S.a_empty[s], 1);
+        }
+        mbar_init(&S.acc_full, 1);
+        mbar_init(&S.drain, 1);
+        S.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&S.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int kt = 0; kt < kt_total; ++kt) {
+                const int s = kt % kStages;
+                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                if (!mbar_wait(&S.x_empty[s], ph ^ 1u, abort, err)) break;
+                mbar_arrive_expect_tx(&S.x_full[s], kXStageBytes);
+                if (kt < kw_steps) tma_load_2d(S.x[s], &tmap_x, &S.x_full[s], kt * kBK, (int)m0);
+                else tma_load_2d(S.x[s], &tmap_t, &S.x_full[s], (kt - kw_steps) * kBK, (int)m0);
+                issued = kt + 1;
+            }
+            // drain: every issued load has landed before the CTA may exit
+            for (int kt = issued - kStages < 0 ? 0 : issued - kStages; kt < issued; ++kt) {
+                const int s = kt % kStages;
+                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                unsigned long long t0 = global_ns();
+                while (!mbar_try_wait(&S.x_full[s], ph) && global_ns() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            bool any = false;
+            for (int kt = 0; kt < kt_total; ++kt) {
+                const int s = kt % kStages;
+                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                if (!mbar_wait(&S.x_full[s], ph, abort, err)) break;
+                if (!mbar_wait(&S.a_full[s], ph, abort, err)) break;
+                tc_fence_after();
+                const uint64_t bdesc = smem_desc_sw128(S.x[s]);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    tc_mma_ts(tmem + kAccCol, tmem + kACol + 32u * s + 8u * kk, bdesc + 2ull * kk,
+                              (kt | kk) != 0 ? 1u : 0u);
+                }
+                any = true;
+                tc_commit(&S.x_empty[s]);
+                tc_commit(&S.a_empty[s]);
+                if (kt == kt_total - 1) tc_commit(&S.acc_full);
+            }
+            if (any && *abort) {  // drain our own MMAs before tensor memory is released
+                tc_commit(&S.drain);
+                unsigned long long t0 = global_ns();
+                while (!mbar_try_wait(&S.drain, 0) && global_ns() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else if (warp >= 4) {
+        // ---------------- dequant warpgroups, then epilogue ----------------
+        const int q = warp & 3;         // tensor-memory lane quarter
+        const int h = (warp - 4) >> 2;  // warpgroup: k-steps with index % 2 == h
+        const int row_in_tile = 32 * q + lane;
+        const int64_t n = n0 + row_in_tile;
+        const bool nvalid = n < N;
+        const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        bool ok = true;
+        for (int kt = h; kt < kt_total; kt += 2) {
+            const int s = kt % kStages;
+            const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+            uint32_t v[32];
+            if (kt < kw_steps) dequant_step<kMode>(packed, q8, scales, mu, n, K, kt, nvalid, v);
+            else lora_step(Bl, r, n, nvalid, kt - kw_steps, v);
+            // warp-uniform outcome: the tcgen05.st below is a warp-wide instruction
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.a_empty[s], ph ^ 1u, abort, err));
+            if (!ok) break;
+            tc_store32(lane_base + kACol + 32u * s, v);
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(&S.a_full[s]);
+        }
+        if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err));
+        if (ok) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                const uint32_t col = kAccCol + 128u * h + 32u * c;
+                tc_load32(lane_base + col, v);
+                tc_wait_ld();
+                const int64_t mb = m0 + 128 * h + 32 * c;
+                if (nvalid) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int64_t m = mb + i;
+                        if (m < M) y[m * N + n] = __float2bfloat16_rn(__uint_as_float(v[i]));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn(cudaError_t *st) {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn != nullptr) {
+        *st = cudaSuccess;
+        return fn;
+    }
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    *st = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (*st != cudaSuccess || q != cudaDriverEntryPointSuccess || p == nullptr) {
+        if (*st == cudaSuccess) *st = cudaErrorNotSupported;
+        return nullptr;
+    }
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] row-major; box = 64 columns x 256 rows,
+// 128-byte swizzle, out-of-range rows read as zero.
+cudaError_t make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols) {
+    cudaError_t st;
+    auto fn = get_encode_fn(&st);
+    if (fn == nullptr) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBT};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int kMode>
+cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, int64_t M, int64_t K, int64_t N,
+                        const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
+                        const __nv_bfloat16 *Bl, int r, int rp, __nv_bfloat16 *y, unsigned *err, cudaStream_t stream) {
+    const size_t smem = sizeof(SmemLayout) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBT - 1) / kBT));
+    k_gemm_tc<kMode><<<grid, kThreads, smem, stream>>>(mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, y, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
+                           const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
+                           void *y, cudaStream_t stream, int /*num_sms*/, unsigned *err_word) {
+    if (M > 0x7FFFFFFF || K > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    CUtensorMap mx, mt;
+    cudaError_t e = make_map(&mx, x, M, K);
+    if (e != cudaSuccess) return e;
+    if (r > 0) e = make_map(&mt, t2, M, rp);
+    else e = make_map(&mt, x, M, K);  // unused: no extension steps
+    if (e != cudaSuccess) return e;
+    auto *Bl = static_cast<const __nv_bfloat16 *>(B);
+    auto *yp = static_cast<__nv_bfloat16 *>(y);
+    if (q8 == nullptr) return launch_mode<2>(mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+    if (offset == nullptr) return launch_mode<1>(mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+    return launch_mode<0>(mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
 }
 
 }  // namespace nf4

@@ -73,3 +73,62 @@ def test_gemv_without_lora_equals_matmul_on_dequantized(nf4lib, cuda_device):
     ref = torch.matmul(xd.float(), wb.float().t())
     torch.cuda.synchronize()
     check(y, ref.cpu().numpy())
+
+
+# ---------------------------------------------------------------- tensor-core GEMM (M > 16)
+@pytest.mark.parametrize("M,K,N,r,dq", [(17, 64, 8, 0, True), (100, 192, 136, 16, True), (256, 256, 128, 64, True),
+                                        (300, 320, 264, 32, False), (513, 128, 256, 16, True)])
+def test_gemm_small_shapes_full_output(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
+    c = wl.LinearCase("gemm small", M, K, N, r, 0.75, 57 + M + K + N)
+    W, x, A, B = wl.linear_inputs(c, with_lora=r > 0)
+    st = quantize_on_gpu(nf4lib, W, cuda_device, dq)
+    dA = None if A is None else A.to(cuda_device)
+    dB = None if B is None else B.to(cuda_device)
+    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, N, dA, dB,
+                                   c.scaling)
+    nf4lib.nf4_device_status()
+    check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
+
+
+def sampled_rows(M, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(M, size=min(count, M), replace=False)).astype(np.int64)
+    return np.unique(np.concatenate([rows, [0, M - 1]])).astype(np.int64)
+
+
+@pytest.mark.parametrize("case,nrows", [(wl.GEMM_TRAIN, 192), (wl.GEMM_70B_MLP, 48)], ids=["train4096", "mlp70b"])
+def test_gemm_full_size_sampled_rows(nf4lib, oracle_mod, cuda_device, case, nrows):
+    W, x, A, B = wl.linear_inputs(case)
+    st = quantize_on_gpu(nf4lib, W, cuda_device)
+    del W
+    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, case.N,
+                                   A.to(cuda_device), B.to(cuda_device), case.scaling)
+    nf4lib.nf4_device_status()
+    rows = sampled_rows(case.M, nrows, case.seed)
+    ref = oracle_linear(oracle_mod, st, x, A, B, case.r, case.scaling, rows=rows)
+    check(y[torch.from_numpy(rows).to(cuda_device)], ref)
+
+
+def test_gemm_without_lora_equals_matmul_on_dequantized(nf4lib, cuda_device):
+    c = wl.LinearCase("gemm vs torch", 1024, 2048, 3072, 0, 1.0, 77)
+    W, x, _, _ = wl.linear_inputs(c, with_lora=False)
+    st = quantize_on_gpu(nf4lib, W, cuda_device)
+    xd = x.to(cuda_device)
+    y = nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N)
+    wb = nf4lib.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N * c.K).view(c.N, c.K)
+    ref = torch.matmul(xd.float(), wb.float().t())
+    nf4lib.nf4_device_status()
+    check(y, ref.cpu().numpy())
+
+
+def test_gemm_and_gemv_agree_on_shared_rows(nf4lib, cuda_device):
+    """T = 16 through the GEMV path equals the first 16 rows of a 64-row GEMM."""
+    c = wl.LinearCase("agree", 64, 1024, 512, 16, 2.0, 91)
+    W, x, A, B = wl.linear_inputs(c)
+    st = quantize_on_gpu(nf4lib, W, cuda_device)
+    xd, Ad, Bd = x.to(cuda_device), A.to(cuda_device), B.to(cuda_device)
+    y64 = nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, Ad, Bd, c.scaling)
+    y16 = nf4lib.nf4_lora_linear_fwd(xd[:16].contiguous(), st.packed, st.absmax_q, st.absmax2, st.offset, c.N, Ad, Bd,
+                                     c.scaling)
+    nf4lib.nf4_device_status()
+    check(y16, y64[:16].float().cpu().numpy())
