@@ -6,18 +6,38 @@
 // quantization state (nf4_device.cuh, block_scale).  bf16 output rounds the
 // binary32 value to nearest even.
 //
-// HBM-bound streaming kernel: a lane owns 8 consecutive elements per step
-// (4 packed bytes: one 32-bit load, a warp reads 128 contiguous bytes), looks
-// the 8 codes up in a 16-entry shared-memory copy of the table (16 distinct
-// words in 16 banks: conflict-free for any code pattern) and writes 32 bytes
-// (fp32) or 16 bytes (bf16) with 128-bit stores.  The 8 lanes that share a
-// 64-block read the same scale byte (one broadcast request).
+// HBM-bound streaming kernel.  A warp handles 2048 consecutive elements per
+// iteration as 8 segments of 256: in segment j lane l owns the 8 elements
+// starting at 256 j + 8 l, i.e. 4 packed bytes (one 32-bit load; the warp's
+// load is 128 contiguous bytes) and 16 output bytes for bf16 (one 128-bit
+// store; the warp's store is 512 contiguous bytes).  All 8 loads of a lane are
+// issued before any arithmetic, so each thread keeps 32 bytes in flight.
+// Codes are looked up in a 16-entry shared-memory copy of the table (16
+// distinct words in 16 banks: conflict-free for any code pattern).
 #include "nf4_device.cuh"
 
 namespace nf4 {
 namespace {
 
 constexpr int kDeqThreads = 256;
+constexpr int kSeg = 8;                  // segments per lane per iteration
+constexpr int kWarpElems = kSeg * 256;   // elements per warp per iteration
+
+template <int kMode, bool kBf16Out>
+__device__ __forceinline__ void store8(void *out, int64_t e0, const float v[8]) {
+    if constexpr (kBf16Out) {
+        uint4 o;
+        o.x = pack_bf16x2(v[0], v[1]);
+        o.y = pack_bf16x2(v[2], v[3]);
+        o.z = pack_bf16x2(v[4], v[5]);
+        o.w = pack_bf16x2(v[6], v[7]);
+        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + e0) = o;
+    } else {
+        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + e0);
+        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
 
 template <int kMode, bool kBf16Out>
 __global__ void __launch_bounds__(kDeqThreads) k_dequantize(const uint8_t *__restrict__ packed,
@@ -29,41 +49,39 @@ __global__ void __launch_bounds__(kDeqThreads) k_dequantize(const uint8_t *__res
     if (threadIdx.x < 16) s_q[threadIdx.x] = c_levels[threadIdx.x];
     __syncthreads();
     const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
-    const int64_t ngroups = (n + 7) >> 3;
-    for (int64_t g = (int64_t)blockIdx.x * kDeqThreads + threadIdx.x; g < ngroups;
-         g += (int64_t)gridDim.x * kDeqThreads) {
-        const int64_t e0 = g << 3;
-        const float c = block_scale<kMode>(q8, scales, mu, e0 >> 6);
-        if (e0 + 8 <= n) {
-            const uint32_t p = __ldg(reinterpret_cast<const uint32_t *>(packed) + g);
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (kDeqThreads / 32);
+    const int64_t nfull = n / kWarpElems;  // warp iterations with no tail
+    for (int64_t c = (int64_t)blockIdx.x * (kDeqThreads / 32) + (threadIdx.x >> 5); c < nfull; c += warps) {
+        const int64_t base = c * kWarpElems + 8 * lane;
+        uint32_t p[kSeg];
+        float sc[kSeg];
+#pragma unroll
+        for (int j = 0; j < kSeg; ++j) p[j] = __ldg(reinterpret_cast<const uint32_t *>(packed) + ((base + 256 * j) >> 3));
+#pragma unroll
+        for (int j = 0; j < kSeg; ++j) sc[j] = block_scale<kMode>(q8, scales, mu, (base + 256 * j) >> 6);
+#pragma unroll
+        for (int j = 0; j < kSeg; ++j) {
             float v[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t byte = (p >> (8 * j)) & 0xFFu;
-                v[2 * j] = __fmul_rn(s_q[byte >> 4], c);       // element 2j: high nibble
-                v[2 * j + 1] = __fmul_rn(s_q[byte & 15u], c);  // element 2j+1: low nibble
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t byte = (p[j] >> (8 * b)) & 0xFFu;
+                v[2 * b] = __fmul_rn(s_q[byte >> 4], sc[j]);       // element 2b: high nibble
+                v[2 * b + 1] = __fmul_rn(s_q[byte & 15u], sc[j]);  // element 2b+1: low nibble
             }
-            if constexpr (kBf16Out) {
-                uint4 o;
-                o.x = pack_bf16x2(v[0], v[1]);
-                o.y = pack_bf16x2(v[2], v[3]);
-                o.z = pack_bf16x2(v[4], v[5]);
-                o.w = pack_bf16x2(v[6], v[7]);
-                reinterpret_cast<uint4 *>(out)[g] = o;
-            } else {
-                float4 *dst = reinterpret_cast<float4 *>(out) + 2 * g;
-                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-            }
-        } else {
-            for (int64_t e = e0; e < n; ++e) {
-                const uint32_t byte = packed[e >> 1];
-                const uint32_t code = (e & 1) ? (byte & 15u) : (byte >> 4);
-                const float v = __fmul_rn(s_q[code], c);
-                if constexpr (kBf16Out) reinterpret_cast<__nv_bfloat16 *>(out)[e] = __float2bfloat16_rn(v);
-                else reinterpret_cast<float *>(out)[e] = v;
-            }
+            store8<kMode, kBf16Out>(out, base + 256 * j, v);
         }
+    }
+    // tail: elements [nfull * kWarpElems, n), one element per thread
+    const int64_t tail0 = nfull * kWarpElems;
+    for (int64_t e = tail0 + (int64_t)blockIdx.x * kDeqThreads + threadIdx.x; e < n;
+         e += (int64_t)gridDim.x * kDeqThreads) {
+        const float c1 = block_scale<kMode>(q8, scales, mu, e >> 6);
+        const uint32_t byte = packed[e >> 1];
+        const uint32_t code = (e & 1) ? (byte & 15u) : (byte >> 4);
+        const float v = __fmul_rn(s_q[code], c1);
+        if constexpr (kBf16Out) reinterpret_cast<__nv_bfloat16 *>(out)[e] = __float2bfloat16_rn(v);
+        else reinterpret_cast<float *>(out)[e] = v;
     }
 }
 
@@ -80,9 +98,9 @@ cudaError_t launch_mode(const uint8_t *packed, const uint8_t *q8, const float *s
 cudaError_t launch_dequantize(const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
                               int64_t n, void *out, bool bf16, cudaStream_t stream, int num_sms) {
     if (n == 0) return cudaSuccess;
-    int64_t ngroups = (n + 7) / 8;
-    int64_t want = (ngroups + kDeqThreads - 1) / kDeqThreads;
-    int64_t cap = (int64_t)num_sms * 8;
+    int64_t witers = (n + kWarpElems - 1) / kWarpElems;
+    int64_t want = (witers + (kDeqThreads / 32) - 1) / (kDeqThreads / 32);
+    int64_t cap = (int64_t)num_sms * 6;
     int grid = (int)(want < cap ? want : cap);
     if (q8 == nullptr) return launch_mode<2>(packed, q8, scales, offset, n, out, bf16, grid, stream);
     if (offset == nullptr) return launch_mode<1>(packed, q8, scales, offset, n, out, bf16, grid, stream);

@@ -268,6 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kt = 0; kt < kt_total; ++kt) {
                 const int s = kt % kStages;
                 const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+                // the t workspace is written by the down-projection kernel
+                // launched just before (programmatic dependent launch)
+                if (kt == kw_steps) asm volatile("griddepcontrol.wait;" ::: "memory");
                 if (!mbar_wait(&S.x_empty[s], ph ^ 1u, abort, err)) break;
                 mbar_arrive_expect_tx(&S.x_full[s], kXStageBytes);
                 if (kt < kw_steps) tma_load_2d(S.x[s], &tmap_x, &S.x_full[s], kt * kBK, (int)m0);
@@ -404,9 +407,17 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, int64_t M,
     const size_t smem = sizeof(SmemLayout) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBT - 1) / kBT));
-    k_gemm_tc<kMode><<<grid, kThreads, smem, stream>>>(mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, y, err);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBT - 1) / kBT));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
+    return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode>, mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, y, err);
 }
 
 }  // namespace

@@ -141,6 +141,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *_
 
     // LoRA K-extension: 2r columns, A operand = [B | B] rows, B operand = [t_hi | t_lo]
     if (r > 0) {
+        // t is written by the down-projection kernel launched just before this
+        // one (programmatic dependent launch): wait for it only here.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int js = 0; js < (2 * r) / 16; ++js) {
             const int j0 = (16 * js) % r;  // column of B for k-slot 0 of this step
             uint32_t tb0[NT], tb1[NT];
@@ -148,8 +151,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *_
             for (int nt = 0; nt < NT; ++nt) {
                 const uint32_t *tr = reinterpret_cast<const uint32_t *>(t2 + (int64_t)(g + 8 * nt) * rp);
                 const int w0 = (16 * js + 2 * tq) >> 1;
-                tb0[nt] = tvalid[nt] ? __ldg(tr + w0) : 0u;
-                tb1[nt] = tvalid[nt] ? __ldg(tr + w0 + 4) : 0u;
+                // L2-coherent loads: t was written by the preceding kernel
+                tb0[nt] = tvalid[nt] ? __ldcg(tr + w0) : 0u;
+                tb1[nt] = tvalid[nt] ? __ldcg(tr + w0 + 4) : 0u;
             }
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
@@ -185,16 +189,22 @@ template <int kMode>
 cudaError_t launch_gemv_mode(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                              const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                              void *y, cudaStream_t stream) {
-    const unsigned grid = (unsigned)((N + kRowsPerCta - 1) / kRowsPerCta);
     auto *xp = static_cast<const __nv_bfloat16 *>(x);
     auto *bp = static_cast<const __nv_bfloat16 *>(B);
     auto *tp = static_cast<const __nv_bfloat16 *>(t2);
     auto *yp = static_cast<__nv_bfloat16 *>(y);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((N + kRowsPerCta - 1) / kRowsPerCta));
+    cfg.blockDim = dim3(kGemvWarps * 32);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
     if (M <= 8)
-        k_gemv<kMode, 1><<<grid, kGemvWarps * 32, 0, stream>>>(xp, M, K, N, packed, q8, scales, offset, bp, r, tp, rp, yp);
-    else
-        k_gemv<kMode, 2><<<grid, kGemvWarps * 32, 0, stream>>>(xp, M, K, N, packed, q8, scales, offset, bp, r, tp, rp, yp);
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, k_gemv<kMode, 1>, xp, M, K, N, packed, q8, scales, offset, bp, r, tp, rp, yp);
+    return cudaLaunchKernelEx(&cfg, k_gemv<kMode, 2>, xp, M, K, N, packed, q8, scales, offset, bp, r, tp, rp, yp);
 }
 
 }  // namespace

@@ -11,15 +11,20 @@
 // about 16 significant bits of v, so the low-rank term is not limited by
 // bf16 rounding of t; the consumers multiply [t_hi | t_lo] by [B | B].
 //
-// Layout of the work: a CTA owns 16 rows of x; its 8 warps split K (warp w
-// takes k16-steps w, w+8, ...), each warp runs m16n8k16 MMAs over all r
-// columns, and the 8 partial tiles are summed in shared memory in warp order.
+// Layout of the work: a CTA owns 16 rows of x; its 16 warps split K (warp w
+// takes k16-steps w, w+16, ...), each warp runs m16n8k16 MMAs over all r
+// columns, and the 16 partial tiles are summed in shared memory in warp
+// order.  For decode-size M the whole projection is one CTA whose warps each
+// issue all their loads up front, so its latency is a few memory round trips.
+// The kernel triggers programmatic dependent launch at entry: the fused
+// linear that follows starts streaming the weight at once and waits for t
+// only where it reads it (griddepcontrol.wait).
 #include "mma_util.cuh"
 
 namespace nf4 {
 namespace {
 
-constexpr int kDownWarps = 8;
+constexpr int kDownWarps = 16;
 
 template <int kR>
 __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat16 *__restrict__ x,
@@ -27,7 +32,9 @@ __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat
                                                                int64_t K, float s, __nv_bfloat16 *__restrict__ t2,
                                                                int rp) {
     constexpr int NT = kR / 8;  // n8 tiles
-    __shared__ float s_part[kDownWarps][NT][4][32];
+    extern __shared__ float s_part_raw[];  // [kDownWarps][NT][4][32]
+    auto s_part = reinterpret_cast<float (*)[NT][4][32]>(s_part_raw);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tq = lane & 3;
     const int64_t m0 = (int64_t)blockIdx.x * 16;
@@ -41,6 +48,7 @@ __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat
     for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
 
     const int64_t ksteps = K / 16;
+#pragma unroll 4
     for (int64_t kk = warp; kk < ksteps; kk += kDownWarps) {
         const int64_t kw = (kk * 16 + 2 * tq) >> 1;  // 32-bit word index of column 16 kk + 2 tq
         uint32_t a[4];
@@ -59,7 +67,7 @@ __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat
 #pragma unroll
         for (int i = 0; i < 4; ++i) s_part[warp][nt][i][lane] = acc[nt][i];
     __syncthreads();
-    // 16 rows x kR columns = 16 kR outputs, the 256 threads share them
+    // 16 rows x kR columns = 16 kR outputs, shared by all threads
     for (int o = threadIdx.x; o < NT * 4 * 32; o += kDownWarps * 32) {
         const int nt = o / 128, i = (o / 32) & 3, ln = o & 31;
         float v = 0.0f;
@@ -83,6 +91,17 @@ __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat
     }
 }
 
+template <int kR>
+cudaError_t launch_down(unsigned grid, size_t smem, cudaStream_t stream, const __nv_bfloat16 *x,
+                        const __nv_bfloat16 *A, int64_t M, int64_t K, float s, __nv_bfloat16 *t2, int rp) {
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_lora_down<kR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_lora_down<kR><<<grid, kDownWarps * 32, smem, stream>>>(x, A, M, K, s, t2, rp);
+    return cudaSuccess;
+}
+
 }  // namespace
 
 int lora_rp(int r) { return ((2 * r + 63) / 64) * 64; }
@@ -91,15 +110,18 @@ cudaError_t launch_lora_down(const void *x, const void *A, int64_t M, int64_t K,
                              cudaStream_t stream) {
     const unsigned grid = (unsigned)((M + 15) / 16);
     const int rp = lora_rp(r);
+    const size_t smem = (size_t)kDownWarps * (r / 8) * 4 * 32 * sizeof(float);
     auto *xp = static_cast<const __nv_bfloat16 *>(x);
     auto *ap = static_cast<const __nv_bfloat16 *>(A);
     auto *tp = static_cast<__nv_bfloat16 *>(t2);
+    cudaError_t e = cudaSuccess;
     switch (r) {
-        case 16: k_lora_down<16><<<grid, kDownWarps * 32, 0, stream>>>(xp, ap, M, K, s, tp, rp); break;
-        case 32: k_lora_down<32><<<grid, kDownWarps * 32, 0, stream>>>(xp, ap, M, K, s, tp, rp); break;
-        case 64: k_lora_down<64><<<grid, kDownWarps * 32, 0, stream>>>(xp, ap, M, K, s, tp, rp); break;
+        case 16: e = launch_down<16>(grid, smem, stream, xp, ap, M, K, s, tp, rp); break;
+        case 32: e = launch_down<32>(grid, smem, stream, xp, ap, M, K, s, tp, rp); break;
+        case 64: e = launch_down<64>(grid, smem, stream, xp, ap, M, K, s, tp, rp); break;
         default: return cudaErrorInvalidValue;
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -6,10 +6,10 @@
 // quotient; ties go to the lower index, i.e. code = #{i : x > t_i} with
 // t_i = RD_f32((q_i + q_{i+1}) / 2) (the exact midpoint rounded down).
 //
-// Layout of the work: one thread owns 8 consecutive elements, so the 8 lanes
-// l..l+7 (l a multiple of 8) of a warp own one 64-block; c1 is a 3-step
-// xor-shuffle max inside that lane group.  Each thread writes its 8 codes as
-// one 32-bit word (4 packed bytes), a warp 128 contiguous bytes.
+// Layout of the work: one thread owns groups of 8 consecutive elements, so
+// the 8 lanes l..l+7 (l a multiple of 8) of a warp own one 64-block; c1 is a
+// 3-step xor-shuffle max inside that lane group.  Each thread writes its 8
+// codes as one 32-bit word (4 packed bytes), a warp 128 contiguous bytes.
 //
 // Division-free exact code selection: instead of the per-element IEEE
 // division, each element uses q = RN(w * RN(1 / c1)), which is within 2^-22
@@ -96,6 +96,60 @@ __device__ __forceinline__ void load8(const void *w, int64_t e0, int64_t n, floa
     }
 }
 
+// One group = 8 consecutive elements, owned by one thread; the 8 lanes of a
+// lane group (lane / 8) own one 64-block.  A thread handles kUnroll groups per
+// iteration, 256 groups apart (so lane groups still cover whole blocks), and
+// issues all their loads before any arithmetic.
+template <bool kBf16>
+__device__ __forceinline__ void quantize_group(float v[8], int64_t g, int64_t e0, int64_t n, int lane,
+                                               const float *s_t, const uint32_t *s_cell,
+                                               uint8_t *__restrict__ packed, float *__restrict__ absmax) {
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 4));
+    const float c1 = a;
+    if (e0 >= n) return;
+    if ((lane & 7) == 0) absmax[g >> 3] = c1;
+
+    int code[8];
+    if (c1 == 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) code[i] = 7;
+    } else if (c1 < 0x1p-125f || c1 >= 0x1p125f) {
+        // c1 < 2^-125 or >= 2^125: 1/c1 may overflow or be subnormal, so
+        // the 2^-22 error bound of the fast path would not hold
+#pragma unroll
+        for (int i = 0; i < 8; ++i) code[i] = exact_code(v[i], c1, s_t);
+    } else {
+        const float rc = __frcp_rn(c1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float q = __fmul_rn(v[i], rc);
+            float f = __fmaf_rn(q, 64.0f, 12582976.0f);  // 1.5 * 2^23 + 64: RN(64 q) + 64 in the low bits
+            // in [0, 128] for finite inputs; the clamp keeps a non-finite
+            // input from indexing outside the table
+            uint32_t e = s_cell[min(__float_as_uint(f) - 0x4B400000u, 128u)];
+            float t = __uint_as_float(e);
+            int c = (int)(e & 15u) + ((q > t) ? 1 : 0);
+            if (fabsf(q - t) <= kAmbiguity) c = exact_code(v[i], c1, s_t);
+            code[i] = c;
+        }
+    }
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) word |= (uint32_t)((code[2 * j] << 4) | code[2 * j + 1]) << (8 * j);
+    if (e0 + 8 <= n) {
+        reinterpret_cast<uint32_t *>(packed)[g] = word;
+    } else {
+        for (int j = 0; 2 * j < (int)(n - e0); ++j) packed[(e0 >> 1) + j] = (uint8_t)(word >> (8 * j));
+    }
+}
+
+constexpr int kUnroll = 1;
+
 template <bool kBf16>
 __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restrict__ w, int64_t n,
                                                              uint8_t *__restrict__ packed,
@@ -106,55 +160,19 @@ __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restri
 
     const int lane = threadIdx.x & 31;
     const int64_t ngroups = (n + 7) >> 3;
+    constexpr int64_t kSpan = (int64_t)kQuantThreads * kUnroll;  // groups per CTA iteration
     // the trip count depends only on blockIdx, so whole warps stay converged
-    for (int64_t base = (int64_t)blockIdx.x * kQuantThreads; base < ngroups;
-         base += (int64_t)gridDim.x * kQuantThreads) {
-        const int64_t g = base + threadIdx.x;
-        const int64_t e0 = g << 3;
-        float v[8];
-        load8<kBf16>(w, e0, n, v);
-
-        float a = 0.0f;
+    for (int64_t base = (int64_t)blockIdx.x * kSpan; base < ngroups; base += (int64_t)gridDim.x * kSpan) {
+        float v[kUnroll][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
-        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
-        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 4));
-        const float c1 = a;
-        if (e0 >= n) continue;
-        if ((lane & 7) == 0) absmax[g >> 3] = c1;
-
-        int code[8];
-        if (c1 == 0.0f) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) code[i] = 7;
-        } else if (c1 < 0x1p-125f || c1 >= 0x1p125f) {
-            // c1 < 2^-125 or >= 2^125: 1/c1 may overflow or be subnormal, so
-            // the 2^-22 error bound of the fast path would not hold
-#pragma unroll
-            for (int i = 0; i < 8; ++i) code[i] = exact_code(v[i], c1, s_t);
-        } else {
-            const float rc = __frcp_rn(c1);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float q = __fmul_rn(v[i], rc);
-                float f = __fmaf_rn(q, 64.0f, 12582976.0f);  // 1.5 * 2^23 + 64: RN(64 q) + 64 in the low bits
-                // in [0, 128] for finite inputs; the clamp keeps a non-finite
-                // input from indexing outside the table
-                uint32_t e = s_cell[min(__float_as_uint(f) - 0x4B400000u, 128u)];
-                float t = __uint_as_float(e);
-                int c = (int)(e & 15u) + ((q > t) ? 1 : 0);
-                if (fabsf(q - t) <= kAmbiguity) c = exact_code(v[i], c1, s_t);
-                code[i] = c;
-            }
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = base + u * kQuantThreads + threadIdx.x;
+            load8<kBf16>(w, g << 3, n, v[u]);
         }
-        uint32_t word = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) word |= (uint32_t)((code[2 * j] << 4) | code[2 * j + 1]) << (8 * j);
-        if (e0 + 8 <= n) {
-            reinterpret_cast<uint32_t *>(packed)[g] = word;
-        } else {
-            for (int j = 0; 2 * j < (int)(n - e0); ++j) packed[(e0 >> 1) + j] = (uint8_t)(word >> (8 * j));
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = base + u * kQuantThreads + threadIdx.x;
+            quantize_group<kBf16>(v[u], g, g << 3, n, lane, s_t, s_cell, packed, absmax);
         }
     }
 }
@@ -165,7 +183,8 @@ cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed
                             cudaStream_t stream, int num_sms) {
     if (n == 0) return cudaSuccess;
     int64_t ngroups = (n + 7) / 8;
-    int64_t want = (ngroups + kQuantThreads - 1) / kQuantThreads;
+    int64_t span = (int64_t)kQuantThreads * kUnroll;
+    int64_t want = (ngroups + span - 1) / span;
     int64_t cap = (int64_t)num_sms * 8;
     int grid = (int)(want < cap ? want : cap);
     if (bf16) k_quantize<true><<<grid, kQuantThreads, 0, stream>>>(w, n, packed, absmax);
