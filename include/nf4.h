@@ -175,6 +175,33 @@ NF4_API nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int6
                                const void *A, const void *B, int r, float scaling,
                                void *y, void *workspace, int64_t workspace_bytes, void *stream);
 
+/* Size of the fixed device scratch array behind nf4_lora_linear_fwd_noalloc
+ * (4 MiB per GPU that loads the library, held until the process exits). */
+#define NF4_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+
+/* nf4_lora_linear_fwd_noalloc -- the same operation, arguments and layouts as
+ * nf4_lora_linear_fwd, for callers that cannot allocate device memory (a
+ * plugin handed only its input and output buffers, a serving loop that must
+ * not call cudaMalloc -- which may synchronize the device -- inside a
+ * latency-critical step, a framework whose memory is fully reserved by its
+ * own pool).  There is no workspace argument: the low-rank intermediate lives
+ * in a fixed device array inside the library.  The pages have no counterpart
+ * to this entry point; it is an interface convenience only.
+ *   Limit: nf4_lora_linear_workspace_size(M, r) must not exceed
+ *          NF4_NOALLOC_SCRATCH_BYTES (M <= 16384 for r = 64, M <= 32768 for
+ *          r <= 32); larger sizes return NF4_ERR_UNSUPPORTED before any work.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls on a device share the array: calls whose kernels may overlap on
+ *   the GPU (unordered streams) race and give undefined results.  Nothing has
+ *   to be cleared between calls.
+ *   Never calls cudaMalloc, cudaFree or any allocating routine. */
+NF4_API nf4_status nf4_lora_linear_fwd_noalloc(const void *x, int64_t M, int64_t K, int64_t N,
+                                               const uint8_t *packed, const uint8_t *absmax_q,
+                                               const float *absmax2, const float *offset,
+                                               const void *A, const void *B, int r, float scaling,
+                                               void *y, void *stream);
+
 /* nf4_device_status -- synchronize `stream`, then read and clear the
  * library's device error word on the current device.  Returns
  * NF4_ERR_TIMEOUT if a bounded wait in a kernel expired since the last call,

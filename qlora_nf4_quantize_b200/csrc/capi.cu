@@ -54,6 +54,11 @@ int sm_count(cudaError_t *status) {
 
 }  // namespace
 
+namespace nf4 {
+// Status mapping shared with entry points defined in other files.
+nf4_status status_of(cudaError_t e) { return cuda_status(e); }
+}  // namespace nf4
+
 extern "C" {
 
 const char *nf4_status_string(nf4_status s) {

@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
     L.nf4_lora_linear_workspace_size.argtypes = [i64, i32]
     L.nf4_lora_linear_fwd.restype = i32
     L.nf4_lora_linear_fwd.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, i32, f32, P, P, i64, P]
+    L.nf4_lora_linear_fwd_noalloc.restype = i32
+    L.nf4_lora_linear_fwd_noalloc.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, i32, f32, P, P]
     L.nf4_device_status.restype = i32
     L.nf4_device_status.argtypes = [P]
     _lib = L
@@ -184,6 +186,31 @@ def nf4_lora_linear_fwd(x: torch.Tensor, packed: torch.Tensor, absmax_q: Optiona
                                    0 if workspace is None else workspace.numel() * workspace.element_size(),
                                    _stream(stream))
     _check("nf4_lora_linear_fwd", st)
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
+
+
+def nf4_lora_linear_fwd_noalloc(x: torch.Tensor, packed: torch.Tensor, absmax_q: Optional[torch.Tensor],
+                                absmax2: torch.Tensor, offset: Optional[torch.Tensor], N: int,
+                                A: Optional[torch.Tensor] = None, B: Optional[torch.Tensor] = None,
+                                scaling: float = 1.0, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """nf4_lora_linear_fwd without a workspace, for callers that cannot
+    allocate device memory: the low-rank intermediate uses the library's
+    fixed 4 MiB device scratch.  Pass a preallocated ``y`` to allocate nothing
+    here either.  Calls that may overlap on the GPU race on the scratch."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    r = 0 if A is None else A.shape[0]
+    if A is not None:
+        _need(A, "A", torch.bfloat16, r * K)
+        _need(B, "B", torch.bfloat16, N * r)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _need(y, "y", torch.bfloat16, M * N)
+    st = lib().nf4_lora_linear_fwd_noalloc(_p(x), M, K, N, _p(packed), _p(absmax_q), _p(absmax2), _p(offset),
+                                           _p(A), _p(B), r, float(scaling), _p(y), _stream(stream))
+    _check("nf4_lora_linear_fwd_noalloc", st)
     return y
 
 
