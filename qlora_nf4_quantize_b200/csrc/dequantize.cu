@@ -6,12 +6,12 @@
 // quantization state (nf4_device.cuh, block_scale).  bf16 output rounds the
 // binary32 value to nearest even.
 //
-// HBM-bound streaming kernel.  A warp handles 2048 consecutive elements per
-// iteration as 8 segments of 256: in segment j lane l owns the 8 elements
+// HBM-bound streaming kernel.  A warp handles 1024 consecutive elements per
+// iteration as 4 segments of 256: in segment j lane l owns the 8 elements
 // starting at 256 j + 8 l, i.e. 4 packed bytes (one 32-bit load; the warp's
 // load is 128 contiguous bytes) and 16 output bytes for bf16 (one 128-bit
-// store; the warp's store is 512 contiguous bytes).  All 8 loads of a lane are
-// issued before any arithmetic, so each thread keeps 32 bytes in flight.
+// store; the warp's store is 512 contiguous bytes).  All 4 loads of a lane are
+// issued before any arithmetic; up to 8 CTAs of 256 threads per SM.
 // Codes are looked up in a 16-entry shared-memory copy of the table (16
 // distinct words in 16 banks: conflict-free for any code pattern).
 #include "nf4_device.cuh"
@@ -20,7 +20,7 @@ namespace nf4 {
 namespace {
 
 constexpr int kDeqThreads = 256;
-constexpr int kSeg = 8;                  // segments per lane per iteration
+constexpr int kSeg = 4;                  // segments per lane per iteration
 constexpr int kWarpElems = kSeg * 256;   // elements per warp per iteration
 
 template <int kMode, bool kBf16Out>
@@ -100,7 +100,7 @@ cudaError_t launch_dequantize(const uint8_t *packed, const uint8_t *q8, const fl
     if (n == 0) return cudaSuccess;
     int64_t witers = (n + kWarpElems - 1) / kWarpElems;
     int64_t want = (witers + (kDeqThreads / 32) - 1) / (kDeqThreads / 32);
-    int64_t cap = (int64_t)num_sms * 6;
+    int64_t cap = (int64_t)num_sms * 8;
     int grid = (int)(want < cap ? want : cap);
     if (q8 == nullptr) return launch_mode<2>(packed, q8, scales, offset, n, out, bf16, grid, stream);
     if (offset == nullptr) return launch_mode<1>(packed, q8, scales, offset, n, out, bf16, grid, stream);

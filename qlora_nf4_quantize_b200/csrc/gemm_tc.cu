@@ -51,6 +51,14 @@ constexpr uint32_t kAccCol = 0;            // accumulator: columns [0, 256)
 constexpr uint32_t kACol = 256;            // A stages: columns [256 + 32 s, +32)
 constexpr uint32_t kXStageBytes = kBT * kBK * 2;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+// Dequantization lookup per warpgroup: bit h set = warpgroup h uses the
+// shared-memory pair table (one shared load per two weights), clear = the
+// register lookup table (byte permutes on the integer pipe).  Mixing the two
+// spreads the work over the integer pipe and the shared-memory pipe.
+#ifndef NF4_GEMM_LUT_MASK
+#define NF4_GEMM_LUT_MASK 0
+#endif
+constexpr int kLutMask = NF4_GEMM_LUT_MASK;
 
 // UMMA instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both
 // K-major, N = 256, M = 128.
@@ -63,6 +71,7 @@ struct __align__(1024) SmemLayout {
     uint64_t x_empty[kStages];
     uint64_t a_full[kStages];
     uint64_t a_empty[kStages];
+    float2 pairs[kLutMask != 0 ? kPairTableFloat2 : 1];
     uint64_t acc_full;
     uint64_t drain;
     uint32_t tmem_base;
@@ -187,27 +196,42 @@ __device__ __forceinline__ void tc_load32(uint32_t taddr, uint32_t v[32]) {
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 64 bf16 weights (one k-step) of weight row n as 32 bf16x2 words, word j =
-// (element 2j low half, element 2j+1 high half).
-template <int kMode>
-__device__ __forceinline__ void dequant_step(const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
-                                             const float *__restrict__ scales, float mu, int64_t n, int64_t K,
-                                             int64_t kt, bool valid, uint32_t out[32]) {
+// The packed codes (8 words) and block constant of one 64-wide k-step of
+// weight row n; all-zero-code words outside the matrix.
+struct StepCodes {
     uint32_t w[8];
-    float c = 0.0f;
+    float c;
+};
+
+template <int kMode>
+__device__ __forceinline__ void load_step(const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
+                                          const float *__restrict__ scales, float mu, int64_t n, int64_t K,
+                                          int64_t kt, bool valid, StepCodes &sc) {
     if (valid) {
         const uint4 *p = reinterpret_cast<const uint4 *>(packed + n * (K >> 1) + kt * 32);
         const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
-        w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
-        w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
-        c = block_scale<kMode>(q8, scales, mu, n * (K >> 6) + kt);
+        sc.w[0] = u0.x; sc.w[1] = u0.y; sc.w[2] = u0.z; sc.w[3] = u0.w;
+        sc.w[4] = u1.x; sc.w[5] = u1.y; sc.w[6] = u1.z; sc.w[7] = u1.w;
+        sc.c = block_scale<kMode>(q8, scales, mu, n * (K >> 6) + kt);
     } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = 0x77777777u;
+        for (int i = 0; i < 8; ++i) sc.w[i] = 0x77777777u;
+        sc.c = 0.0f;
     }
-    const Lut lut = make_lut(c);
+}
+
+// 64 bf16 weights (one k-step) as 32 bf16x2 words, word j = (element 2j low
+// half, element 2j+1 high half).
+__device__ __forceinline__ void dequant_step(const StepCodes &sc, uint32_t out[32]) {
+    const Lut lut = make_lut(sc.c);
 #pragma unroll
-    for (int s = 0; s < 16; ++s) lut_lookup4(lut, w[s >> 1] >> ((s & 1) * 16), out[2 * s], out[2 * s + 1]);
+    for (int s = 0; s < 16; ++s) lut_lookup4(lut, sc.w[s >> 1] >> ((s & 1) * 16), out[2 * s], out[2 * s + 1]);
+}
+
+__device__ __forceinline__ void dequant_step_smem(const StepCodes &sc, const float2 *tbl_lane, uint32_t out[32]) {
+#pragma unroll
+    for (int s = 0; s < 16; ++s)
+        pair_lookup4(tbl_lane, sc.w[s >> 1] >> ((s & 1) * 16), sc.c, out[2 * s], out[2 * s + 1]);
 }
 
 // 64 columns [64 e, 64 e + 64) of the row n of [B | B | 0] (bf16 pairs).
@@ -223,7 +247,8 @@ __device__ __forceinline__ void lora_step(const __nv_bfloat16 *__restrict__ Bl, 
 
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_t, int64_t M,
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_t,
+              const __grid_constant__ CUtensorMap tmap_y, int64_t M,
               int64_t K, int64_t N, const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
               const float *__restrict__ scales, const float *__restrict__ offset,
               const __nv_bfloat16 *__restrict__ Bl, int r, int rp, __nv_bfloat16 *__restrict__ y, unsigned *err) {
@@ -250,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
+    if constexpr (kLutMask != 0) fill_pair_table(S.pairs);
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&S.tmem_base)),
                      "r"(kTmemCols)
@@ -324,12 +350,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         bool ok = true;
+        // software pipeline: the codes of this warpgroup's next k-step are in
+        // flight while the current one is converted
+        StepCodes cur, nxt;
+        if (h < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, h, nvalid, cur);
         for (int kt = h; kt < kt_total; kt += 2) {
             const int s = kt % kStages;
             const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
             uint32_t v[32];
-            if (kt < kw_steps) dequant_step<kMode>(packed, q8, scales, mu, n, K, kt, nvalid, v);
-            else lora_step(Bl, r, n, nvalid, kt - kw_steps, v);
+            if (kt < kw_steps) {
+                if (kt + 2 < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, kt + 2, nvalid, nxt);
+                if ((kLutMask >> h) & 1) dequant_step_smem(cur, S.pairs + (lane & 15), v);
+                else dequant_step(cur, v);
+                cur = nxt;
+            } else {
+                lora_step(Bl, r, n, nvalid, kt - kw_steps, v);
+            }
             // warp-uniform outcome: the tcgen05.st below is a warp-wide instruction
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.a_empty[s], ph ^ 1u, abort, err));
             if (!ok) break;
@@ -340,22 +376,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err));
         if (ok) {
+            // Epilogue: accumulators -> bf16 -> staging tile Y[m][n] (256 x 128,
+            // row-major, in the now idle x ring) -> one TMA store, which also
+            // clips rows and columns outside y.
             tc_fence_after();
+            __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(&S.x[0][0]);
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t v[32];
                 const uint32_t col = kAccCol + 128u * h + 32u * c;
                 tc_load32(lane_base + col, v);
                 tc_wait_ld();
-                const int64_t mb = m0 + 128 * h + 32 * c;
-                if (nvalid) {
+                const int mrow = 128 * h + 32 * c;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int64_t m = mb + i;
-                        if (m < M) y[m * N + n] = __float2bfloat16_rn(__uint_as_float(v[i]));
-                    }
-                }
+                for (int i = 0; i < 32; ++i)
+                    stage[(mrow + i) * kBN + row_in_tile] = __float2bfloat16_rn(__uint_as_float(v[i]));
             }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        // all 256 epilogue threads have staged their values (or given up)
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (threadIdx.x == 128 && !*abort) {
+            asm volatile(
+                "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                    reinterpret_cast<uint64_t>(&tmap_y)),
+                "r"((int)n0), "r"((int)m0), "r"(smem_addr(&S.x[0][0]))
+                : "memory");
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
     }
     tc_fence_before();
@@ -384,24 +432,26 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn(cudaError_t *st) {
     return fn;
 }
 
-// 2-D bf16 tensor [rows, cols] row-major; box = 64 columns x 256 rows,
-// 128-byte swizzle, out-of-range rows read as zero.
-cudaError_t make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols) {
+// 2-D bf16 tensor [rows, cols] row-major with a box of box_cols x box_rows.
+// Operand maps (x, t): box 64 x 256 with 128-byte swizzle, out-of-range rows
+// read as zero.  Output map (y): box 128 x 256, no swizzle; stores clip.
+cudaError_t make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int box_cols, int box_rows,
+                     bool swizzle) {
     cudaError_t st;
     auto fn = get_encode_fn(&st);
     if (fn == nullptr) return st;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBT};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int kMode>
-cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, int64_t M, int64_t K, int64_t N,
+cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUtensorMap &my, int64_t M, int64_t K, int64_t N,
                         const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
                         const __nv_bfloat16 *Bl, int r, int rp, __nv_bfloat16 *y, unsigned *err, cudaStream_t stream) {
     const size_t smem = sizeof(SmemLayout) + 1024;
@@ -417,7 +467,8 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, int64_t M,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
-    return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode>, mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, y, err);
+    return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode>, mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, y,
+                              err);
 }
 
 }  // namespace
@@ -426,17 +477,19 @@ cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const
                            const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                            void *y, cudaStream_t stream, int /*num_sms*/, unsigned *err_word) {
     if (M > 0x7FFFFFFF || K > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    CUtensorMap mx, mt;
-    cudaError_t e = make_map(&mx, x, M, K);
+    CUtensorMap mx, mt, my;
+    cudaError_t e = make_map(&mx, x, M, K, kBK, kBT, true);
     if (e != cudaSuccess) return e;
-    if (r > 0) e = make_map(&mt, t2, M, rp);
-    else e = make_map(&mt, x, M, K);  // unused: no extension steps
+    if (r > 0) e = make_map(&mt, t2, M, rp, kBK, kBT, true);
+    else e = make_map(&mt, x, M, K, kBK, kBT, true);  // unused: no extension steps
+    if (e != cudaSuccess) return e;
+    e = make_map(&my, y, M, N, kBN, kBT, false);
     if (e != cudaSuccess) return e;
     auto *Bl = static_cast<const __nv_bfloat16 *>(B);
     auto *yp = static_cast<__nv_bfloat16 *>(y);
-    if (q8 == nullptr) return launch_mode<2>(mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
-    if (offset == nullptr) return launch_mode<1>(mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
-    return launch_mode<0>(mx, mt, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+    if (q8 == nullptr) return launch_mode<2>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+    if (offset == nullptr) return launch_mode<1>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+    return launch_mode<0>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
 }
 
 }  // namespace nf4

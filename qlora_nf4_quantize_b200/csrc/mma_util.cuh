@@ -55,3 +55,39 @@ __device__ __forceinline__ void lut_lookup4(const Lut &t, uint32_t p16, uint32_t
 }
 
 }  // namespace nf4
+
+namespace nf4 {
+
+// Shared-memory table of unscaled level pairs for byte-wise dequantization:
+// entry b (one packed byte: code of element 2j in the high nibble, 2j+1 in
+// the low nibble) = (q[b >> 4], q[b & 15]).  kPairCopies interleaved copies,
+// entry b of copy c at float2 index 16 b + c, so the 16 lanes of a half-warp
+// (which a 64-bit shared load serves together) read 16 different bank pairs
+// whatever bytes they look up.  32 KB.
+constexpr int kPairCopies = 16;
+constexpr int kPairTableFloat2 = 256 * kPairCopies;
+
+__device__ __forceinline__ void fill_pair_table(float2 *tbl) {
+    for (int i = threadIdx.x; i < kPairTableFloat2; i += blockDim.x) {
+        const int b = i / kPairCopies;
+        tbl[i] = make_float2(c_levels[b >> 4], c_levels[b & 15]);
+    }
+}
+
+// Two bf16 weights of one packed byte: RNE_bf16(RN_f32(q * c)) for both
+// nibbles, returned as a bf16x2 word (element 2j in the low half).
+// tbl_lane = table + (lane & 15).
+__device__ __forceinline__ uint32_t pair_lookup(const float2 *tbl_lane, uint32_t byte, float c) {
+    const float2 q = tbl_lane[byte * kPairCopies];
+    return pack_bf16x2(__fmul_rn(q.x, c), __fmul_rn(q.y, c));
+}
+
+// Same four-code lookup as lut_lookup4 (same output layout) through the
+// shared-memory pair table: p16 holds two packed bytes in its low 16 bits.
+__device__ __forceinline__ void pair_lookup4(const float2 *tbl_lane, uint32_t p16, float c, uint32_t &w01,
+                                             uint32_t &w23) {
+    w01 = pair_lookup(tbl_lane, __byte_perm(p16, 0u, 0x4440), c);
+    w23 = pair_lookup(tbl_lane, __byte_perm(p16, 0u, 0x4441), c);
+}
+
+}  // namespace nf4

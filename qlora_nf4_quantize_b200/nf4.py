@@ -15,7 +15,9 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libnf4.so")
+# NF4_LIB_PATH selects another build of the same library (alternative kernel
+# configurations built with build.build(out=..., defines=...)).
+LIB_PATH = os.environ.get("NF4_LIB_PATH", os.path.join(_PKG, "libnf4.so"))
 BLOCKSIZE = 64
 DQ_BLOCKSIZE = 256
 
