@@ -44,8 +44,17 @@ namespace {
 constexpr int kBN = 128;                   // weight rows per CTA (MMA M)
 constexpr int kBT = 256;                   // tokens per CTA (MMA N)
 constexpr int kBK = 64;                    // k per pipeline step
-constexpr int kStages = 4;
-constexpr int kThreads = 384;
+#ifndef NF4_GEMM_STAGES
+#define NF4_GEMM_STAGES 4
+#endif
+constexpr int kStages = NF4_GEMM_STAGES;  // x tiles in shared memory and A tiles in tensor memory
+static_assert(256 + 32 * kStages <= 512, "tensor memory: 256 accumulator columns + 32 per A stage");
+// Dequant warpgroups: warpgroup h produces the k-steps with index % kWG == h.
+#ifndef NF4_GEMM_WG
+#define NF4_GEMM_WG 2
+#endif
+constexpr int kWG = NF4_GEMM_WG;
+constexpr int kThreads = 128 + 128 * kWG;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;            // accumulator: columns [0, 256)
 constexpr uint32_t kACol = 256;            // A stages: columns [256 + 32 s, +32)
@@ -113,13 +122,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep in hardware until the phase
+// completes or about 0.1 ms pass, instead of spinning on issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(100000u)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: true when the phase completed; false after the time limit
 // (abort raised) or when another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
         if (global_ns() - t0 > kWaitLimitNs) {
             *abort = 1;
@@ -200,38 +223,42 @@ __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sy
 // weight row n; all-zero-code words outside the matrix.
 struct StepCodes {
     uint32_t w[8];
-    float c;
+    ScaleRaw sr;  // block constant operands (decoded at use)
 };
 
 template <int kMode>
 __device__ __forceinline__ void load_step(const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
-                                          const float *__restrict__ scales, float mu, int64_t n, int64_t K,
+                                          const float *__restrict__ scales, float /*mu*/, int64_t n, int64_t K,
                                           int64_t kt, bool valid, StepCodes &sc) {
     if (valid) {
         const uint4 *p = reinterpret_cast<const uint4 *>(packed + n * (K >> 1) + kt * 32);
         const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
         sc.w[0] = u0.x; sc.w[1] = u0.y; sc.w[2] = u0.z; sc.w[3] = u0.w;
         sc.w[4] = u1.x; sc.w[5] = u1.y; sc.w[6] = u1.z; sc.w[7] = u1.w;
-        sc.c = block_scale<kMode>(q8, scales, mu, n * (K >> 6) + kt);
+        sc.sr = block_scale_load<kMode>(q8, scales, n * (K >> 6) + kt);
     } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) sc.w[i] = 0x77777777u;
-        sc.c = 0.0f;
+        sc.sr.q8 = 0;
+        sc.sr.v = 0.0f;
     }
 }
 
 // 64 bf16 weights (one k-step) as 32 bf16x2 words, word j = (element 2j low
 // half, element 2j+1 high half).
-__device__ __forceinline__ void dequant_step(const StepCodes &sc, uint32_t out[32]) {
-    const Lut lut = make_lut(sc.c);
+template <int kMode>
+__device__ __forceinline__ void dequant_step(const StepCodes &sc, float mu, uint32_t out[32]) {
+    const Lut lut = make_lut(block_scale_finish<kMode>(sc.sr, mu));
 #pragma unroll
     for (int s = 0; s < 16; ++s) lut_lookup4(lut, sc.w[s >> 1] >> ((s & 1) * 16), out[2 * s], out[2 * s + 1]);
 }
 
-__device__ __forceinline__ void dequant_step_smem(const StepCodes &sc, const float2 *tbl_lane, uint32_t out[32]) {
+template <int kMode>
+__device__ __forceinline__ void dequant_step_smem(const StepCodes &sc, float mu, const float2 *tbl_lane,
+                                                  uint32_t out[32]) {
+    const float c = block_scale_finish<kMode>(sc.sr, mu);
 #pragma unroll
-    for (int s = 0; s < 16; ++s)
-        pair_lookup4(tbl_lane, sc.w[s >> 1] >> ((s & 1) * 16), sc.c, out[2 * s], out[2 * s + 1]);
+    for (int s = 0; s < 16; ++s) pair_lookup4(tbl_lane, sc.w[s >> 1] >> ((s & 1) * 16), c, out[2 * s], out[2 * s + 1]);
 }
 
 // 64 columns [64 e, 64 e + 64) of the row n of [B | B | 0] (bf16 pairs).
@@ -343,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 4) {
         // ---------------- dequant warpgroups, then epilogue ----------------
         const int q = warp & 3;         // tensor-memory lane quarter
-        const int h = (warp - 4) >> 2;  // warpgroup: k-steps with index % 2 == h
+        const int h = (warp - 4) >> 2;  // warpgroup: k-steps with index % kWG == h
         const int row_in_tile = 32 * q + lane;
         const int64_t n = n0 + row_in_tile;
         const bool nvalid = n < N;
@@ -354,14 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // flight while the current one is converted
         StepCodes cur, nxt;
         if (h < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, h, nvalid, cur);
-        for (int kt = h; kt < kt_total; kt += 2) {
+        for (int kt = h; kt < kt_total; kt += kWG) {
             const int s = kt % kStages;
             const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
             uint32_t v[32];
             if (kt < kw_steps) {
-                if (kt + 2 < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, kt + 2, nvalid, nxt);
-                if ((kLutMask >> h) & 1) dequant_step_smem(cur, S.pairs + (lane & 15), v);
-                else dequant_step(cur, v);
+                if (kt + kWG < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, kt + kWG, nvalid, nxt);
+                if ((kLutMask >> h) & 1) dequant_step_smem<kMode>(cur, mu, S.pairs + (lane & 15), v);
+                else dequant_step<kMode>(cur, mu, v);
                 cur = nxt;
             } else {
                 lora_step(Bl, r, n, nvalid, kt - kw_steps, v);
@@ -382,20 +409,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(&S.x[0][0]);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = h; c < kBT / 32; c += kWG) {  // 32-token chunks of the tile
                 uint32_t v[32];
-                const uint32_t col = kAccCol + 128u * h + 32u * c;
-                tc_load32(lane_base + col, v);
+                tc_load32(lane_base + kAccCol + 32u * c, v);
                 tc_wait_ld();
-                const int mrow = 128 * h + 32 * c;
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    stage[(mrow + i) * kBN + row_in_tile] = __float2bfloat16_rn(__uint_as_float(v[i]));
+                    stage[(32 * c + i) * kBN + row_in_tile] = __float2bfloat16_rn(__uint_as_float(v[i]));
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
-        // all 256 epilogue threads have staged their values (or given up)
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        // all dequant/epilogue threads have staged their values (or given up)
+        asm volatile("bar.sync 1, %0;" ::"n"(128 * kWG) : "memory");
         if (threadIdx.x == 128 && !*abort) {
             asm volatile(
                 "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(

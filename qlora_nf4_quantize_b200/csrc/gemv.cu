@@ -43,12 +43,12 @@ constexpr bool kGemvSmemLut = NF4_GEMV_SMEM_LUT != 0;
 template <int MT>
 struct BlockSet {
     uint32_t w[2 * MT][8];
-    float c[2 * MT];
+    ScaleRaw sr[2 * MT];  // block constant operands (decoded at use)
 };
 
 template <int kMode, int MT>
 __device__ __forceinline__ void load_set(const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
-                                         const float *__restrict__ scales, float mu, const int64_t *row,
+                                         const float *__restrict__ scales, float /*mu*/, const int64_t *row,
                                          const bool *rvalid, int64_t K, int64_t kblocks, int64_t bk,
                                          BlockSet<MT> &bp) {
     const bool kvalid = bk < kblocks;
@@ -59,11 +59,12 @@ __device__ __forceinline__ void load_set(const uint8_t *__restrict__ packed, con
             const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
             bp.w[i][0] = u0.x; bp.w[i][1] = u0.y; bp.w[i][2] = u0.z; bp.w[i][3] = u0.w;
             bp.w[i][4] = u1.x; bp.w[i][5] = u1.y; bp.w[i][6] = u1.z; bp.w[i][7] = u1.w;
-            bp.c[i] = block_scale<kMode>(q8, scales, mu, row[i] * kblocks + bk);
+            bp.sr[i] = block_scale_load<kMode>(q8, scales, row[i] * kblocks + bk);
         } else {
 #pragma unroll
             for (int j = 0; j < 8; ++j) bp.w[i][j] = 0x77777777u;
-            bp.c[i] = 0.0f;
+            bp.sr[i].q8 = 0;
+            bp.sr[i].v = 0.0f;
         }
     }
 }
@@ -129,10 +130,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *_
         const bool kvalid = bk < kblocks;
         if (ss + kGemvWarps < nsuper)
             load_set<kMode, MT>(packed, q8, scales, mu, row, rvalid, K, kblocks, (ss + kGemvWarps) * 4 + tq, nxt);
+        float cs[2 * MT];
+#pragma unroll
+        for (int i = 0; i < 2 * MT; ++i) cs[i] = block_scale_finish<kMode>(cur.sr[i], mu);
         Lut lut[kSmemLut ? 1 : 2 * MT];
         if constexpr (!kSmemLut) {
 #pragma unroll
-            for (int i = 0; i < 2 * MT; ++i) lut[i] = make_lut(cur.c[i]);
+            for (int i = 0; i < 2 * MT; ++i) lut[i] = make_lut(cs[i]);
         }
         const int64_t kx4 = bk * 16;  // x offset of this block in 4-element units
 #pragma unroll
@@ -146,8 +150,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *_
                 const uint32_t p0 = cur.w[2 * mt][s >> 1] >> ((s & 1) * 16);
                 const uint32_t p1 = cur.w[2 * mt + 1][s >> 1] >> ((s & 1) * 16);
                 if constexpr (kSmemLut) {
-                    pair_lookup4(tbl_lane, p0, cur.c[2 * mt], a[0], a[2]);
-                    pair_lookup4(tbl_lane, p1, cur.c[2 * mt + 1], a[1], a[3]);
+                    pair_lookup4(tbl_lane, p0, cs[2 * mt], a[0], a[2]);
+                    pair_lookup4(tbl_lane, p1, cs[2 * mt + 1], a[1], a[3]);
                 } else {
                     lut_lookup4(lut[2 * mt], p0, a[0], a[2]);
                     lut_lookup4(lut[2 * mt + 1], p1, a[1], a[3]);

@@ -44,14 +44,47 @@ __device__ __forceinline__ Lut make_lut(float c) {
 // lo01 = (e0 in the low half, e1 in the high half), lo23 = (e2, e3).
 // Each byte permute selects within 8 bytes, so codes 0-7 and 8-15 are looked
 // up separately and merged on bit 3 of each code.
-__device__ __forceinline__ void lut_lookup4(const Lut &t, uint32_t p16, uint32_t &w01, uint32_t &w23) {
-    const uint32_t s = p16 & 0x7777u;
-    const uint32_t s2 = ((p16 >> 1) & 0x4444u) | 0x3210u;
+__device__ __forceinline__ void lut_lookup4_sel(const Lut &t, uint32_t s, uint32_t s2, uint32_t &w01,
+                                                uint32_t &w23) {
     const uint32_t loA = __byte_perm(t.L0, t.L1, s), loB = __byte_perm(t.L2, t.L3, s);
     const uint32_t hiA = __byte_perm(t.H0, t.H1, s), hiB = __byte_perm(t.H2, t.H3, s);
     const uint32_t lo = __byte_perm(loA, loB, s2), hi = __byte_perm(hiA, hiB, s2);
     w01 = __byte_perm(lo, hi, 0x4051);
     w23 = __byte_perm(lo, hi, 0x6273);
+}
+
+static __constant__ uint32_t c_selector_mul[2] = {1u << 16, 1u << 31};
+
+// Selectors of the byte permutes for the 8 codes of one 32-bit word of packed
+// codes: s = low 3 bits of each code (bit 3 cleared, so no sign-replicate
+// mode), s2 = per output byte i, i + 4 * (bit 3 of code i).  A byte permute
+// reads only the low 16 bits of its selector, so the high halves serve the
+// codes of bytes 2 and 3 after a 16-bit shift.
+__device__ __forceinline__ void lut_selectors(uint32_t w, uint32_t &s_lo, uint32_t &s_hi, uint32_t &s2_lo,
+                                              uint32_t &s2_hi) {
+    // The right shifts are high halves of products (w >> k = umulhi(w, 2^(32-k))),
+    // which issue on the multiply-add pipe and leave the integer pipe, the
+    // bottleneck of the dequantization, to the masks and byte permutes.
+    // The multipliers are read from constant memory so that the compiler
+    // does not turn the products back into shifts.
+    const uint32_t m16 = c_selector_mul[0], m31 = c_selector_mul[1];
+    s_lo = w & 0x77777777u;
+    s_hi = __umulhi(s_lo, m16);
+    s2_lo = (__umulhi(w, m31) & 0x44444444u) | 0x32103210u;
+    s2_hi = __umulhi(s2_lo, m16);
+}
+
+__device__ __forceinline__ void lut_lookup4(const Lut &t, uint32_t p16, uint32_t &w01, uint32_t &w23) {
+    lut_lookup4_sel(t, p16 & 0x7777u, ((p16 >> 1) & 0x4444u) | 0x3210u, w01, w23);
+}
+
+// The 8 weights of one 32-bit word of packed codes (bytes 0..3, two codes
+// each) as four bf16x2 words, in element order.
+__device__ __forceinline__ void lut_lookup8(const Lut &t, uint32_t w, uint32_t out[4]) {
+    uint32_t s_lo, s_hi, s2_lo, s2_hi;
+    lut_selectors(w, s_lo, s_hi, s2_lo, s2_hi);
+    lut_lookup4_sel(t, s_lo, s2_lo, out[0], out[1]);
+    lut_lookup4_sel(t, s_hi, s2_hi, out[2], out[3]);
 }
 
 }  // namespace nf4

@@ -59,6 +59,38 @@ __device__ __forceinline__ float block_scale(const uint8_t *__restrict__ q8, con
     }
 }
 
+// Raw operands of a block constant, loaded ahead of use so that the loads
+// overlap other work; block_scale_finish() turns them into c1'.
+struct ScaleRaw {
+    uint32_t q8;  // E4M3 code (kMode 0, 1)
+    float v;      // c2 (kMode 0, 1) or the fp32 c1 itself (kMode 2)
+};
+
+template <int kMode>
+__device__ __forceinline__ ScaleRaw block_scale_load(const uint8_t *__restrict__ q8, const float *__restrict__ scales,
+                                                     int64_t b) {
+    ScaleRaw r;
+    if constexpr (kMode == 2) {
+        r.q8 = 0;
+        r.v = __ldg(scales + b);
+    } else {
+        r.q8 = __ldg(q8 + b);
+        r.v = __ldg(scales + (b >> 8));
+    }
+    return r;
+}
+
+template <int kMode>
+__device__ __forceinline__ float block_scale_finish(const ScaleRaw &r, float mu) {
+    if constexpr (kMode == 2) {
+        return r.v;
+    } else {
+        const float d = e4m3_to_f32((uint8_t)r.q8);
+        if constexpr (kMode == 0) return __fmaf_rn(d, r.v, mu);
+        else return __fmul_rn(d, r.v);
+    }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
     return *reinterpret_cast<uint32_t *>(&v);

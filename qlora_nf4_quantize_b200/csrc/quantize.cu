@@ -26,7 +26,8 @@ namespace nf4 {
 namespace {
 
 constexpr float kAmbiguity = 0x1p-18f;
-constexpr int kCells = 129;
+constexpr int kCells = 129;       // cells 0..128 cover q in [-1, 1]
+constexpr int kCellTable = 256;   // indexed by the low byte of RN(64 q) + 64 (+ 1.5 * 2^23)
 constexpr int kQuantThreads = 256;
 
 __device__ __forceinline__ int exact_code(float w, float c1, const float *s_t) {
@@ -45,6 +46,7 @@ __device__ void build_tables(float *s_t, uint32_t *s_cell) {
         s_t[tid] = __double2float_rd(m);
     }
     __syncthreads();
+    if (tid >= kCells && tid < kCellTable) s_cell[tid] = 0x40800000u | 15u;  // never reached by finite q
     if (tid < kCells) {
         // cell tid holds q with RN(64 q) = tid - 64, i.e. q in [lo, hi]
         float lo = ((float)tid - 64.5f) * 0.015625f;
@@ -125,22 +127,28 @@ __device__ __forceinline__ void quantize_group(float v[8], int64_t g, int64_t e0
         for (int i = 0; i < 8; ++i) code[i] = exact_code(v[i], c1, s_t);
     } else {
         const float rc = __frcp_rn(c1);
+        bool amb = false;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            float q = __fmul_rn(v[i], rc);
-            float f = __fmaf_rn(q, 64.0f, 12582976.0f);  // 1.5 * 2^23 + 64: RN(64 q) + 64 in the low bits
-            // in [0, 128] for finite inputs; the clamp keeps a non-finite
-            // input from indexing outside the table
-            uint32_t e = s_cell[min(__float_as_uint(f) - 0x4B400000u, 128u)];
-            float t = __uint_as_float(e);
-            int c = (int)(e & 15u) + ((q > t) ? 1 : 0);
-            if (fabsf(q - t) <= kAmbiguity) c = exact_code(v[i], c1, s_t);
-            code[i] = c;
+            const float q = __fmul_rn(v[i], rc);
+            const float f = __fmaf_rn(q, 64.0f, 12582976.0f);  // 1.5 * 2^23 + 64: RN(64 q) + 64 in the low bits
+            // RN(64 q) + 64 is in [0, 128] for finite inputs; the byte mask
+            // keeps any input inside the 256-entry table
+            const uint32_t e = s_cell[__float_as_uint(f) & 0xFFu];
+            const float t = __uint_as_float(e);
+            code[i] = (int)(e & 15u) + ((q > t) ? 1 : 0);
+            amb |= fabsf(q - t) <= kAmbiguity;
+        }
+        if (amb) {  // rare: some quotient is within 2^-18 of a threshold
+#pragma unroll
+            for (int i = 0; i < 8; ++i) code[i] = exact_code(v[i], c1, s_t);
         }
     }
-    uint32_t word = 0;
+    // byte j = code[2j] << 4 | code[2j+1]; word = bytes 0..3
+    uint32_t b[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) word |= (uint32_t)((code[2 * j] << 4) | code[2 * j + 1]) << (8 * j);
+    for (int j = 0; j < 4; ++j) b[j] = (uint32_t)(code[2 * j] * 16 + code[2 * j + 1]);
+    const uint32_t word = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     if (e0 + 8 <= n) {
         reinterpret_cast<uint32_t *>(packed)[g] = word;
     } else {
@@ -155,7 +163,7 @@ __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restri
                                                              uint8_t *__restrict__ packed,
                                                              float *__restrict__ absmax) {
     __shared__ float s_t[16];
-    __shared__ uint32_t s_cell[kCells + 3];
+    __shared__ uint32_t s_cell[kCellTable];
     build_tables(s_t, s_cell);
 
     const int lane = threadIdx.x & 31;
