@@ -496,6 +496,171 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUte
                               err);
 }
 
+// ---------------------------------------------------------------------------
+// LoRA down-projection for large M on the tensor cores:
+//   t = s x A^T,  x [M, K] bf16,  A [r, K] bf16,  t as [t_hi | t_lo | 0] bf16
+// (same output as the warp-MMA kernel in lora_down.cu).  A CTA owns 128 rows
+// of x: D[128, r] += X[128, k] A[r, k]^T with both operands brought by TMA
+// (128-byte swizzle, kDownStages-deep ring) and one thread issuing the MMAs
+// (M = 128, N = r, K = 16) into r fp32 columns of tensor memory; the four
+// warps then read one token row per thread and write its hi/lo pair.
+constexpr int kDownStages = 4;
+constexpr int kDownRows = 128;
+
+template <int kR>
+struct __align__(1024) DownSmem {
+    uint8_t x[kDownStages][kDownRows * 128];
+    uint8_t a[kDownStages][kR * 128];
+    uint64_t full[kDownStages];
+    uint64_t empty[kDownStages];
+    uint64_t acc_full;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+template <int kR>
+__global__ void __launch_bounds__(128, 1)
+    k_lora_down_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_a, int64_t M,
+                   int64_t K, float scaling, __nv_bfloat16 *__restrict__ t2, int rp, unsigned *err) {
+    constexpr uint32_t kCols = kR < 32 ? 32 : kR;  // tensor memory allocation (power of 2, >= 32)
+    constexpr uint32_t kIdescDown = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kR >> 3) << 17) |
+                                    ((uint32_t)(kDownRows >> 4) << 24);
+    constexpr uint32_t kStageBytes = kDownRows * 128 + kR * 128;
+    extern __shared__ uint8_t smem_raw[];
+    DownSmem<kR> &S =
+        *reinterpret_cast<DownSmem<kR> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    volatile int *abort = &S.abort;
+    // the fused linear launched next may start now; it waits for t itself
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m0 = (int64_t)blockIdx.x * kDownRows;
+    const int kt_total = (int)(K / 64);
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kDownStages; ++st) {
+            mbar_init(&S.full[st], 1);
+            mbar_init(&S.empty[st], 1);
+        }
+        mbar_init(&S.acc_full, 1);
+        S.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&S.tmem_base)),
+                     "r"(kCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    bool ok = true;
+    if (threadIdx.x == 0) {
+        // producer and MMA issuer in one thread: loads run kDownStages - 1 ahead
+        auto issue = [&](int kt) -> bool {
+            const int st = kt % kDownStages;
+            const uint32_t ph = (uint32_t)(kt / kDownStages) & 1u;
+            if (!mbar_wait(&S.empty[st], ph ^ 1u, abort, err)) return false;
+            mbar_arrive_expect_tx(&S.full[st], kStageBytes);
+            tma_load_2d(S.x[st], &tmap_x, &S.full[st], kt * 64, (int)m0);
+            tma_load_2d(S.a[st], &tmap_a, &S.full[st], kt * 64, 0);
+            return true;
+        };
+        int issued = 0;
+        for (; issued < kDownStages - 1 && issued < kt_total && ok; ++issued) ok = issue(issued);
+        for (int kt = 0; kt < kt_total && ok; ++kt) {
+            if (issued < kt_total) {
+                ok = issue(issued);
+                ++issued;
+                if (!ok) break;
+            }
+            const int st = kt % kDownStages;
+            if (!mbar_wait(&S.full[st], (uint32_t)(kt / kDownStages) & 1u, abort, err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint64_t ad = smem_desc_sw128(S.x[st]), bd = smem_desc_sw128(S.a[st]);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc_mma_ss(tmem, ad + 2ull * kk, bd + 2ull * kk, kIdescDown, (kt | kk) != 0 ? 1u : 0u);
+            tc_commit(&S.empty[st]);
+        }
+        tc_commit(&S.acc_full);
+        // every issued load has landed before the CTA may exit
+        for (int kt = issued - kDownStages < 0 ? 0 : issued - kDownStages; kt < issued; ++kt) {
+            unsigned long long t0 = global_ns();
+            while (!mbar_try_wait(&S.full[kt % kDownStages], (uint32_t)(kt / kDownStages) & 1u) &&
+                   global_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    }
+    __syncwarp();
+    // epilogue: thread = token row m0 + 32 warp + lane, r fp32 columns
+    if (__all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err))) {
+        tc_fence_after();
+        const int64_t m = m0 + 32 * warp + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+        for (int c0 = 0; c0 < kR; c0 += 16) {
+            uint32_t v[32];
+            tc_load32(taddr + (uint32_t)(c0 & ~31), v);  // 32 columns (the allocation holds at least 32)
+            tc_wait_ld();
+            if (m < M) {
+                uint32_t hi[8], lo[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float a0 = __uint_as_float(v[(c0 & 31) + 2 * j]) * scaling;
+                    const float a1 = __uint_as_float(v[(c0 & 31) + 2 * j + 1]) * scaling;
+                    const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
+                    hi[j] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+                    lo[j] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+                }
+                uint4 *th = reinterpret_cast<uint4 *>(t2 + m * rp + c0);
+                uint4 *tl = reinterpret_cast<uint4 *>(t2 + m * rp + kR + c0);
+                th[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                th[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+                tl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                tl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            }
+        }
+        if (m < M)
+            for (int j = 2 * kR; j < rp; j += 8)
+                *reinterpret_cast<uint4 *>(t2 + m * rp + j) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols) : "memory");
+    }
+}
+
+template <int kR>
+cudaError_t launch_down_tc(const CUtensorMap &mx, const CUtensorMap &ma, int64_t M, int64_t K, float s, void *t2,
+                           int rp, unsigned *err, cudaStream_t stream) {
+    const size_t smem = sizeof(DownSmem<kR>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_lora_down_tc<kR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((M + kDownRows - 1) / kDownRows);
+    k_lora_down_tc<kR><<<grid, 128, smem, stream>>>(mx, ma, M, K, s, static_cast<__nv_bfloat16 *>(t2), rp, err);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
@@ -515,6 +680,23 @@ cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const
     if (q8 == nullptr) return launch_mode<2>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
     if (offset == nullptr) return launch_mode<1>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
     return launch_mode<0>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+}
+
+// Tensor-core LoRA down-projection (M > 16): see k_lora_down_tc.
+cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
+                                unsigned *err, cudaStream_t stream) {
+    if (M > 0x7FFFFFFF || K > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    CUtensorMap mx, ma;
+    cudaError_t e = make_map(&mx, x, M, K, 64, kDownRows, true);
+    if (e != cudaSuccess) return e;
+    e = make_map(&ma, A, r, K, 64, r, true);
+    if (e != cudaSuccess) return e;
+    switch (r) {
+        case 16: return launch_down_tc<16>(mx, ma, M, K, s, t2, rp, err, stream);
+        case 32: return launch_down_tc<32>(mx, ma, M, K, s, t2, rp, err, stream);
+        case 64: return launch_down_tc<64>(mx, ma, M, K, s, t2, rp, err, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace nf4

@@ -11,6 +11,8 @@ cudaError_t launch_lora_down(const void *x, const void *A, int64_t M, int64_t K,
 cudaError_t launch_gemv(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                         const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                         void *y, cudaStream_t stream);
+cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
+                                unsigned *err, cudaStream_t stream);
 cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                            const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                            void *y, cudaStream_t stream, int num_sms, unsigned *err_word);
@@ -42,7 +44,9 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
                                cudaStream_t stream, int num_sms, unsigned *err_word) {
     const int rp = r > 0 ? lora_rp(r) : 0;
     if (r > 0) {
-        cudaError_t e = launch_lora_down(x, A, M, K, r, scaling, workspace, stream);
+        // decode-size M: warp-MMA kernel; larger M: tensor-core kernel
+        cudaError_t e = M <= kGemvMaxTokens ? launch_lora_down(x, A, M, K, r, scaling, workspace, stream)
+                                            : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream);
         if (e != cudaSuccess) return e;
     }
     if (M <= kGemvMaxTokens)
