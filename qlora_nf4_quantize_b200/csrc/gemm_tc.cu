@@ -36,6 +36,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "mbarrier.cuh"
 #include "mma_util.cuh"
 
 namespace nf4 {
@@ -59,7 +60,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;            // accumulator: columns [0, 256)
 constexpr uint32_t kACol = 256;            // A stages: columns [256 + 32 s, +32)
 constexpr uint32_t kXStageBytes = kBT * kBK * 2;
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
 // Dequantization lookup per warpgroup: bit h set = warpgroup h uses the
 // shared-memory pair table (one shared load per two weights), clear = the
 // register lookup table (byte permutes on the integer pipe).  Mixing the two
@@ -86,71 +86,6 @@ struct __align__(1024) SmemLayout {
     uint32_t tmem_base;
     int abort;
 };
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// As mbar_try_wait, but the thread may sleep in hardware until the phase
-// completes or about 0.1 ms pass, instead of spinning on issue slots.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity), "r"(100000u)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait: true when the phase completed; false after the time limit
-// (abort raised) or when another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    while (true) {
-        if (mbar_try_wait_sleep(bar, parity)) return true;
-        if (*abort) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
-            *abort = 1;
-            atomicOr(err, 1u);
-            return false;
-        }
-    }
-}
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
     asm volatile(

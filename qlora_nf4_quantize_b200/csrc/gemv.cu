@@ -32,10 +32,20 @@
 namespace nf4 {
 namespace {
 
-constexpr int kGemvWarps = 4;
+#ifndef NF4_GEMV_WARPS
+#define NF4_GEMV_WARPS 4
+#endif
+constexpr int kGemvWarps = NF4_GEMV_WARPS;
+// resident CTAs per SM the register allocation must allow
+#ifndef NF4_GEMV_MINB
+#define NF4_GEMV_MINB 1
+#endif
+// 0 = register lookup table, 1 = shared-memory pair table, 2 = pair table for
+// the first row of each m16 tile and register table for the second
 #ifndef NF4_GEMV_SMEM_LUT
 #define NF4_GEMV_SMEM_LUT 0
 #endif
+constexpr int kGemvLut = NF4_GEMV_SMEM_LUT;
 constexpr bool kGemvSmemLut = NF4_GEMV_SMEM_LUT != 0;
 
 // Packed codes (8 words = one 64-block) and block constants of the 2 MT rows a
@@ -73,8 +83,8 @@ __device__ __forceinline__ void load_set(const uint8_t *__restrict__ packed, con
 // pair_lookup4: one byte permute, one shared load and two multiplies per two
 // weights) instead of the per-block register lookup table (lut_lookup4: about
 // three byte permutes per weight, all on the integer pipe).
-template <int kMode, int NT, int MT, bool kSmemLut>
-__global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *__restrict__ x, int M, int64_t K,
+template <int kMode, int NT, int MT, int kLutSel>
+__global__ void __launch_bounds__(kGemvWarps * 32, NF4_GEMV_MINB) k_gemv(const __nv_bfloat16 *__restrict__ x, int M, int64_t K,
                                                           int64_t N, const uint8_t *__restrict__ packed,
                                                           const uint8_t *__restrict__ q8,
                                                           const float *__restrict__ scales,
@@ -82,6 +92,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *_
                                                           const __nv_bfloat16 *__restrict__ Bl, int r,
                                                           const __nv_bfloat16 *__restrict__ t2, int rp,
                                                           __nv_bfloat16 *__restrict__ y) {
+    constexpr bool kSmemLut = kLutSel != 0;
     __shared__ float s_part[kGemvWarps][MT][NT][4][32];
     extern __shared__ float2 s_pairs[];  // kPairTableFloat2 entries when kSmemLut
     if constexpr (kSmemLut) {
@@ -133,10 +144,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *_
         float cs[2 * MT];
 #pragma unroll
         for (int i = 0; i < 2 * MT; ++i) cs[i] = block_scale_finish<kMode>(cur.sr[i], mu);
-        Lut lut[kSmemLut ? 1 : 2 * MT];
-        if constexpr (!kSmemLut) {
+        Lut lut[2 * MT];
+        if constexpr (kLutSel != 1) {
 #pragma unroll
-            for (int i = 0; i < 2 * MT; ++i) lut[i] = make_lut(cs[i]);
+            for (int i = (kLutSel == 2 ? 1 : 0); i < 2 * MT; i += (kLutSel == 2 ? 2 : 1)) lut[i] = make_lut(cs[i]);
         }
         const int64_t kx4 = bk * 16;  // x offset of this block in 4-element units
 #pragma unroll
@@ -149,9 +160,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *_
                 uint32_t a[4];
                 const uint32_t p0 = cur.w[2 * mt][s >> 1] >> ((s & 1) * 16);
                 const uint32_t p1 = cur.w[2 * mt + 1][s >> 1] >> ((s & 1) * 16);
-                if constexpr (kSmemLut) {
+                if constexpr (kLutSel == 1) {
                     pair_lookup4(tbl_lane, p0, cs[2 * mt], a[0], a[2]);
                     pair_lookup4(tbl_lane, p1, cs[2 * mt + 1], a[1], a[3]);
+                } else if constexpr (kLutSel == 2) {
+                    pair_lookup4(tbl_lane, p0, cs[2 * mt], a[0], a[2]);
+                    lut_lookup4(lut[2 * mt + 1], p1, a[1], a[3]);
                 } else {
                     lut_lookup4(lut[2 * mt], p0, a[0], a[2]);
                     lut_lookup4(lut[2 * mt + 1], p1, a[1], a[3]);
@@ -229,10 +243,425 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(const __nv_bfloat16 *_
             }
 }
 
+// ---------------------------------------------------------------------------
+// Persistent variant (K % 256 == 0 and x fits in shared memory): one CTA of
+// 16 warps per SM walks 16-row weight tiles (tile = blockIdx.x + i gridDim.x).
+//   - Work unit = (tile, super-step ss): 256 columns of packed codes (16 rows
+//     x 128 bytes) plus the block constants' raw operands.  Warp w takes the
+//     units of tile i with (ss + i) % 16 == w.
+//   - Each warp streams its units through its own ring of D slots in shared
+//     memory with cp.async, D units ahead of the one it computes (D from the
+//     shared memory left over, 2..8); 16-byte chunks are XOR-swizzled by row
+//     so that the fragment reads are conflict-free.
+//   - x (M rows, compact, in MMA-fragment order: one conflict-free 128-bit
+//     load per fragment pair) is staged once per CTA.
+//   - Per tile the 16 warps' partial tiles meet in shared memory and every
+//     thread adds one output's 16 partials in warp order.  Without LoRA the
+//     sum is stored; with LoRA it is kept (fp32, shared memory) and, once all
+//     tiles are done, the down-projection's t is awaited and staged and each
+//     tile's K-extension of 2r columns is added by MMA before the store, so
+//     the down-projection runs entirely under the main loop.
+//   - kLut: 0 = register lookup table (integer pipe), 1 = shared-memory pair
+//     table (shared-memory pipe), 2 = pair table for a lane's first row and
+//     register table for its second, spreading the work over both pipes.
+constexpr int kPWarps = 16;
+constexpr int kPSlotBytes = 2048 + 256;  // codes + block constants
+
+__host__ __device__ constexpr int gemv_p_t2_stride(int rp) { return rp + 8; }  // bf16 per staged t row
+
+struct GemvPLayout {
+    int64_t x_off, t2_off, res_off, part_off, pair_off, ring_off, total;
+};
+
+// my_tiles_max: most tiles one CTA walks (kept results, LoRA only)
+__host__ __device__ inline GemvPLayout gemv_p_layout(int M, int64_t K, int rp, int nt, bool smem_lut, int depth,
+                                                     int my_tiles_max) {
+    GemvPLayout L;
+    L.x_off = 0;
+    L.t2_off = L.x_off + (int64_t)M * K * 2;
+    L.res_off = L.t2_off + (rp > 0 ? (int64_t)M * gemv_p_t2_stride(rp) * 2 : 0);
+    L.res_off = (L.res_off + 15) & ~(int64_t)15;
+    L.part_off = L.res_off + (rp > 0 ? (int64_t)my_tiles_max * nt * 128 * 4 : 0);
+    L.pair_off = L.part_off + (int64_t)kPWarps * nt * 4 * 32 * 4;
+    L.ring_off = L.pair_off + (smem_lut ? kPairTableFloat2 * (int64_t)sizeof(float2) : 0);
+    L.total = L.ring_off + (int64_t)kPWarps * depth * kPSlotBytes;
+    return L;
+}
+
+// cp.async of `bytes` (4 or 16) with zero fill when !valid
+template <int kBytes>
+__device__ __forceinline__ void cp_async(void *dst, const void *src, bool valid) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    if constexpr (kBytes == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most n (0..8) of this thread's groups are pending
+__device__ __forceinline__ void cp_async_wait_dyn(int n) {
+    switch (n) {
+        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+        case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+        case 7: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+        default: asm volatile("cp.async.wait_group 8;" ::: "memory"); break;
+    }
+}
+
+// The sequence of units of one warp: tiles in order, within a tile the
+// super-steps ss = (w - i) mod 16, + 16, ... below nsuper.
+struct UnitIter {
+    int tile_i, ss;
+    __device__ __forceinline__ void settle(int w, int my_tiles, int nsuper) {
+        while (tile_i < my_tiles && ss >= nsuper) {
+            ++tile_i;
+            ss = ((w - tile_i) % kPWarps + kPWarps) % kPWarps;
+        }
+    }
+    __device__ __forceinline__ void start(int w, int my_tiles, int nsuper) {
+        tile_i = 0;
+        ss = w;
+        settle(w, my_tiles, nsuper);
+    }
+    __device__ __forceinline__ void next(int w, int my_tiles, int nsuper) {
+        ss += kPWarps;
+        settle(w, my_tiles, nsuper);
+    }
+};
+
+template <int kMode, int NT, int kLut>
+__global__ void __launch_bounds__(kPWarps * 32, 1)
+    k_gemv_p(const __nv_bfloat16 *__restrict__ x, int M, int64_t K, int64_t N, const uint8_t *__restrict__ packed,
+             const uint8_t *__restrict__ q8, const float *__restrict__ scales, const float *__restrict__ offset,
+             const __nv_bfloat16 *__restrict__ Bl, int r, const __nv_bfloat16 *__restrict__ t2, int rp,
+             __nv_bfloat16 *__restrict__ y, int depth, int my_tiles_max) {
+    extern __shared__ __align__(16) uint8_t s_dyn[];
+    constexpr bool kSmemLut = kLut != 0;
+    const GemvPLayout L = gemv_p_layout(M, K, rp, NT, kSmemLut, depth, my_tiles_max);
+    uint4 *xs = reinterpret_cast<uint4 *>(s_dyn + L.x_off);
+    __nv_bfloat16 *t2s = reinterpret_cast<__nv_bfloat16 *>(s_dyn + L.t2_off);
+    float *s_res = reinterpret_cast<float *>(s_dyn + L.res_off);
+    float *s_part = reinterpret_cast<float *>(s_dyn + L.part_off);
+    const float2 *s_pairs = reinterpret_cast<const float2 *>(s_dyn + L.pair_off);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, tq = lane & 3;
+    uint8_t *ring = s_dyn + L.ring_off + (int64_t)warp * depth * kPSlotBytes;
+    const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
+    const int64_t kblocks = K >> 6;
+    const int nsuper = (int)(kblocks >> 2);
+    const int64_t n_tiles = (N + 15) >> 4;
+    const int my_tiles = (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1);
+
+    // Copies of one unit, per lane: code chunk `ch` of rows ch_row + 4 i
+    // (i = 0..3, 8 lanes per 128-byte row) and the block constants of row
+    // lane & 15.  The row pointers change only with the tile.
+    const int ch = lane & 7, ch_row = lane >> 3, sc_row = lane & 15;
+    int staged_tile = -1;
+    const uint8_t *code_src[4];
+    bool code_ok[4];
+    const uint8_t *sc_src = nullptr;
+    int64_t sc_b = 0;  // first block of row lane & 15
+    bool sc_ok = false;
+    auto stage = [&](const UnitIter &it, int slot) {
+        if (it.tile_i < my_tiles) {
+            if (it.tile_i != staged_tile) {
+                staged_tile = it.tile_i;
+                const int64_t row0 = ((int64_t)blockIdx.x + (int64_t)it.tile_i * gridDim.x) * 16;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int64_t n = row0 + ch_row + 4 * i;
+                    code_ok[i] = n < N;
+                    code_src[i] = packed + (code_ok[i] ? n : 0) * (K >> 1) + ch * 16;
+                }
+                const int64_t n = row0 + sc_row;
+                sc_ok = n < N;
+                sc_b = (sc_ok ? n : 0) * kblocks;
+                if constexpr (kMode == 2) sc_src = reinterpret_cast<const uint8_t *>(scales + sc_b);
+                else sc_src = q8 + sc_b;
+            }
+            uint8_t *sb = ring + slot * kPSlotBytes;
+            const int64_t kb = (int64_t)it.ss * 128;  // byte offset of the unit in a packed row
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = ch_row + 4 * i;
+                cp_async<16>(sb + (row * 8 + (ch ^ (row & 7))) * 16, code_src[i] + kb, code_ok[i]);
+            }
+            if constexpr (kMode == 2) {  // fp32 constants: 16 bytes per row
+                if (lane < 16) cp_async<16>(sb + 2048 + lane * 16, sc_src + it.ss * 16, sc_ok);
+            } else {  // E4M3 codes (4 bytes per row) and the row's c2 (the same for the unit's 4 blocks)
+                if (lane < 16) cp_async<4>(sb + 2048 + sc_row * 4, sc_src + it.ss * 4, sc_ok);
+                else cp_async<4>(sb + 2048 + 64 + sc_row * 4, scales + ((sc_b + it.ss * 4) >> 8), sc_ok);
+            }
+        }
+        cp_async_commit();
+    };
+
+    // prologue: x (one group), then the first `depth` units
+    {
+        const int64_t kchunks = K >> 3;
+        const int64_t total = (int64_t)M * kchunks;
+        for (int64_t c = threadIdx.x; c < total; c += blockDim.x) {
+            const int tok = (int)(c / kchunks);
+            const int64_t k = (c - (int64_t)tok * kchunks) * 8;
+            const int64_t ss = k >> 8;
+            const int t = (int)((k >> 6) & 3), p = (int)((k >> 3) & 7);
+            cp_async<16>(xs + ((ss * 8 + p) * M + tok) * 4 + t, x + (int64_t)tok * K + k, true);
+        }
+        cp_async_commit();
+    }
+    UnitIter issue, cons;
+    issue.start(warp, my_tiles, nsuper);
+    cons = issue;
+    for (int d = 0; d < depth; ++d) {
+        stage(issue, d);
+        issue.next(warp, my_tiles, nsuper);
+    }
+    if constexpr (kSmemLut) fill_pair_table(const_cast<float2 *>(s_pairs));
+    const uint32_t tbl_lane = (uint32_t)__cvta_generic_to_shared(s_pairs + (lane & 15));
+    cp_async_wait_dyn(depth);  // x complete (the `depth` unit groups may pend)
+    __syncthreads();           // x and the table visible to all
+
+    int u = 0;  // units consumed by this warp
+    for (int tile_i = 0; tile_i < my_tiles; ++tile_i) {
+        float accs[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) accs[nt][0] = accs[nt][1] = accs[nt][2] = accs[nt][3] = 0.0f;
+        while (cons.tile_i == tile_i) {
+            cp_async_wait_dyn(depth - 1);  // pending: units u+1 .. u+depth-1
+            __syncwarp();
+            const int slot = u % depth;
+            const uint8_t *sb = ring + slot * kPSlotBytes;
+            const uint4 *wb = reinterpret_cast<const uint4 *>(sb);
+            uint32_t w[2][8];
+            ScaleRaw sr[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int row = g + 8 * i;
+                const uint4 c0 = wb[row * 8 + ((2 * tq) ^ (row & 7))];
+                const uint4 c1 = wb[row * 8 + ((2 * tq + 1) ^ (row & 7))];
+                w[i][0] = c0.x; w[i][1] = c0.y; w[i][2] = c0.z; w[i][3] = c0.w;
+                w[i][4] = c1.x; w[i][5] = c1.y; w[i][6] = c1.z; w[i][7] = c1.w;
+                if constexpr (kMode == 2) {
+                    sr[i].q8 = 0;
+                    sr[i].v = reinterpret_cast<const float *>(sb + 2048)[row * 4 + tq];
+                } else {
+                    sr[i].q8 = sb[2048 + row * 4 + tq];
+                    sr[i].v = reinterpret_cast<const float *>(sb + 2048 + 64)[row];
+                }
+            }
+            __syncwarp();  // slot free: refill it with the unit `depth` ahead
+            stage(issue, slot);
+            issue.next(warp, my_tiles, nsuper);
+
+            const float c0 = block_scale_finish<kMode>(sr[0], mu);
+            const float c1 = block_scale_finish<kMode>(sr[1], mu);
+            const uint64_t cc0 = pack_f32x2(c0, c0), cc1 = pack_f32x2(c1, c1);
+            Lut lut0, lut1;
+            if constexpr (kLut == 0) lut0 = make_lut(c0);
+            if constexpr (kLut != 1) lut1 = make_lut(c1);
+            const uint4 *xq = xs + ((int64_t)cons.ss * 8 * M) * 4 + tq;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {  // packed word q = MMA steps 2q, 2q+1
+                uint32_t wa[4], wbb[4];
+                if constexpr (kLut == 0) {
+                    lut_lookup8(lut0, w[0][q], wa);
+                } else {
+                    pair_lookup4_s(tbl_lane, w[0][q], cc0, wa[0], wa[1]);
+                    pair_lookup4_s(tbl_lane, w[0][q] >> 16, cc0, wa[2], wa[3]);
+                }
+                if constexpr (kLut == 1) {
+                    pair_lookup4_s(tbl_lane, w[1][q], cc1, wbb[0], wbb[1]);
+                    pair_lookup4_s(tbl_lane, w[1][q] >> 16, cc1, wbb[2], wbb[3]);
+                } else {
+                    lut_lookup8(lut1, w[1][q], wbb);
+                }
+                uint4 xv[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int tok = g + 8 * nt;
+                    xv[nt] = tok < M ? xq[(q * M + tok) * 4] : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t a[4] = {wa[2 * h], wbb[2 * h], wa[2 * h + 1], wbb[2 * h + 1]};
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const uint32_t b0 = h ? xv[nt].z : xv[nt].x, b1 = h ? xv[nt].w : xv[nt].y;
+                        mma_bf16_16816(accs[nt], a, b0, b1);
+                    }
+                }
+            }
+            ++u;
+            cons.next(warp, my_tiles, nsuper);
+        }
+        // the 16 partial tiles meet in shared memory; thread e adds output e's
+        // partials in warp order
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s_part[((warp * NT + nt) * 4 + i) * 32 + lane] = accs[nt][i];
+        __syncthreads();
+        if (threadIdx.x < NT * 128) {
+            const int e = threadIdx.x;
+            float v = 0.0f;
+#pragma unroll
+            for (int ww = 0; ww < kPWarps; ++ww) v += s_part[ww * NT * 128 + e];
+            if (r > 0) {
+                s_res[tile_i * NT * 128 + e] = v;
+            } else {
+                const int nt = e >> 7, i = (e >> 5) & 3, ln = e & 31;
+                const int64_t n = ((int64_t)blockIdx.x + (int64_t)tile_i * gridDim.x) * 16 + (ln >> 2) + 8 * (i >> 1);
+                const int m = 8 * nt + 2 * (ln & 3) + (i & 1);
+                if (n < N && m < M) y[(int64_t)m * N + n] = __float2bfloat16_rn(v);
+            }
+        }
+        __syncthreads();  // s_part is rewritten by the next tile
+    }
+    cp_async_wait_dyn(0);
+    if (r <= 0) return;
+
+    // LoRA K-extension of every tile: 2r columns, A = [B | B] (column j ->
+    // B[:, j % r]), B operand = [t_hi | t_lo], accumulated onto the kept sums.
+    // t is written by the down-projection kernel launched just before this
+    // one (programmatic dependent launch): wait for it only here.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int t2_stride = gemv_p_t2_stride(rp);
+    {
+        const int cpr = (2 * r + 7) >> 3;  // 16-byte chunks of a row of t actually read
+        for (int c = threadIdx.x; c < M * cpr; c += blockDim.x) {
+            const int tok = c / cpr, ch = c - tok * cpr;
+            cp_async<16>(t2s + tok * t2_stride + ch * 8, t2 + (int64_t)tok * rp + ch * 8, true);
+        }
+        cp_async_commit();
+        cp_async_wait_dyn(0);
+        __syncthreads();
+    }
+    for (int tile_i = warp; tile_i < my_tiles; tile_i += kPWarps) {
+        const int64_t tile = (int64_t)blockIdx.x + (int64_t)tile_i * gridDim.x;
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[nt][i] = s_res[tile_i * NT * 128 + (nt * 4 + i) * 32 + lane];
+        const int64_t row0 = tile * 16 + g, row1 = row0 + 8;
+        const bool rv0 = row0 < N, rv1 = row1 < N;
+        const uint32_t *ba = reinterpret_cast<const uint32_t *>(Bl + (rv0 ? row0 : 0) * r);
+        const uint32_t *bb = reinterpret_cast<const uint32_t *>(Bl + (rv1 ? row1 : 0) * r);
+        for (int js = 0; js < (2 * r) / 16; ++js) {
+            const int w0 = (((16 * js) % r) + 2 * tq) >> 1;
+            uint32_t a[4];
+            a[0] = rv0 ? __ldg(ba + w0) : 0u;
+            a[1] = rv1 ? __ldg(bb + w0) : 0u;
+            a[2] = rv0 ? __ldg(ba + w0 + 4) : 0u;
+            a[3] = rv1 ? __ldg(bb + w0 + 4) : 0u;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int tok = g + 8 * nt;
+                const uint32_t *tr = reinterpret_cast<const uint32_t *>(t2s + tok * t2_stride);
+                const int tw = (16 * js + 2 * tq) >> 1;
+                const uint32_t tb0 = tok < M ? tr[tw] : 0u, tb1 = tok < M ? tr[tw + 4] : 0u;
+                mma_bf16_16816(acc[nt], a, tb0, tb1);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t n = (i >> 1) ? row1 : row0;
+                const int m = 8 * nt + 2 * tq + (i & 1);
+                if (n < N && m < M) y[(int64_t)m * N + n] = __float2bfloat16_rn(acc[nt][i]);
+            }
+    }
+}
+
+template <int kMode, int NT, int kLut>
+cudaError_t launch_gemv_p(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
+                          const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
+                          void *y, cudaStream_t stream, int num_sms, int depth, size_t smem) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemv_p<kMode, NT, kLut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (N + 15) / 16;
+    const int64_t grid = tiles < num_sms ? tiles : num_sms;  // num_sms: SMs this grid may take
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kPWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = r > 0 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_gemv_p<kMode, NT, kLut>, static_cast<const __nv_bfloat16 *>(x), M, K, N,
+                              packed, q8, scales, offset, static_cast<const __nv_bfloat16 *>(B), r,
+                              static_cast<const __nv_bfloat16 *>(t2), rp, static_cast<__nv_bfloat16 *>(y), depth,
+                              (int)((tiles + grid - 1) / grid));
+}
+
+constexpr int64_t kPSmemMax = 227 * 1024;
+
+// Deepest ring (up to 8 units per warp) that fits, or 0.
+int gemv_p_depth(int M, int64_t K, int64_t N, int rp, bool smem_lut, int num_sms) {
+    const int nt = M <= 8 ? 1 : 2;
+    const int64_t tiles = (N + 15) / 16;
+    const int64_t grid = tiles < num_sms ? tiles : num_sms;
+    const int64_t mt = (tiles + grid - 1) / grid;
+    if (mt > (1 << 20)) return 0;
+    for (int d = 8; d >= 2; --d)
+        if (gemv_p_layout(M, K, rp, nt, smem_lut, d, (int)mt).total <= kPSmemMax) return d;
+    return 0;
+}
+
+// Which GEMV runs: 0 = persistent, with the pair table where a ring of at
+// least 3 units still fits, else with the register table; 1 = persistent,
+// register table only; 2 = always the per-tile kernel; 3 = as 0 with the
+// mixed lookup instead of the pair table.
+#ifndef NF4_GEMV_P_MODE
+#define NF4_GEMV_P_MODE 0
+#endif
+#ifndef NF4_GEMV_P_MIN_M
+#define NF4_GEMV_P_MIN_M 9
+#endif
+
 template <int kMode>
 cudaError_t launch_gemv_mode(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                              const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
-                             void *y, cudaStream_t stream) {
+                             void *y, cudaStream_t stream, int num_sms) {
+    // Persistent kernel for M >= NF4_GEMV_P_MIN_M when x fits in shared
+    // memory (below that the per-tile kernel, with more warps in flight,
+    // is faster).  With LoRA one SM is
+    // left to the down-projection that runs alongside (one CTA, whose
+    // registers would not fit beside a persistent CTA).
+    const int sms = r > 0 && num_sms > 1 ? num_sms - 1 : num_sms;
+    if (NF4_GEMV_P_MODE != 2 && K % 256 == 0 && M >= NF4_GEMV_P_MIN_M) {
+        constexpr bool kTryPair = NF4_GEMV_P_MODE == 0 || NF4_GEMV_P_MODE == 3;
+        constexpr int kPairLut = NF4_GEMV_P_MODE == 3 ? 2 : 1;
+        const int d_pair = kTryPair ? gemv_p_depth(M, K, N, rp, true, sms) : 0;
+        const int d_reg = gemv_p_depth(M, K, N, rp, false, sms);
+        const int nt = M <= 8 ? 1 : 2;
+        if (d_pair >= 3 || d_reg >= 2) {
+            const bool pair = d_pair >= 3;
+            const int d = pair ? d_pair : d_reg;
+            const int64_t tiles = (N + 15) / 16, grid = tiles < sms ? tiles : sms;
+            const size_t smem = (size_t)gemv_p_layout(M, K, rp, nt, pair, d, (int)((tiles + grid - 1) / grid)).total;
+            if (nt == 1)
+                return pair ? launch_gemv_p<kMode, 1, kPairLut>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp,
+                                                                y, stream, sms, d, smem)
+                            : launch_gemv_p<kMode, 1, 0>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y,
+                                                         stream, sms, d, smem);
+            return pair ? launch_gemv_p<kMode, 2, kPairLut>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y,
+                                                            stream, sms, d, smem)
+                        : launch_gemv_p<kMode, 2, 0>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream,
+                                                     sms, d, smem);
+        }
+    }
     auto *xp = static_cast<const __nv_bfloat16 *>(x);
     auto *bp = static_cast<const __nv_bfloat16 *>(B);
     auto *tp = static_cast<const __nv_bfloat16 *>(t2);
@@ -252,9 +681,9 @@ cudaError_t launch_gemv_mode(const void *x, int M, int64_t K, int64_t N, const u
     cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
     cfg.dynamicSmemBytes = kGemvSmemLut ? kPairTableFloat2 * sizeof(float2) : 0;
     if (M <= 8)
-        return cudaLaunchKernelEx(&cfg, k_gemv<kMode, 1, 1, kGemvSmemLut>, xp, M, K, N, packed, q8, scales, offset, bp,
+        return cudaLaunchKernelEx(&cfg, k_gemv<kMode, 1, 1, kGemvLut>, xp, M, K, N, packed, q8, scales, offset, bp,
                                   r, tp, rp, yp);
-    return cudaLaunchKernelEx(&cfg, k_gemv<kMode, 2, 2, kGemvSmemLut>, xp, M, K, N, packed, q8, scales, offset, bp, r,
+    return cudaLaunchKernelEx(&cfg, k_gemv<kMode, 2, 2, kGemvLut>, xp, M, K, N, packed, q8, scales, offset, bp, r,
                               tp, rp, yp);
 }
 
@@ -262,10 +691,12 @@ cudaError_t launch_gemv_mode(const void *x, int M, int64_t K, int64_t N, const u
 
 cudaError_t launch_gemv(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                         const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
-                        void *y, cudaStream_t stream) {
-    if (q8 == nullptr) return launch_gemv_mode<2>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream);
-    if (offset == nullptr) return launch_gemv_mode<1>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream);
-    return launch_gemv_mode<0>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream);
+                        void *y, cudaStream_t stream, int num_sms) {
+    if (q8 == nullptr)
+        return launch_gemv_mode<2>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream, num_sms);
+    if (offset == nullptr)
+        return launch_gemv_mode<1>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream, num_sms);
+    return launch_gemv_mode<0>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream, num_sms);
 }
 
 }  // namespace nf4

@@ -10,7 +10,7 @@ cudaError_t launch_lora_down(const void *x, const void *A, int64_t M, int64_t K,
                              cudaStream_t stream);
 cudaError_t launch_gemv(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                         const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
-                        void *y, cudaStream_t stream);
+                        void *y, cudaStream_t stream, int num_sms);
 cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
                                 unsigned *err, cudaStream_t stream);
 cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
@@ -50,7 +50,7 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
         if (e != cudaSuccess) return e;
     }
     if (M <= kGemvMaxTokens)
-        return launch_gemv(x, (int)M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream);
+        return launch_gemv(x, (int)M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms);
     return launch_gemm_tc(x, M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms,
                           err_word);
 }

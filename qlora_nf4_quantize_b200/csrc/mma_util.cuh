@@ -110,9 +110,17 @@ __device__ __forceinline__ void fill_pair_table(float2 *tbl) {
 // Two bf16 weights of one packed byte: RNE_bf16(RN_f32(q * c)) for both
 // nibbles, returned as a bf16x2 word (element 2j in the low half).
 // tbl_lane = table + (lane & 15).
+// The two products are one packed f32x2 multiply (each lane rounded to
+// nearest, as two binary32 multiplies).
 __device__ __forceinline__ uint32_t pair_lookup(const float2 *tbl_lane, uint32_t byte, float c) {
     const float2 q = tbl_lane[byte * kPairCopies];
-    return pack_bf16x2(__fmul_rn(q.x, c), __fmul_rn(q.y, c));
+    uint64_t qq, cc, d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(qq) : "f"(q.x), "f"(q.y));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(qq), "l"(cc));
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+    return pack_bf16x2(lo, hi);
 }
 
 // Same four-code lookup as lut_lookup4 (same output layout) through the
@@ -121,6 +129,39 @@ __device__ __forceinline__ void pair_lookup4(const float2 *tbl_lane, uint32_t p1
                                              uint32_t &w23) {
     w01 = pair_lookup(tbl_lane, __byte_perm(p16, 0u, 0x4440), c);
     w23 = pair_lookup(tbl_lane, __byte_perm(p16, 0u, 0x4441), c);
+}
+
+// pair_lookup4 with the table addressed by a 32-bit shared-memory address
+// (base_lane = shared address of table + (lane & 15)) and c given as the
+// packed pair (c, c): per byte one byte permute, one multiply-add for the
+// address, one 64-bit shared load, one packed f32x2 multiply (each half
+// rounded to nearest) and one conversion to bf16x2.
+__device__ __forceinline__ void pair_lookup4_s(uint32_t base_lane, uint32_t p16, uint64_t cc, uint32_t &w01,
+                                               uint32_t &w23) {
+    asm("{\n\t"
+        ".reg .b32 b0, b1, l0, h0, l1, h1;\n\t"
+        ".reg .b64 q0, q1;\n\t"
+        "prmt.b32 b0, %2, 0, 0x4440;\n\t"
+        "prmt.b32 b1, %2, 0, 0x4441;\n\t"
+        "mad.lo.u32 b0, b0, %5, %3;\n\t"
+        "mad.lo.u32 b1, b1, %5, %3;\n\t"
+        "ld.shared.b64 q0, [b0];\n\t"
+        "ld.shared.b64 q1, [b1];\n\t"
+        "mul.rn.f32x2 q0, q0, %4;\n\t"
+        "mul.rn.f32x2 q1, q1, %4;\n\t"
+        "mov.b64 {l0, h0}, q0;\n\t"
+        "mov.b64 {l1, h1}, q1;\n\t"
+        "cvt.rn.bf16x2.f32 %0, h0, l0;\n\t"
+        "cvt.rn.bf16x2.f32 %1, h1, l1;\n\t"
+        "}"
+        : "=r"(w01), "=r"(w23)
+        : "r"(p16), "r"(base_lane), "l"(cc), "n"(kPairCopies * 8));
+}
+
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
 }
 
 }  // namespace nf4

@@ -50,7 +50,9 @@ def test_decode_gemv_full_size(nf4lib, oracle_mod, cuda_device, case):
 
 
 @pytest.mark.parametrize("M,K,N,r,dq", [(1, 192, 200, 16, True), (7, 64, 40, 32, True), (16, 320, 96, 64, False),
-                                        (9, 1024, 8, 16, True), (16, 4096, 1000, 0, True)])
+                                        (9, 1024, 8, 16, True), (16, 4096, 1000, 0, True),
+                                        (3, 256, 24, 64, False), (5, 768, 4000, 32, True),
+                                        (12, 512, 2400, 16, False), (8, 8192, 520, 64, True)])
 def test_gemv_ragged_shapes(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
     c = wl.LinearCase("ragged", M, K, N, r, 1.5, 31 + M + K + N)
     W, x, A, B = wl.linear_inputs(c, with_lora=r > 0)
@@ -59,6 +61,20 @@ def test_gemv_ragged_shapes(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
     dB = None if B is None else B.to(cuda_device)
     y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, N, dA, dB,
                                    c.scaling)
+    torch.cuda.synchronize()
+    check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
+
+
+@pytest.mark.parametrize("M,K,N,r", [(1, 512, 2400, 16), (13, 256, 200, 64), (4, 192, 64, 32), (40, 512, 264, 16)])
+def test_linear_double_quant_without_centring(nf4lib, oracle_mod, cuda_device, M, K, N, r):
+    """Block constants decoded as E4M3 * c2 (no centring offset), through
+    the persistent GEMV, the per-tile GEMV and the tensor-core GEMM."""
+    c = wl.LinearCase("no centring", M, K, N, r, 1.25, 211 + M + K + N)
+    W, x, A, B = wl.linear_inputs(c)
+    st = nf4lib.quantize_weight(W.to(cuda_device), centre=False)
+    assert st.offset is None
+    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, N,
+                                   A.to(cuda_device), B.to(cuda_device), c.scaling)
     torch.cuda.synchronize()
     check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
 
