@@ -434,17 +434,35 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUte
 // ---------------------------------------------------------------------------
 // LoRA down-projection for large M on the tensor cores:
 //   t = s x A^T,  x [M, K] bf16,  A [r, K] bf16,  t as [t_hi | t_lo | 0] bf16
-// (same output as the warp-MMA kernel in lora_down.cu).  A CTA owns 128 rows
-// of x: D[128, r] += X[128, k] A[r, k]^T with both operands brought by TMA
-// (128-byte swizzle, kDownStages-deep ring) and one thread issuing the MMAs
-// (M = 128, N = r, K = 16) into r fp32 columns of tensor memory; the four
-// warps then read one token row per thread and write its hi/lo pair.
-constexpr int kDownStages = 4;
+// (same output as the warp-MMA kernel in lora_down.cu).  A thread-block
+// cluster of kDownSplit CTAs (1, 2 or 4) owns 128 rows of x and splits K: CTA c runs the
+// k-steps [c kt / kDownSplit, (c + 1) kt / kDownSplit) as
+// D[128, r] += X[128, k] A[r, k]^T with both operands brought by TMA (128-byte
+// swizzle, kDownStages-deep ring) and one thread issuing the MMAs (M = 128,
+// N = r, K = 16) into r fp32 columns of its tensor memory.  Each CTA then
+// stages its partial tile in shared memory, and CTA c finishes rows
+// [128 c / kDownSplit, 128 (c + 1) / kDownSplit) of the tile: it adds the
+// kDownSplit partials in rank order
+// through distributed shared memory (so the result does not depend on
+// timing), scales, and writes the hi/lo pair.
+// The kernel runs alongside the fused GEMM (programmatic dependent launch),
+// so what it costs the GEMM is SMs x time: one CTA per 128 rows with a deep
+// ring (no split) takes the fewest SM-microseconds; splitting K over a
+// cluster shortens the kernel but holds more SMs.
+#ifndef NF4_DOWN_STAGES
+#define NF4_DOWN_STAGES 8
+#endif
+#ifndef NF4_DOWN_SPLIT
+#define NF4_DOWN_SPLIT 1
+#endif
+constexpr int kDownStages = NF4_DOWN_STAGES;
 constexpr int kDownRows = 128;
+constexpr int kDownSplit = NF4_DOWN_SPLIT;  // cluster size along K
+static_assert(kDownSplit == 1 || kDownSplit == 2 || kDownSplit == 4, "128 rows split evenly over the cluster");
 
 template <int kR>
 struct __align__(1024) DownSmem {
-    uint8_t x[kDownStages][kDownRows * 128];
+    uint8_t x[kDownStages][kDownRows * 128];  // after the main loop: the fp32 partial tile [kR][128]
     uint8_t a[kDownStages][kR * 128];
     uint64_t full[kDownStages];
     uint64_t empty[kDownStages];
@@ -452,6 +470,7 @@ struct __align__(1024) DownSmem {
     uint32_t tmem_base;
     int abort;
 };
+static_assert(kDownStages * kDownRows * 128 >= 64 * kDownRows * 4, "partial tile fits in the x ring");
 
 __device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -461,6 +480,29 @@ __device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// address of the same shared-memory location in cluster CTA `rank`
+__device__ __forceinline__ uint32_t map_rank(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
 }
 
 template <int kR>
@@ -479,8 +521,11 @@ __global__ void __launch_bounds__(128, 1)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m0 = (int64_t)blockIdx.x * kDownRows;
-    const int kt_total = (int)(K / 64);
+    const uint32_t rank = cluster_rank();
+    const int64_t m0 = (int64_t)blockIdx.y * kDownRows;
+    const int kt_all = (int)(K / 64);
+    const int kt_begin = (int)((int64_t)rank * kt_all / kDownSplit);
+    const int kt_total = (int)((int64_t)(rank + 1) * kt_all / kDownSplit) - kt_begin;
     if (threadIdx.x == 0) {
         for (int st = 0; st < kDownStages; ++st) {
             mbar_init(&S.full[st], 1);
@@ -503,15 +548,15 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t tmem = S.tmem_base;
 
     bool ok = true;
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && kt_total > 0) {
         // producer and MMA issuer in one thread: loads run kDownStages - 1 ahead
         auto issue = [&](int kt) -> bool {
             const int st = kt % kDownStages;
             const uint32_t ph = (uint32_t)(kt / kDownStages) & 1u;
             if (!mbar_wait(&S.empty[st], ph ^ 1u, abort, err)) return false;
             mbar_arrive_expect_tx(&S.full[st], kStageBytes);
-            tma_load_2d(S.x[st], &tmap_x, &S.full[st], kt * 64, (int)m0);
-            tma_load_2d(S.a[st], &tmap_a, &S.full[st], kt * 64, 0);
+            tma_load_2d(S.x[st], &tmap_x, &S.full[st], (kt_begin + kt) * 64, (int)m0);
+            tma_load_2d(S.a[st], &tmap_a, &S.full[st], (kt_begin + kt) * 64, 0);
             return true;
         };
         int issued = 0;
@@ -544,38 +589,69 @@ __global__ void __launch_bounds__(128, 1)
         }
     }
     __syncwarp();
-    // epilogue: thread = token row m0 + 32 warp + lane, r fp32 columns
-    if (__all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err))) {
-        tc_fence_after();
-        const int64_t m = m0 + 32 * warp + lane;
-        const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
+    // this CTA's partial tile -> shared memory, column-major [kR][128] fp32
+    // (the x ring is free: every MMA that read it has completed)
+    float *part = reinterpret_cast<float *>(&S.x[0][0]);
+    const int row = 32 * warp + lane;  // tensor-memory lane = tile row
+    if (kt_total > 0) {
+        if (__all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err))) {
+            tc_fence_after();
+            const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
-        for (int c0 = 0; c0 < kR; c0 += 16) {
-            uint32_t v[32];
-            tc_load32(taddr + (uint32_t)(c0 & ~31), v);  // 32 columns (the allocation holds at least 32)
-            tc_wait_ld();
-            if (m < M) {
-                uint32_t hi[8], lo[8];
+            for (int c0 = 0; c0 < (int)kCols; c0 += 32) {
+                uint32_t v[32];
+                tc_load32(taddr + (uint32_t)c0, v);
+                tc_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float a0 = __uint_as_float(v[(c0 & 31) + 2 * j]) * scaling;
-                    const float a1 = __uint_as_float(v[(c0 & 31) + 2 * j + 1]) * scaling;
-                    const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
-                    hi[j] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-                    lo[j] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
-                }
-                uint4 *th = reinterpret_cast<uint4 *>(t2 + m * rp + c0);
-                uint4 *tl = reinterpret_cast<uint4 *>(t2 + m * rp + kR + c0);
-                th[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                th[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-                tl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                tl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+                for (int j = 0; j < 32; ++j)
+                    if (c0 + j < kR) part[(c0 + j) * kDownRows + row] = __uint_as_float(v[j]);
             }
         }
-        if (m < M)
+    } else {
+        for (int c = 0; c < kR; ++c) part[c * kDownRows + row] = 0.0f;  // no k-steps: a zero partial
+    }
+    cluster_sync_all();  // every CTA's partial is complete and visible in the cluster
+    // finish rows [kRowsPer rank, kRowsPer (rank + 1)): thread t takes row
+    // kRowsPer rank + t % kRowsPer and the kCw columns of group t / kRowsPer
+    {
+        constexpr int kRowsPer = kDownRows / kDownSplit;
+        constexpr int kCw = kR / (128 / kRowsPer);  // columns per thread (>= 4)
+        static_assert(kCw % 4 == 0, "whole 4-column chunks");
+        const int t = threadIdx.x;
+        const int r_loc = kRowsPer * (int)rank + t % kRowsPer;
+        const int64_t m = m0 + r_loc;
+        const int cb = (t / kRowsPer) * kCw;
+        uint32_t base[kDownSplit];
+#pragma unroll
+        for (int c = 0; c < kDownSplit; ++c) base[c] = map_rank(part + cb * kDownRows + r_loc, (uint32_t)c);
+#pragma unroll 1
+        for (int j0 = 0; j0 < kCw; j0 += 4) {
+            float v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float a = 0.0f;
+#pragma unroll
+                for (int c = 0; c < kDownSplit; ++c)
+                    a += ld_cluster_f32(base[c] + (uint32_t)((j0 + j) * kDownRows * 4));
+                v[j] = a * scaling;
+            }
+            if (m < M) {
+                uint32_t hi[2], lo[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * j]), h1 = __float2bfloat16_rn(v[2 * j + 1]);
+                    hi[j] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+                    lo[j] = pack_bf16x2(v[2 * j] - __bfloat162float(h0), v[2 * j + 1] - __bfloat162float(h1));
+                }
+                *reinterpret_cast<uint2 *>(t2 + m * rp + cb + j0) = make_uint2(hi[0], hi[1]);
+                *reinterpret_cast<uint2 *>(t2 + m * rp + kR + cb + j0) = make_uint2(lo[0], lo[1]);
+            }
+        }
+        if (m < M && cb == 0)
             for (int j = 2 * kR; j < rp; j += 8)
                 *reinterpret_cast<uint4 *>(t2 + m * rp + j) = make_uint4(0u, 0u, 0u, 0u);
     }
+    cluster_sync_all();  // no CTA leaves while another may still read its partial
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -591,9 +667,19 @@ cudaError_t launch_down_tc(const CUtensorMap &mx, const CUtensorMap &ma, int64_t
     const size_t smem = sizeof(DownSmem<kR>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_lora_down_tc<kR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)((M + kDownRows - 1) / kDownRows);
-    k_lora_down_tc<kR><<<grid, 128, smem, stream>>>(mx, ma, M, K, s, static_cast<__nv_bfloat16 *>(t2), rp, err);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kDownSplit, (unsigned)((M + kDownRows - 1) / kDownRows));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kDownSplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_lora_down_tc<kR>, mx, ma, M, K, s, static_cast<__nv_bfloat16 *>(t2), rp, err);
 }
 
 }  // namespace
