@@ -386,6 +386,208 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ isolated per-call suite
+def graph_us(fn, reps, warm=3, trials=3):
+    """Median over `trials` of the per-call time (us) of `reps` calls of
+    `fn` captured in one CUDA graph and replayed (no launch gaps)."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(trials):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        g.replay()
+        e.record()
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e) * 1e3 / reps)
+    del g
+    return sorted(times)[len(times) // 2]
+
+
+def run_suite(args):
+    """Every call of the path timed in isolation (CUDA graphs, inputs rotating
+    over copies larger than L2), with and without double quantization, plus
+    the 8B-shaped whole-model sweep and one decoder layer's linears through
+    the fused NF4 path against unquantized bf16 LoRA GEMMs (torch.matmul on
+    cuBLAS).  One JSON line per measurement on rank 0."""
+    import torch
+    import nf4_workloads as wl
+    import qlora_nf4_quantize_b200 as q
+
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    q.lib()
+    peaks = measured_peaks()
+
+    def emit(name, us, work, unit, **extra):
+        if unit == "GB/s":
+            ach, peak = work / (us * 1e-6) / 1e9, peaks["hbm_gbs"]
+        else:
+            ach, peak = work / (us * 1e-6) / 1e12, peaks["bf16_tflops"]
+        line = {"suite": name, "us": round(us, 3), "achieved": round(ach, 2), "unit": unit, "peak": peak,
+                "frac": round(ach / peak, 4), "work_per_call": work, "timing": "CUDA graph, isolated call"}
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+
+    rot = [0]
+
+    def nxt(c):
+        rot[0] += 1
+        return rot[0] % c
+
+    # ---- projection 4096x4096 bf16: quantize, double-quantize, dequantize (with / without DQ)
+    wp = wl.weight_case(wl.PROJECTION).to(dev).reshape(-1)
+    n, C = wp.numel(), 6
+    nb = n // BLOCK
+    Ws = [wp.clone() for _ in range(C)]
+    sts = [q.quantize_weight(w) for w in Ws]
+    raw = [q.nf4_quantize(w) for w in Ws[:C]]  # (packed, fp32 absmax): the no-DQ state
+    absb = [torch.empty(nb, device=dev) for _ in range(C)]
+    outs = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(C)]
+    outs32 = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(C)]
+    q8s = [torch.empty(nb, dtype=torch.uint8, device=dev) for _ in range(C)]
+    c2s = [torch.empty(-(-nb // DQ_BLOCK), device=dev) for _ in range(C)]
+    offs = [torch.empty(1, device=dev) for _ in range(C)]
+    ws = torch.empty(q.nf4_double_quantize_workspace_size(nb), dtype=torch.uint8, device=dev)
+
+    def f_quant():
+        k = nxt(C)
+        q.nf4_quantize(Ws[k], packed=sts[k].packed, absmax=absb[k])
+
+    def f_dq():
+        k = nxt(C)
+        q.nf4_double_quantize(absb[k], absmax_q=q8s[k], absmax2=c2s[k], offset=offs[k], workspace=ws)
+
+    def f_deq(dq, f32):
+        def f():
+            k = nxt(C)
+            o = outs32[k] if f32 else outs[k]
+            if dq:
+                st = sts[k]
+                q.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, n,
+                                 torch.float32 if f32 else torch.bfloat16, out=o)
+            else:
+                q.nf4_dequantize(raw[k][0], None, raw[k][1], None, n, torch.float32 if f32 else torch.bfloat16,
+                                 out=o)
+        return f
+
+    proj = "projection 4096x4096 bf16"
+    emit(f"quantize {proj}", graph_us(f_quant, 20), quantize_bytes(n), "GB/s")
+    emit(f"double_quantize {nb} constants", graph_us(f_dq, 20), dq_bytes(nb), "GB/s")
+    emit(f"dequantize {proj} -> bf16, DQ", graph_us(f_deq(True, False), 20), dequant_bytes(n), "GB/s")
+    emit(f"dequantize {proj} -> fp32, DQ", graph_us(f_deq(True, True), 20), dequant_bytes(n, 4), "GB/s")
+    nodq_b = n // 2 + nb * 4 + n * 2
+    emit(f"dequantize {proj} -> bf16, no DQ (fp32 c1)", graph_us(f_deq(False, False), 20), nodq_b, "GB/s",
+         bytes_per_param=round(nodq_b / n - 2, 6))
+    del Ws, sts, raw, absb, outs, outs32, q8s, c2s, offs
+    torch.cuda.empty_cache()
+
+    # ---- fused linear: decode GEMV and tensor-core GEMM, with / without DQ
+    def linear_case(c, dq, copies, reps):
+        W, x, A, B = wl.linear_inputs(c)
+        Wd = W.to(dev)
+        stl = [q.quantize_weight(Wd, double_quant=dq) for _ in range(copies)]
+        del W, Wd
+        xd, Ad, Bd = x.to(dev), A.to(dev), B.to(dev)
+        y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+        wsl = torch.empty(max(1, q.nf4_lora_linear_workspace_size(c.M, c.r)), dtype=torch.uint8, device=dev)
+
+        def f():
+            st = stl[nxt(copies)]
+            q.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, Ad, Bd, c.scaling,
+                                  y=y, workspace=wsl)
+        us = graph_us(f, reps)
+        q.nf4_device_status()
+        wb = c.N * c.K // 2 + (c.N * c.K // BLOCK) * (1 if dq else 4) + (-(-(c.N * c.K // BLOCK) // DQ_BLOCK) * 4 + 4
+                                                                          if dq else 0)
+        byts = wb + c.M * c.K * 2 + c.r * c.K * 2 + c.N * c.r * 2 + c.M * c.N * 2
+        return us, byts
+
+    for c in wl.GEMV_CASES:
+        for dq in (True, False):
+            us, byts = linear_case(c, dq, 8, 20)
+            emit(f"{c.name}{'' if dq else ', no DQ'}", us, byts, "GB/s",
+                 tflops=round(linear_flops(c.M, c.K, c.N, c.r) / (us * 1e-6) / 1e12, 3))
+    for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
+        for dq in (True, False):
+            us, _ = linear_case(c, dq, 1, 5)
+            emit(f"{c.name}{'' if dq else ', no DQ'}", us, linear_flops(c.M, c.K, c.N, c.r), "TFLOP/s",
+                 peak_sustained=peaks["bf16_tflops_sustained"])
+    torch.cuda.empty_cache()
+
+    # ---- one 8B-shaped decoder layer, M = 4096 tokens, r = 64, s = 0.25:
+    # fused NF4 + LoRA against bf16 x W^T + s (x A^T) B^T on cuBLAS
+    M, r, sc = 4096, 64, 0.25
+    t_nf4 = t_bf16 = 0.0
+    flops = 0
+    for idx, (name, N, K) in enumerate(wl.LAYER_8B):
+        W = wl.sweep_weight(0, idx).to(dev)
+        g = torch.Generator().manual_seed(wl.sweep_seed(0, idx) + 1)
+        x = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
+        A = (torch.randn(r, K, generator=g) * 0.01).to(torch.bfloat16).to(dev)
+        B = (torch.randn(N, r, generator=g) * 0.01).to(torch.bfloat16).to(dev)
+        st = q.quantize_weight(W)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        wsl = torch.empty(q.nf4_lora_linear_workspace_size(M, r), dtype=torch.uint8, device=dev)
+        Wt, At, Bt = W.t(), A.t(), B.t()
+
+        def f_nf4():
+            q.nf4_lora_linear_fwd(x, st.packed, st.absmax_q, st.absmax2, st.offset, N, A, B, sc, y=y, workspace=wsl)
+
+        def f_bf16():
+            yb = torch.matmul(x, Wt)
+            torch.addmm(yb, torch.matmul(x, At), Bt, alpha=sc, out=y)
+
+        a_us, b_us = graph_us(f_nf4, 3), graph_us(f_bf16, 3)
+        fl = linear_flops(M, K, N, r)
+        emit(f"layer {name} {N}x{K} M={M} r={r}: fused NF4+LoRA", a_us, fl, "TFLOP/s",
+             bf16_lora_us=round(b_us, 3), ratio_nf4_over_bf16=round(a_us / b_us, 4))
+        t_nf4, t_bf16, flops = t_nf4 + a_us, t_bf16 + b_us, flops + fl
+        del W, x, A, B, st, y, wsl
+    emit(f"8B decoder layer (7 linears) M={M} r={r}: fused NF4+LoRA", t_nf4, flops, "TFLOP/s",
+         bf16_lora_us=round(t_bf16, 3), overhead_vs_bf16=round(t_nf4 / t_bf16 - 1, 4),
+         note="forward linears only; the pages' 25-40 % slowdown figure is per training step")
+    torch.cuda.empty_cache()
+
+    # ---- 8B-shaped whole-model sweep: quantize + DQ + dequantize of every
+    # linear weight, layer by layer (layer 0's seeded weights stand in for all
+    # 32 layers: the same shapes and work; 224 weights, 6.98e9 parameters)
+    Wl = [wl.sweep_weight(0, idx).to(dev).reshape(-1) for idx in range(len(wl.LAYER_8B))]
+    bufs = []
+    for w in Wl:
+        m = w.numel()
+        mb = m // BLOCK
+        bufs.append((torch.empty(m // 2, dtype=torch.uint8, device=dev), torch.empty(mb, device=dev),
+                     torch.empty(mb, dtype=torch.uint8, device=dev), torch.empty(-(-mb // DQ_BLOCK), device=dev),
+                     torch.empty(1, device=dev),
+                     torch.empty(q.nf4_double_quantize_workspace_size(mb), dtype=torch.uint8, device=dev),
+                     torch.empty(m, dtype=torch.bfloat16, device=dev)))
+
+    def f_layer():
+        for w, (pk, ab, q8, c2, off, wsd, out) in zip(Wl, bufs):
+            m = w.numel()
+            q.nf4_quantize(w, packed=pk, absmax=ab)
+            q.nf4_double_quantize(ab, absmax_q=q8, absmax2=c2, offset=off, workspace=wsd)
+            q.nf4_dequantize(pk, q8, c2, off, m, torch.bfloat16, out=out)
+
+    layer_us = graph_us(f_layer, 4)
+    per_layer = sum(quantize_bytes(w.numel()) + dq_bytes(w.numel() // BLOCK) + dequant_bytes(w.numel()) for w in Wl)
+    L = wl.N_LAYERS_8B
+    emit(f"8B-shaped sweep: quantize + DQ + dequantize, {L} layers x 7 linears", layer_us * L, per_layer * L,
+         "GB/s", params=sum(w.numel() for w in Wl) * L, seconds=round(layer_us * L * 1e-6, 4))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -393,11 +595,16 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--suite", action="store_true",
+                    help="time every call in isolation (no-DQ variant, sweep, decoder layer); one line each")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.suite:
+        run_suite(args)
         return
     run_ours(args)
     rank, world, _ = dist_env()

@@ -208,6 +208,17 @@ NF4_API nf4_status nf4_lora_linear_fwd_noalloc(const void *x, int64_t M, int64_t
  * NF4_ERR_CUDA on a CUDA error, NF4_OK otherwise. */
 NF4_API nf4_status nf4_device_status(void *stream);
 
+/* nf4_selftest_wait_timeout -- failure-detection check (no counterpart on
+ * the pages).  Launches on `stream` one thread that waits on a shared-memory
+ * mbarrier nothing arrives on; after limit_ns nanoseconds of %globaltimer
+ * (1 <= limit_ns <= 1e9) it raises the device error word and returns, as the
+ * fused kernels do when one of their bounded waits expires.  The GPU is
+ * neither faulted nor hung and the context stays usable.  Returns NF4_OK once
+ * launched (NF4_ERR_INVALID for a limit out of range, NF4_ERR_CUDA on a launch
+ * error); the following nf4_device_status() returns NF4_ERR_TIMEOUT and
+ * clears the word. */
+NF4_API nf4_status nf4_selftest_wait_timeout(int64_t limit_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,6 +25,7 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
                                cudaStream_t stream, int num_sms, unsigned *err_word);
 int64_t lora_workspace_bytes(int64_t M, int r);
 unsigned *device_error_word(cudaError_t *status);
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream);
 }  // namespace nf4
 
 namespace {
@@ -162,6 +163,11 @@ nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N, c
     return cuda_status(nf4::launch_lora_linear(x, M, K, N, packed, absmax_q, absmax2, offset, lora ? A : nullptr,
                                                lora ? B : nullptr, lora ? r : 0, scaling, y, workspace,
                                                (cudaStream_t)stream, sms, err));
+}
+
+nf4_status nf4_selftest_wait_timeout(int64_t limit_ns, void *stream) {
+    if (limit_ns < 1 || limit_ns > 1000000000) return NF4_ERR_INVALID;
+    return cuda_status(nf4::launch_selftest_wait((unsigned long long)limit_ns, (cudaStream_t)stream));
 }
 
 nf4_status nf4_device_status(void *stream) {

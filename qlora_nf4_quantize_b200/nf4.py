@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
     L.nf4_lora_linear_fwd_noalloc.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, i32, f32, P, P]
     L.nf4_device_status.restype = i32
     L.nf4_device_status.argtypes = [P]
+    L.nf4_selftest_wait_timeout.restype = i32
+    L.nf4_selftest_wait_timeout.argtypes = [i64, P]
     _lib = L
     return L
 
@@ -221,6 +223,12 @@ def nf4_device_status(stream=None) -> int:
     st = lib().nf4_device_status(_stream(stream))
     _check("nf4_device_status", st)
     return st
+
+
+def nf4_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launch the bounded-wait check (a wait that expires after limit_ns);
+    the next nf4_device_status() raises Nf4Error with NF4_ERR_TIMEOUT."""
+    _check("nf4_selftest_wait_timeout", lib().nf4_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 @dataclass

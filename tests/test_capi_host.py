@@ -40,6 +40,12 @@ def test_codebook_call_matches_oracle(nf4lib, oracle_mod):
     assert np.array_equal(got, oracle_mod.codebook())
 
 
+def test_selftest_limit_checked_on_the_host(nf4lib):
+    L = nf4lib.lib()
+    for bad in (0, -5, 1000000001):
+        assert L.nf4_selftest_wait_timeout(bad, None) == 1  # NF4_ERR_INVALID, nothing launched
+
+
 def test_host_validation_before_any_device_work(nf4lib):
     L = nf4lib.lib()
     fake = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
