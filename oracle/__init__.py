@@ -74,6 +74,10 @@ def lib() -> ctypes.CDLL:
             L.nf4o_dequantize_bf16.argtypes = [P, P, P, P, i64, ctypes.c_int, ctypes.c_int, P]
             L.nf4o_lora_linear.argtypes = [P, i64, i64, i64, P, P, P, P, ctypes.c_int, ctypes.c_int,
                                            P, P, ctypes.c_int, ctypes.c_float, P, i64, P]
+            L.nf4o_merge_weight.argtypes = [P, P, P, P, i64, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int,
+                                            ctypes.c_float, i64, i64, P]
+            L.nf4o_merge_requantize.argtypes = [P, P, P, P, i64, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int,
+                                                ctypes.c_float, i64, i64, P, P]
             L.nf4o_e4m3_encode_array.argtypes = [P, i64, P]
             L.nf4o_f32_to_bf16_array.argtypes = [P, i64, P]
             L.nf4o_code_of_array.argtypes = [P, i64, P]
@@ -230,3 +234,44 @@ def lora_linear(x_bf16, K, N, packed, codes, scales, offset, A_bf16, B_bf16, r, 
                            blocksize, dq_blocksize, _ptr(A), _ptr(B), int(r if A is not None else 0),
                            float(s), _ptr(rows), rows.size, _ptr(y))
     return y
+
+
+def _merge_args(packed, codes, scales, offset, K, A_bf16, B_bf16, r):
+    packed = np.ascontiguousarray(packed, np.uint8)
+    scales = np.ascontiguousarray(scales, np.float32)
+    codes = None if codes is None else np.ascontiguousarray(codes, np.uint8)
+    off = None if offset is None else np.array([offset], np.float32)
+    A = np.ascontiguousarray(A_bf16, np.uint16).reshape(r, K)
+    B = np.ascontiguousarray(B_bf16, np.uint16).reshape(-1, r)
+    return packed, codes, scales, off, A, B
+
+
+def merge_weight(packed, codes, scales, offset, K, A_bf16, B_bf16, r, s, row0=0, nrows=None,
+                 blocksize: int = BLOCKSIZE, dq_blocksize: int = DQ_BLOCKSIZE):
+    """W' = fma(s, d, w~) with d the fixed-order binary32 fma chain of
+    B[n, :] A[:, k] (the merge reading of nf4o_merge_weight), rows
+    [row0, row0 + nrows) of W[N, K]; float32 [nrows, K].
+    Pinned by the delta against an fp64 matmul, the s = 0 identity, and an
+    exact-rational re-evaluation of the chain on a tiny case."""
+    packed, codes, scales, off, A, B = _merge_args(packed, codes, scales, offset, K, A_bf16, B_bf16, r)
+    N = B.shape[0]
+    nrows = N - row0 if nrows is None else nrows
+    out = np.empty((nrows, K), np.float32)
+    lib().nf4o_merge_weight(_ptr(packed), _ptr(codes), _ptr(scales), _ptr(off), int(K), blocksize, dq_blocksize,
+                            _ptr(A), _ptr(B), int(r), float(s), int(row0), int(nrows), _ptr(out))
+    return out
+
+
+def merge_requantize(packed, codes, scales, offset, K, A_bf16, B_bf16, r, s, row0=0, nrows=None,
+                     blocksize: int = BLOCKSIZE, dq_blocksize: int = DQ_BLOCKSIZE):
+    """merge_weight's rows quantized again (blockwise NF4, fp32 constants):
+    (packed uint8 [nrows K / 2], absmax float32 [nrows K / 64])."""
+    packed, codes, scales, off, A, B = _merge_args(packed, codes, scales, offset, K, A_bf16, B_bf16, r)
+    N = B.shape[0]
+    nrows = N - row0 if nrows is None else nrows
+    pk = np.empty(nrows * K // 2, np.uint8)
+    ab = np.empty(nrows * K // blocksize, np.float32)
+    lib().nf4o_merge_requantize(_ptr(packed), _ptr(codes), _ptr(scales), _ptr(off), int(K), blocksize,
+                                dq_blocksize, _ptr(A), _ptr(B), int(r), float(s), int(row0), int(nrows), _ptr(pk),
+                                _ptr(ab))
+    return pk, ab

@@ -385,6 +385,53 @@ void nf4o_lora_linear(const uint16_t *x, int64_t M, int64_t K, int64_t N,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Merging the adapter into the quantized base, then requantizing            */
+/* ------------------------------------------------------------------------ */
+
+/* [QP] section "Step 4: Merging and Inference" merges the trained adapter into
+ * the quantized base for deployment; [AD] section "What it costs" (item 3,
+ * "Merging is awkward") notes that a merge into the quantized base must be
+ * requantized, with its own error.  The pages give no arithmetic.  READING:
+ * the merge is formed in binary32 on the exact dequantized weight,
+ *   d[n, k]  = B[n, 0] A[0, k] + ... + B[n, r-1] A[r-1, k] as the chain
+ *              d <- fma(B[n, j], A[j, k], d), j = 0, 1, ..., r - 1, from +0
+ *   W'[n, k] = fma(s, d[n, k], w~[n, k])
+ * (A, B bf16 widened exactly; w~ as in nf4o_dequantize_f32).  Rows
+ * row0 .. row0 + nrows - 1 of W[N, K]; out is [nrows, K]. */
+void nf4o_merge_weight(const uint8_t *packed, const uint8_t *codes, const float *scales,
+                       const float *offset, int64_t K, int bs, int dqbs,
+                       const uint16_t *A, const uint16_t *B, int r, float s,
+                       int64_t row0, int64_t nrows, float *out) {
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t nn = row0 + i;
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t j = nn * K + k;
+            float c = block_constant(codes, scales, offset, j / bs, dqbs);
+            int code = (j & 1) ? (packed[j >> 1] & 15) : (packed[j >> 1] >> 4);
+            float w = NF4_LEVELS[code] * c;
+            float d = 0.0f;
+            for (int q = 0; q < r; ++q)
+                d = fmaf(nf4o_bf16_to_f32(B[nn * r + q]), nf4o_bf16_to_f32(A[(int64_t)q * K + k]), d);
+            out[i * K + k] = fmaf(s, d, w);
+        }
+    }
+}
+
+/* The merged rows quantized again by the blockwise NF4 of nf4o_quantize_f32
+ * (K is a multiple of bs, so every block lies inside one row):
+ * packed_out [nrows K / 2], absmax_out [nrows K / bs], the fp32 constants of
+ * W' (double-quantizing them is the separate step nf4o_double_quantize). */
+void nf4o_merge_requantize(const uint8_t *packed, const uint8_t *codes, const float *scales,
+                           const float *offset, int64_t K, int bs, int dqbs,
+                           const uint16_t *A, const uint16_t *B, int r, float s,
+                           int64_t row0, int64_t nrows, uint8_t *packed_out, float *absmax_out) {
+    float *wm = (float *)malloc((size_t)(nrows * K > 0 ? nrows * K : 1) * sizeof(float));
+    nf4o_merge_weight(packed, codes, scales, offset, K, bs, dqbs, A, B, r, s, row0, nrows, wm);
+    nf4o_quantize_f32(wm, nrows * K, bs, packed_out, absmax_out);
+    free(wm);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Array forms of the scalar routines (loops only, for the tests)           */
 /* ------------------------------------------------------------------------ */
 
