@@ -526,6 +526,37 @@ def run_suite(args):
                  peak_sustained=peaks["bf16_tflops_sustained"])
     torch.cuda.empty_cache()
 
+    # ---- merge the adapter into the quantized base and requantize (+ double
+    # quantization of the new constants), and the error the requantization adds
+    for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
+        W, _, A, B = wl.linear_inputs(c)
+        Wd, Ad, Bd = W.to(dev), A.to(dev), B.to(dev)
+        st = q.quantize_weight(Wd)
+        m = c.N * c.K
+        pk = torch.empty(m // 2, dtype=torch.uint8, device=dev)
+        ab = torch.empty(m // BLOCK, device=dev)
+
+        def f_merge():
+            q.nf4_merge_requantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N, c.K, Ad, Bd, c.scaling,
+                                   packed_out=pk, absmax_out=ab)
+        us = graph_us(f_merge, 3)
+        byts = dequant_bytes(m, 0) + c.r * c.K * 2 + c.N * c.r * 2 + m // 2 + (m // BLOCK) * 4
+        merged = q.merge_and_requantize(st, Ad, Bd, c.scaling)
+        w_base = q.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, m, torch.float32).view(c.N, c.K)
+        w_new = q.nf4_dequantize(merged.packed, merged.absmax_q, merged.absmax2, merged.offset, m,
+                                 torch.float32).view(c.N, c.K)
+        delta = c.scaling * (Bd.float() @ Ad.float())
+        w_exact = w_base + delta
+        rms = lambda t: float(t.pow(2).mean().sqrt())
+        emit(f"merge + requantize {c.N}x{c.K} r={c.r}", us, byts, "GB/s",
+             fma_per_s=round(m * c.r / (us * 1e-6) / 1e12, 3), fma_unit="T fma/s (fp32 chain)",
+             base_quant_rel_rms=round(rms(w_base - Wd.float()) / rms(Wd.float()), 6),
+             requant_rel_rms=round(rms(w_new - w_exact) / rms(w_exact), 6),
+             adapter_rel_rms=round(rms(delta) / rms(w_base), 6),
+             adapter_retained=round(float(((w_new - w_base) * delta).sum() / (delta * delta).sum()), 4))
+        del W, Wd, Ad, Bd, st, pk, ab, merged, w_base, w_new, delta, w_exact
+        torch.cuda.empty_cache()
+
     # ---- one 8B-shaped decoder layer, M = 4096 tokens, r = 64, s = 0.25:
     # fused NF4 + LoRA against bf16 x W^T + s (x A^T) B^T on cuBLAS
     M, r, sc = 4096, 64, 0.25

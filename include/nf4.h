@@ -208,6 +208,31 @@ NF4_API nf4_status nf4_lora_linear_fwd_noalloc(const void *x, int64_t M, int64_t
  * NF4_ERR_CUDA on a CUDA error, NF4_OK otherwise. */
 NF4_API nf4_status nf4_device_status(void *stream);
 
+/* nf4_merge_requantize -- merge the LoRA adapter into the quantized base and
+ * quantize the result again ("QLoRA in Production ...", section "Step 4:
+ * Merging and Inference"; "QLoRA: quantising the part you are not training",
+ * section "What it costs", item 3: a merge into the quantized base must be
+ * requantized).  READING of the arithmetic (the pages give none), in binary32:
+ *   w~[n, k] = RN(q[code] * c1')                      (as nf4_dequantize, fp32)
+ *   d[n, k]  = chain d <- fma(B[n, j], A[j, k], d), j = 0 .. r-1, from +0
+ *   W'[n, k] = fma(scaling, d[n, k], w~[n, k])
+ * then blockwise NF4 of W' (as nf4_quantize on an fp32 tensor).
+ *   packed, absmax_q, absmax2, offset: the quantized W[N, K], as for
+ *       nf4_dequantize (absmax_q NULL: absmax2 holds fp32 constants;
+ *       offset NULL: no centring).  K % 64 == 0.
+ *   A: bf16 [r, K], B: bf16 [N, r] (device), 0 <= r <= 64 (r = 0 or NULL A/B:
+ *       no adapter, W' = w~).
+ *   packed_out: uint8 [N K / 2], absmax_out: fp32 [N K / 64] (device),
+ *       caller-owned; packed_out may alias packed, absmax_out may alias
+ *       absmax2 when absmax_q is NULL.  Double-quantize absmax_out with
+ *       nf4_double_quantize to return to the stored format.
+ * Errors: NF4_ERR_INVALID (null or misaligned pointers, N < 1, K not a
+ * positive multiple of 64, offset without absmax_q), NF4_ERR_UNSUPPORTED
+ * (r > 64), NF4_ERR_CUDA on a launch error.  Asynchronous on stream. */
+NF4_API nf4_status nf4_merge_requantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2,
+                                        const float *offset, int64_t N, int64_t K, const void *A, const void *B,
+                                        int r, float scaling, uint8_t *packed_out, float *absmax_out, void *stream);
+
 /* nf4_selftest_wait_timeout -- failure-detection check (no counterpart on
  * the pages).  Launches on `stream` one thread that waits on a shared-memory
  * mbarrier nothing arrives on; after limit_ns nanoseconds of %globaltimer

@@ -241,9 +241,12 @@ def _merge_args(packed, codes, scales, offset, K, A_bf16, B_bf16, r):
     scales = np.ascontiguousarray(scales, np.float32)
     codes = None if codes is None else np.ascontiguousarray(codes, np.uint8)
     off = None if offset is None else np.array([offset], np.float32)
+    N = packed.size * 2 // K
+    if r == 0:  # no adapter: W' = w~
+        return packed, codes, scales, off, np.zeros(1, np.uint16), np.zeros(1, np.uint16), N
     A = np.ascontiguousarray(A_bf16, np.uint16).reshape(r, K)
-    B = np.ascontiguousarray(B_bf16, np.uint16).reshape(-1, r)
-    return packed, codes, scales, off, A, B
+    B = np.ascontiguousarray(B_bf16, np.uint16).reshape(N, r)
+    return packed, codes, scales, off, A, B, N
 
 
 def merge_weight(packed, codes, scales, offset, K, A_bf16, B_bf16, r, s, row0=0, nrows=None,
@@ -253,8 +256,7 @@ def merge_weight(packed, codes, scales, offset, K, A_bf16, B_bf16, r, s, row0=0,
     [row0, row0 + nrows) of W[N, K]; float32 [nrows, K].
     Pinned by the delta against an fp64 matmul, the s = 0 identity, and an
     exact-rational re-evaluation of the chain on a tiny case."""
-    packed, codes, scales, off, A, B = _merge_args(packed, codes, scales, offset, K, A_bf16, B_bf16, r)
-    N = B.shape[0]
+    packed, codes, scales, off, A, B, N = _merge_args(packed, codes, scales, offset, K, A_bf16, B_bf16, r)
     nrows = N - row0 if nrows is None else nrows
     out = np.empty((nrows, K), np.float32)
     lib().nf4o_merge_weight(_ptr(packed), _ptr(codes), _ptr(scales), _ptr(off), int(K), blocksize, dq_blocksize,
@@ -266,8 +268,7 @@ def merge_requantize(packed, codes, scales, offset, K, A_bf16, B_bf16, r, s, row
                      blocksize: int = BLOCKSIZE, dq_blocksize: int = DQ_BLOCKSIZE):
     """merge_weight's rows quantized again (blockwise NF4, fp32 constants):
     (packed uint8 [nrows K / 2], absmax float32 [nrows K / 64])."""
-    packed, codes, scales, off, A, B = _merge_args(packed, codes, scales, offset, K, A_bf16, B_bf16, r)
-    N = B.shape[0]
+    packed, codes, scales, off, A, B, N = _merge_args(packed, codes, scales, offset, K, A_bf16, B_bf16, r)
     nrows = N - row0 if nrows is None else nrows
     pk = np.empty(nrows * K // 2, np.uint8)
     ab = np.empty(nrows * K // blocksize, np.float32)

@@ -26,6 +26,10 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
 int64_t lora_workspace_bytes(int64_t M, int r);
 unsigned *device_error_word(cudaError_t *status);
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream);
+cudaError_t launch_merge_requantize(const uint8_t *packed, const uint8_t *q8, const float *scales,
+                                    const float *offset, int64_t N, int64_t K, const void *A, const void *B, int r,
+                                    float s, uint8_t *packed_out, float *absmax_out, cudaStream_t stream);
+int merge_max_rank();
 }  // namespace nf4
 
 namespace {
@@ -163,6 +167,23 @@ nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N, c
     return cuda_status(nf4::launch_lora_linear(x, M, K, N, packed, absmax_q, absmax2, offset, lora ? A : nullptr,
                                                lora ? B : nullptr, lora ? r : 0, scaling, y, workspace,
                                                (cudaStream_t)stream, sms, err));
+}
+
+nf4_status nf4_merge_requantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2,
+                                const float *offset, int64_t N, int64_t K, const void *A, const void *B, int r,
+                                float scaling, uint8_t *packed_out, float *absmax_out, void *stream) {
+    if (N < 1 || K < nf4::kBlock || (K % nf4::kBlock) != 0) return NF4_ERR_INVALID;
+    if (r < 0) return NF4_ERR_INVALID;
+    if (r > nf4::merge_max_rank()) return NF4_ERR_UNSUPPORTED;
+    if (!packed || !absmax2 || !packed_out || !absmax_out) return NF4_ERR_INVALID;
+    if (absmax_q == nullptr && offset != nullptr) return NF4_ERR_INVALID;
+    const bool lora = r > 0 && A != nullptr && B != nullptr;
+    if (!aligned16(packed) || !aligned16(absmax_q) || !aligned16(absmax2) || !aligned16(offset) ||
+        !aligned16(A) || !aligned16(B) || !aligned16(packed_out) || !aligned16(absmax_out))
+        return NF4_ERR_INVALID;
+    return cuda_status(nf4::launch_merge_requantize(packed, absmax_q, absmax2, offset, N, K, lora ? A : nullptr,
+                                                    lora ? B : nullptr, lora ? r : 0, scaling, packed_out,
+                                                    absmax_out, (cudaStream_t)stream));
 }
 
 nf4_status nf4_selftest_wait_timeout(int64_t limit_ns, void *stream) {

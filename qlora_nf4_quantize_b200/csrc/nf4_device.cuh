@@ -91,6 +91,25 @@ __device__ __forceinline__ float block_scale_finish(const ScaleRaw &r, float mu)
     }
 }
 
+// Code selection (section "Block-Wise Quantization Mechanics"): the code of a
+// normalised value x is the arg-min of |x - q_i| with ties to the lower
+// index, i.e. #{i : x > t_i} with t_i = RD_f32((q_i + q_{i+1}) / 2), the exact
+// midpoint rounded down.  fill_thresholds writes t_0..t_14 (call from one
+// thread or with a barrier after).
+__device__ __forceinline__ void fill_thresholds(float *s_t) {
+    for (int i = threadIdx.x; i < 15; i += blockDim.x) {
+        const double m = ((double)c_levels[i] + (double)c_levels[i + 1]) * 0.5;  // exact in binary64
+        s_t[i] = __double2float_rd(m);
+    }
+}
+
+__device__ __forceinline__ int code_of_quotient(float x, const float *s_t) {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < 15; ++i) c += (x > s_t[i]) ? 1 : 0;
+    return c;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
     return *reinterpret_cast<uint32_t *>(&v);

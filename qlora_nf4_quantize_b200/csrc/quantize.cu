@@ -31,20 +31,13 @@ constexpr int kCellTable = 256;   // indexed by the low byte of RN(64 q) + 64 (+
 constexpr int kQuantThreads = 256;
 
 __device__ __forceinline__ int exact_code(float w, float c1, const float *s_t) {
-    float x = __fdiv_rn(w, c1);
-    int c = 0;
-#pragma unroll
-    for (int i = 0; i < 15; ++i) c += (x > s_t[i]) ? 1 : 0;
-    return c;
+    return code_of_quotient(__fdiv_rn(w, c1), s_t);
 }
 
 // Fill the thresholds and the cell table in shared memory (once per CTA).
 __device__ void build_tables(float *s_t, uint32_t *s_cell) {
     int tid = threadIdx.x;
-    if (tid < 15) {
-        double m = ((double)c_levels[tid] + (double)c_levels[tid + 1]) * 0.5;  // exact
-        s_t[tid] = __double2float_rd(m);
-    }
+    fill_thresholds(s_t);
     __syncthreads();
     if (tid >= kCells && tid < kCellTable) s_cell[tid] = 0x40800000u | 15u;  // never reached by finite q
     if (tid < kCells) {

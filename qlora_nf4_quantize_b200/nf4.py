@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
     L.nf4_lora_linear_fwd_noalloc.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, i32, f32, P, P]
     L.nf4_device_status.restype = i32
     L.nf4_device_status.argtypes = [P]
+    L.nf4_merge_requantize.restype = i32
+    L.nf4_merge_requantize.argtypes = [P, P, P, P, i64, i64, P, P, i32, f32, P, P, P]
     L.nf4_selftest_wait_timeout.restype = i32
     L.nf4_selftest_wait_timeout.argtypes = [i64, P]
     _lib = L
@@ -225,6 +227,35 @@ def nf4_device_status(stream=None) -> int:
     return st
 
 
+def nf4_merge_requantize(packed: torch.Tensor, absmax_q: Optional[torch.Tensor], absmax2: torch.Tensor,
+                         offset: Optional[torch.Tensor], N: int, K: int, A: Optional[torch.Tensor] = None,
+                         B: Optional[torch.Tensor] = None, scaling: float = 1.0,
+                         packed_out: Optional[torch.Tensor] = None, absmax_out: Optional[torch.Tensor] = None,
+                         stream=None):
+    """W' = fma(scaling, B A, dequant(W)) quantized again; returns (packed_out
+    uint8 [N K / 2], absmax_out fp32 [N K / 64])."""
+    n = N * K
+    _need(packed, "packed", torch.uint8, n // 2)
+    if absmax_q is not None:
+        _need(absmax_q, "absmax_q", torch.uint8, n // BLOCKSIZE)
+    _need(absmax2, "absmax2", torch.float32)
+    r = 0
+    if A is not None and B is not None:
+        r = A.shape[0]
+        _need(A, "A", torch.bfloat16, r * K)
+        _need(B, "B", torch.bfloat16, N * r)
+    if packed_out is None:
+        packed_out = torch.empty(n // 2, dtype=torch.uint8, device=packed.device)
+    if absmax_out is None:
+        absmax_out = torch.empty(n // BLOCKSIZE, dtype=torch.float32, device=packed.device)
+    _need(packed_out, "packed_out", torch.uint8, n // 2)
+    _need(absmax_out, "absmax_out", torch.float32, n // BLOCKSIZE)
+    st = lib().nf4_merge_requantize(_p(packed), _p(absmax_q), _p(absmax2), _p(offset), N, K, _p(A), _p(B), r,
+                                    float(scaling), _p(packed_out), _p(absmax_out), _stream(stream))
+    _check("nf4_merge_requantize", st)
+    return packed_out, absmax_out
+
+
 def nf4_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     """Launch the bounded-wait check (a wait that expires after limit_ns);
     the next nf4_device_status() raises Nf4Error with NF4_ERR_TIMEOUT."""
@@ -247,6 +278,19 @@ class QuantState:
     def nbytes(self) -> int:
         t = [self.packed, self.absmax_q, self.absmax2, self.offset]
         return sum(x.numel() * x.element_size() for x in t if x is not None)
+
+
+def merge_and_requantize(state: "QuantState", A: torch.Tensor, B: torch.Tensor, scaling: float,
+                         double_quant: bool = True, centre: bool = True, stream=None) -> "QuantState":
+    """nf4_merge_requantize followed (optionally) by nf4_double_quantize: the
+    adapter merged into the quantized base, in the stored format again."""
+    N, K = state.shape
+    packed, absmax = nf4_merge_requantize(state.packed, state.absmax_q, state.absmax2, state.offset, N, K, A, B,
+                                          scaling, stream=stream)
+    if not double_quant:
+        return QuantState(packed, None, absmax, None, (N, K))
+    q8, c2, off = nf4_double_quantize(absmax, centre=centre, stream=stream)
+    return QuantState(packed, q8, c2, off, (N, K))
 
 
 def quantize_weight(w: torch.Tensor, double_quant: bool = True, centre: bool = True, stream=None) -> QuantState:

@@ -40,6 +40,18 @@ def test_codebook_call_matches_oracle(nf4lib, oracle_mod):
     assert np.array_equal(got, oracle_mod.codebook())
 
 
+def test_merge_arguments_checked_on_the_host(nf4lib):
+    L = nf4lib.lib()
+    fake = ctypes.c_void_p(0x1000)
+    args = lambda N, K, r: (fake, fake, fake, fake, N, K, fake, fake, r, 1.0, fake, fake, None)
+    assert L.nf4_merge_requantize(*args(8, 100, 16)) == 1   # K not a multiple of 64
+    assert L.nf4_merge_requantize(*args(0, 128, 16)) == 1   # no rows
+    assert L.nf4_merge_requantize(*args(8, 128, 65)) == 2   # rank above 64
+    assert L.nf4_merge_requantize(*args(8, 128, -1)) == 1
+    bad = ctypes.c_void_p(0x1004)                            # misaligned output
+    assert L.nf4_merge_requantize(fake, fake, fake, fake, 8, 128, fake, fake, 16, 1.0, bad, fake, None) == 1
+
+
 def test_selftest_limit_checked_on_the_host(nf4lib):
     L = nf4lib.lib()
     for bad in (0, -5, 1000000001):
