@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             L.nf4o_dequantize_bf16.argtypes = [P, P, P, P, i64, ctypes.c_int, ctypes.c_int, P]
             L.nf4o_lora_linear.argtypes = [P, i64, i64, i64, P, P, P, P, ctypes.c_int, ctypes.c_int,
                                            P, P, ctypes.c_int, ctypes.c_float, P, i64, P]
+            L.nf4o_lora_linear_bwd.argtypes = [P, P, i64, i64, i64, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                               P, P, ctypes.c_int, ctypes.c_float, P, i64, P, P, P]
             L.nf4o_merge_weight.argtypes = [P, P, P, P, i64, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int,
                                             ctypes.c_float, i64, i64, P]
             L.nf4o_merge_requantize.argtypes = [P, P, P, P, i64, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int,
@@ -276,3 +278,35 @@ def merge_requantize(packed, codes, scales, offset, K, A_bf16, B_bf16, r, s, row
                                 dq_blocksize, _ptr(A), _ptr(B), int(r), float(s), int(row0), int(nrows), _ptr(pk),
                                 _ptr(ab))
     return pk, ab
+
+
+def lora_linear_bwd(g_bf16, x_bf16, K, N, packed, codes, scales, offset, A_bf16, B_bf16, r, s, rows=None,
+                    want=("dx", "dA", "dB"), blocksize: int = BLOCKSIZE, dq_blocksize: int = DQ_BLOCKSIZE):
+    """Backward of lora_linear (the adjoint of the forward in the frozen
+    weight's layout): returns a dict with float64 'dx' [len(rows), K],
+    'dA' [r, K], 'dB' [N, r] as requested (g = dL/dy, bf16 bit patterns
+    [M, N]; x bf16 [M, K] needed for dA, dB).  Pinned by the adjoint
+    identities <g, y(x)> = <dx, x>, <g, y_A(E)> = <dA, E>, <g, y_B(F)> =
+    <dB, F> against the (separately pinned) forward."""
+    g = np.ascontiguousarray(g_bf16, np.uint16).reshape(-1, N)
+    M = g.shape[0]
+    x = None if x_bf16 is None else np.ascontiguousarray(x_bf16, np.uint16).reshape(M, K)
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, np.int64)
+    packed = np.ascontiguousarray(packed, np.uint8)
+    scales = np.ascontiguousarray(scales, np.float32)
+    codes = None if codes is None else np.ascontiguousarray(codes, np.uint8)
+    off = None if offset is None else np.array([offset], np.float32)
+    lora = A_bf16 is not None and B_bf16 is not None and r > 0
+    A = np.ascontiguousarray(A_bf16, np.uint16) if lora else None
+    B = np.ascontiguousarray(B_bf16, np.uint16) if lora else None
+    out = {}
+    dx = np.empty((rows.size, K), np.float64) if "dx" in want else None
+    dA = np.empty((r, K), np.float64) if ("dA" in want and lora) else None
+    dB = np.empty((N, r), np.float64) if ("dB" in want and lora) else None
+    lib().nf4o_lora_linear_bwd(_ptr(g), _ptr(x), M, int(K), int(N), _ptr(packed), _ptr(codes), _ptr(scales),
+                               _ptr(off), blocksize, dq_blocksize, _ptr(A), _ptr(B), int(r if lora else 0), float(s),
+                               _ptr(rows), rows.size, _ptr(dx), _ptr(dA), _ptr(dB))
+    for name, arr in (("dx", dx), ("dA", dA), ("dB", dB)):
+        if arr is not None:
+            out[name] = arr
+    return out

@@ -385,6 +385,94 @@ void nf4o_lora_linear(const uint16_t *x, int64_t M, int64_t K, int64_t N,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Backward pass through the frozen base                                     */
+/* ------------------------------------------------------------------------ */
+
+/* [MF] section "Gradient Computation" (after "Forward Pass Computation"):
+ * gradients go to the adapter only, and the activation gradient flows through
+ * both paths.  In the weight layout used here (W[N, K], L1 = A^T, L2 = B^T,
+ * w the bf16 dequantized weight) and with g = dL/dy [M, N]:
+ *   dx[m, k] = sum_n g[m, n] w[n, k] + s sum_j u[m, j] A[j, k],
+ *              u[m, j] = sum_n g[m, n] B[n, j]
+ *   dA[j, k] = s sum_m u[m, j] x[m, k]
+ *   dB[n, j] = s sum_m g[m, n] t[m, j],  t[m, j] = sum_k x[m, k] A[j, k]
+ * Every sum in binary64 (products of bf16 values are exact there); u and t are
+ * kept unrounded.  dx is computed for the token rows rows[0..nrows) only
+ * ([nrows, K]); dA ([r, K]) and dB ([N, r]) use all M rows; any output may be
+ * NULL.  x may be NULL when dA and dB are. */
+void nf4o_lora_linear_bwd(const uint16_t *g, const uint16_t *x, int64_t M, int64_t K, int64_t N,
+                          const uint8_t *packed, const uint8_t *codes, const float *scales,
+                          const float *offset, int bs, int dqbs,
+                          const uint16_t *A, const uint16_t *B, int r, float s,
+                          const int64_t *rows, int64_t nrows, double *dx, double *dA, double *dB) {
+    int lora = (A != NULL && B != NULL && r > 0);
+    double *u = NULL, *t = NULL;
+    if (lora) {
+        u = (double *)calloc((size_t)(M * r > 0 ? M * r : 1), sizeof(double));
+#pragma omp parallel for schedule(static)
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t n = 0; n < N; ++n) {
+                double gv = nf4o_bf16_to_f32(g[m * N + n]);
+                for (int j = 0; j < r; ++j) u[m * r + j] += gv * nf4o_bf16_to_f32(B[n * r + j]);
+            }
+    }
+    if (dx) {
+        for (int64_t i = 0; i < nrows * K; ++i) dx[i] = 0.0;
+        float *wf = (float *)malloc((size_t)(K > 0 ? K : 1) * sizeof(float));
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t j = n * K + k;
+                float c = block_constant(codes, scales, offset, j / bs, dqbs);
+                int code = (j & 1) ? (packed[j >> 1] & 15) : (packed[j >> 1] >> 4);
+                wf[k] = nf4o_bf16_to_f32(nf4o_f32_to_bf16(NF4_LEVELS[code] * c));
+            }
+#pragma omp parallel for schedule(static)
+            for (int64_t i = 0; i < nrows; ++i) {
+                double gv = nf4o_bf16_to_f32(g[rows[i] * N + n]);
+                if (gv != 0.0)
+                    for (int64_t k = 0; k < K; ++k) dx[i * K + k] += gv * (double)wf[k];
+            }
+        }
+        free(wf);
+        if (lora)
+#pragma omp parallel for schedule(static)
+            for (int64_t i = 0; i < nrows; ++i)
+                for (int64_t k = 0; k < K; ++k) {
+                    double acc = 0.0;
+                    for (int j = 0; j < r; ++j) acc += u[rows[i] * r + j] * nf4o_bf16_to_f32(A[(int64_t)j * K + k]);
+                    dx[i * K + k] += (double)s * acc;
+                }
+    }
+    if (lora && dA)
+#pragma omp parallel for schedule(static)
+        for (int64_t k = 0; k < K; ++k)
+            for (int j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t m = 0; m < M; ++m) acc += u[m * r + j] * nf4o_bf16_to_f32(x[m * K + k]);
+                dA[(int64_t)j * K + k] = (double)s * acc;
+            }
+    if (lora && dB) {
+        t = (double *)malloc((size_t)(M * r > 0 ? M * r : 1) * sizeof(double));
+#pragma omp parallel for schedule(static)
+        for (int64_t m = 0; m < M; ++m)
+            for (int j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k) acc += nf4o_bf16_to_f32(x[m * K + k]) * nf4o_bf16_to_f32(A[(int64_t)j * K + k]);
+                t[m * r + j] = acc;
+            }
+#pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < N; ++n)
+            for (int j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t m = 0; m < M; ++m) acc += nf4o_bf16_to_f32(g[m * N + n]) * t[m * r + j];
+                dB[n * r + j] = (double)s * acc;
+            }
+    }
+    free(u);
+    free(t);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Merging the adapter into the quantized base, then requantizing            */
 /* ------------------------------------------------------------------------ */
 
