@@ -208,6 +208,36 @@ NF4_API nf4_status nf4_lora_linear_fwd_noalloc(const void *x, int64_t M, int64_t
  * NF4_ERR_CUDA on a CUDA error, NF4_OK otherwise. */
 NF4_API nf4_status nf4_device_status(void *stream);
 
+/* nf4_lora_linear_bwd_workspace_size -- bytes of device workspace that
+ * nf4_lora_linear_bwd needs for these sizes (0 when r = 0). */
+NF4_API int64_t nf4_lora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
+
+/* nf4_lora_linear_bwd -- backward pass of nf4_lora_linear_fwd ("QLoRA:
+ * Mathematical Foundations ...", section "Gradient Computation": gradients go
+ * to the adapter only; the activation gradient flows through both paths).  In
+ * the layout W[N, K], A[r, K], B[N, r], with g = dL/dy bf16 [M, N]:
+ *   dx = g W~ + s (g B) A            bf16 [M, K] (W~ = bf16 dequantized W,
+ *                                    exactly nf4_dequantize's output)
+ *   dA = s (g B)^T x                 fp32 [r, K]
+ *   dB = s g^T (x A^T)               fp32 [N, r]
+ * bf16 operands, fp32 accumulation.  Any of dx, dA, dB may be NULL (not
+ * computed); x is needed only for dA and dB; A, B NULL or r = 0 drop the
+ * adapter (then dA, dB must be NULL).
+ *   g, x, A, B, packed, absmax_q, absmax2, offset: as for nf4_lora_linear_fwd
+ *       (device pointers, 16-byte aligned, caller-owned).
+ *   N % 8 == 0 (rows of g are read by TMA), K % 64 == 0, r in {0,16,32,64}.
+ *   workspace: >= nf4_lora_linear_bwd_workspace_size(M, N, K, r) bytes of
+ *       device memory, 256-byte aligned (scratch: s g B as a bf16 hi/lo pair,
+ *       B^T and A^T).
+ * Errors: NF4_ERR_INVALID, NF4_ERR_UNSUPPORTED (r or shapes outside the
+ * above), NF4_ERR_CUDA.  Asynchronous on stream; NF4_ERR_TIMEOUT (a bounded
+ * wait expired) is reported by nf4_device_status. */
+NF4_API nf4_status nf4_lora_linear_bwd(const void *g, const void *x, int64_t M, int64_t K, int64_t N,
+                                       const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2,
+                                       const float *offset, const void *A, const void *B, int r, float scaling,
+                                       void *dx, float *dA, float *dB, void *workspace, int64_t workspace_bytes,
+                                       void *stream);
+
 /* nf4_merge_requantize -- merge the LoRA adapter into the quantized base and
  * quantize the result again ("QLoRA in Production ...", section "Step 4:
  * Merging and Inference"; "QLoRA: quantising the part you are not training",

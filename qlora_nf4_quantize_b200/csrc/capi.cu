@@ -30,6 +30,15 @@ cudaError_t launch_merge_requantize(const uint8_t *packed, const uint8_t *q8, co
                                     const float *offset, int64_t N, int64_t K, const void *A, const void *B, int r,
                                     float s, uint8_t *packed_out, float *absmax_out, cudaStream_t stream);
 int merge_max_rank();
+int64_t lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+cudaError_t launch_lora_linear_bwd_dx(const void *g, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
+                                      const uint8_t *q8, const float *scales, const float *offset, const void *A,
+                                      const void *B, int r, float s, void *dx, void *workspace, unsigned *err,
+                                      cudaStream_t stream);
+cudaError_t launch_lora_grads(const void *g, const void *x, int64_t M, int64_t K, int64_t N, const void *A,
+                              const void *B, int r, float s, float *dA, float *dB, void *workspace,
+                              cudaStream_t stream);
+int64_t lora_grads_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 }  // namespace nf4
 
 namespace {
@@ -167,6 +176,48 @@ nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N, c
     return cuda_status(nf4::launch_lora_linear(x, M, K, N, packed, absmax_q, absmax2, offset, lora ? A : nullptr,
                                                lora ? B : nullptr, lora ? r : 0, scaling, y, workspace,
                                                (cudaStream_t)stream, sms, err));
+}
+
+int64_t nf4_lora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
+    if (M < 0 || N < 0 || K < 0 || r <= 0) return 0;
+    const int64_t a = nf4::lora_bwd_workspace_bytes(M, N, K, r), b = nf4::lora_grads_workspace_bytes(M, N, K, r);
+    return a > b ? a : b;
+}
+
+nf4_status nf4_lora_linear_bwd(const void *g, const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
+                               const uint8_t *absmax_q, const float *absmax2, const float *offset, const void *A,
+                               const void *B, int r, float scaling, void *dx, float *dA, float *dB, void *workspace,
+                               int64_t workspace_bytes, void *stream) {
+    if (M < 1 || N < 1 || K < nf4::kBlock || (K % nf4::kBlock) != 0) return NF4_ERR_INVALID;
+    if ((N % 8) != 0) return NF4_ERR_UNSUPPORTED;
+    if (r != 0 && r != 16 && r != 32 && r != 64) return NF4_ERR_UNSUPPORTED;
+    if (!g) return NF4_ERR_INVALID;
+    const bool lora = r > 0 && A != nullptr && B != nullptr;
+    if (!lora && (dA || dB)) return NF4_ERR_INVALID;
+    if ((dA || dB) && !x) return NF4_ERR_INVALID;
+    if (dx && (!packed || !absmax2)) return NF4_ERR_INVALID;
+    if (absmax_q == nullptr && offset != nullptr) return NF4_ERR_INVALID;
+    if (!aligned16(g) || !aligned16(x) || !aligned16(packed) || !aligned16(absmax_q) || !aligned16(absmax2) ||
+        !aligned16(offset) || !aligned16(A) || !aligned16(B) || !aligned16(dx) || !aligned16(dA) || !aligned16(dB))
+        return NF4_ERR_INVALID;
+    const int rr = lora ? r : 0;
+    if (lora) {
+        if (workspace == nullptr || ((uintptr_t)workspace & 255u) != 0) return NF4_ERR_INVALID;
+        if (workspace_bytes < nf4_lora_linear_bwd_workspace_size(M, N, K, r)) return NF4_ERR_INVALID;
+    }
+    cudaError_t st;
+    unsigned *err = nf4::device_error_word(&st);
+    if (st != cudaSuccess) return cuda_status(st);
+    if (dx) {
+        st = nf4::launch_lora_linear_bwd_dx(g, M, K, N, packed, absmax_q, absmax2, offset, lora ? A : nullptr,
+                                            lora ? B : nullptr, rr, scaling, dx, workspace, err, (cudaStream_t)stream);
+        if (st != cudaSuccess) return cuda_status(st);
+    }
+    if (dA || dB) {
+        st = nf4::launch_lora_grads(g, x, M, K, N, A, B, r, scaling, dA, dB, workspace, (cudaStream_t)stream);
+        if (st != cudaSuccess) return cuda_status(st);
+    }
+    return NF4_OK;
 }
 
 nf4_status nf4_merge_requantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2,

@@ -1,0 +1,395 @@
+// gemm_bwd.cu -- K8: the input gradient of the fused frozen-base LoRA linear
+// on the tensor cores (tcgen05 / TMEM / TMA, sm_100a).
+//
+// "QLoRA: Mathematical Foundations ...", section "Gradient Computation": the
+// activation gradient flows through both paths,
+//   dx[m, k] = sum_n g[m, n] W~[n, k] + s sum_j u[m, j] A[j, k],  u = g B,
+// in the layout W[N, K], A[r, K], B[N, r], g = dL/dy [M, N].  W~ is the bf16
+// dequantized weight, bit-identical to nf4_dequantize's output; bf16 operands,
+// fp32 accumulation, bf16 output.
+//
+// Unlike the forward, the contraction runs along W's rows (n), across the
+// 64-blocks.  A CTA computes a 256 (tokens) x 256 (k) tile of dx as two MMA
+// accumulators of 128 tokens each (512 tensor-memory columns):
+//   D_h[m, k] += G[m, n] * WT[k, n],  M_mma = 128, N_mma = 256, K = 16
+//   G  = g tile (256 tokens x 64 n) brought by TMA with 128-byte swizzle;
+//   WT = the dequantized weight tile transposed (256 k x 64 n), written by
+//        two dequant warpgroups into shared memory in the same 128-byte
+//        swizzled K-major layout that TMA produces for G: a lane owns two
+//        rows n, n+1 and one 64-block of k, so it still dequantizes whole
+//        blocks with one register lookup table each (mma_util.cuh), and pairs
+//        the two rows' values of one k into one 32-bit word (one byte permute
+//        per two weights) for a conflict-free 32-bit shared store;
+// both operands come from shared memory (SS MMA).  Each dequantized weight
+// feeds 256 tokens, as in the forward.  After the N / 64 weight steps, RP / 64
+// extension steps add the LoRA term the same way: G' = [u_hi | u_lo | 0]
+// (u scaled by s, as a bf16 hi/lo pair, from the down-projection kernel run
+// on g with B^T) and WT' = rows k of [A^T | A^T | 0].
+//
+// Warp roles (12 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
+// MMA issuer (one elected thread), warps 4..11 = two dequant warpgroups
+// (warpgroup h produces the k-steps with index % 2 == h) and, at the end, the
+// epilogue (warpgroup h stores accumulator h: tcgen05.ld, bf16, 64-byte row
+// segments).  Every mbarrier wait is bounded as in the forward GEMM.
+#include "mma_util.cuh"
+#include "tc_util.cuh"
+
+namespace nf4 {
+namespace {
+
+constexpr int kGM = 256;       // tokens per CTA (two accumulators of 128)
+constexpr int kGN = 256;       // output columns k per CTA (MMA N)
+constexpr int kGK = 64;        // contraction (n) per pipeline step
+constexpr int kGStages = 3;
+constexpr int kGThreads = 128 + 256;
+constexpr uint32_t kGTmemCols = 512;
+constexpr uint32_t kGStageBytes = kGM * kGK * 2;  // also the WT tile: kGN x kGK bf16
+static_assert(kGM * kGK == kGN * kGK, "G and WT tiles have the same size");
+
+// UMMA instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kGIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kGN >> 3) << 17) |
+                             ((uint32_t)(128 >> 4) << 24);
+
+struct __align__(1024) BwdSmem {
+    uint8_t g[kGStages][kGStageBytes];
+    uint8_t wt[kGStages][kGStageBytes];
+    uint64_t g_full[kGStages];
+    uint64_t g_empty[kGStages];
+    uint64_t w_full[kGStages];
+    uint64_t w_empty[kGStages];
+    uint64_t acc_full;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// 64 codes and the block constant of weight row n, k-block kb (whole block).
+struct BlockCodes {
+    uint32_t w[8];
+    ScaleRaw sr;
+};
+
+template <int kMode>
+__device__ __forceinline__ void load_block(const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
+                                           const float *__restrict__ scales, int64_t n, int64_t K, int64_t kb,
+                                           bool valid, BlockCodes &bc) {
+    if (valid) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(packed + n * (K >> 1) + kb * 32);
+        const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
+        bc.w[0] = u0.x; bc.w[1] = u0.y; bc.w[2] = u0.z; bc.w[3] = u0.w;
+        bc.w[4] = u1.x; bc.w[5] = u1.y; bc.w[6] = u1.z; bc.w[7] = u1.w;
+        bc.sr = block_scale_load<kMode>(q8, scales, n * (K >> 6) + kb);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bc.w[i] = 0x77777777u;  // code 7 = level 0
+        bc.sr.q8 = 0;
+        bc.sr.v = 0.0f;
+    }
+}
+
+// byte offset of the 32-bit word (k-row kk, n-pair p) in a 128-byte swizzled tile
+__device__ __forceinline__ uint32_t wt_offset(int kk, int p) {
+    return (uint32_t)kk * 128u + ((uint32_t)((p >> 2) ^ (kk & 7)) << 4) + (uint32_t)(p & 3) * 4u;
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kGThreads, 1)
+    k_gemm_bwd(const __grid_constant__ CUtensorMap tmap_g, const __grid_constant__ CUtensorMap tmap_u, int64_t M,
+               int64_t K, int64_t N, const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
+               const float *__restrict__ scales, const float *__restrict__ offset,
+               const __nv_bfloat16 *__restrict__ At, int r, int rp, __nv_bfloat16 *__restrict__ dx, unsigned *err) {
+    extern __shared__ uint8_t smem_raw[];
+    BwdSmem &S = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    volatile int *abort = &S.abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t k0 = (int64_t)blockIdx.x * kGN;
+    const int64_t m0 = (int64_t)blockIdx.y * kGM;
+    const int kn_steps = (int)((N + kGK - 1) / kGK);
+    const int kt_total = kn_steps + (r > 0 ? rp / kGK : 0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            mbar_init(&S.g_full[s], 1);
+            mbar_init(&S.g_empty[s], 1);
+            mbar_init(&S.w_full[s], 4);  // one arrival per warp of the producing warpgroup
+            mbar_init(&S.w_empty[s], 1);
+        }
+        mbar_init(&S.acc_full, 1);
+        mbar_init(&S.drain, 1);
+        S.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&S.tmem_base)),
+                     "r"(kGTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 0) {
+        // ---------------- TMA producer: g tiles, then [u_hi | u_lo] tiles ----------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int kt = 0; kt < kt_total; ++kt) {
+                const int s = kt % kGStages;
+                const uint32_t ph = (uint32_t)(kt / kGStages) & 1u;
+                // u is written by the down-projection kernel launched just
+                // before (programmatic dependent launch)
+                if (kt == kn_steps) asm volatile("griddepcontrol.wait;" ::: "memory");
+                if (!mbar_wait(&S.g_empty[s], ph ^ 1u, abort, err)) break;
+                mbar_arrive_expect_tx(&S.g_full[s], kGStageBytes);
+                if (kt < kn_steps) tma_load_2d(S.g[s], &tmap_g, &S.g_full[s], kt * kGK, (int)m0);
+                else tma_load_2d(S.g[s], &tmap_u, &S.g_full[s], (kt - kn_steps) * kGK, (int)m0);
+                issued = kt + 1;
+            }
+            for (int kt = issued - kGStages < 0 ? 0 : issued - kGStages; kt < issued; ++kt) {
+                unsigned long long t0 = global_ns();
+                while (!mbar_try_wait(&S.g_full[kt % kGStages], (uint32_t)(kt / kGStages) & 1u) &&
+                       global_ns() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            bool any = false;
+            for (int kt = 0; kt < kt_total; ++kt) {
+                const int s = kt % kGStages;
+                const uint32_t ph = (uint32_t)(kt / kGStages) & 1u;
+                if (!mbar_wait(&S.g_full[s], ph, abort, err)) break;
+                if (!mbar_wait(&S.w_full[s], ph, abort, err)) break;
+                tc_fence_after();
+                const uint64_t a0 = smem_desc_sw128(S.g[s]);
+                const uint64_t a1 = smem_desc_sw128(S.g[s] + kGStageBytes / 2);  // tokens 128..255
+                const uint64_t bd = smem_desc_sw128(S.wt[s]);
+#pragma unroll
+                for (int kk = 0; kk < kGK / 16; ++kk) {
+                    const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
+                    tc_mma_ss(tmem, a0 + 2ull * kk, bd + 2ull * kk, kGIdesc, acc);
+                    tc_mma_ss(tmem + 256u, a1 + 2ull * kk, bd + 2ull * kk, kGIdesc, acc);
+                }
+                any = true;
+                tc_commit(&S.g_empty[s]);
+                tc_commit(&S.w_empty[s]);
+                if (kt == kt_total - 1) tc_commit(&S.acc_full);
+            }
+            if (any && *abort) {  // drain our own MMAs before tensor memory is released
+                tc_commit(&S.drain);
+                unsigned long long t0 = global_ns();
+                while (!mbar_try_wait(&S.drain, 0) && global_ns() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else if (warp >= 4) {
+        // ---------------- dequant warpgroups (transposed tiles), then epilogue ----------------
+        const int q = warp & 3;         // k-block of the tile / tensor-memory lane quarter
+        const int h = (warp - 4) >> 2;  // warpgroup: k-steps with index % 2 == h
+        const int p = lane;             // n-pair: rows 2p, 2p + 1 of the step
+        const int64_t kb = (k0 >> 6) + q;  // this lane's k-block of W
+        const bool kvalid = kb * 64 < K;
+        const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
+        bool ok = true;
+        BlockCodes ca, cb, na, nb;
+        auto load_pair = [&](int kt, BlockCodes &x0, BlockCodes &x1) {
+            const int64_t n = (int64_t)kt * kGK + 2 * p;
+            load_block<kMode>(packed, q8, scales, n, K, kb, kvalid && n < N, x0);
+            load_block<kMode>(packed, q8, scales, n + 1, K, kb, kvalid && n + 1 < N, x1);
+        };
+        if (h < kn_steps) load_pair(h, ca, cb);
+        for (int kt = h; kt < kt_total; kt += 2) {
+            const int s = kt % kGStages;
+            const uint32_t ph = (uint32_t)(kt / kGStages) & 1u;
+            const uint32_t tile = smem_addr(S.wt[s]);
+            if (kt < kn_steps) {
+                if (kt + 2 < kn_steps) load_pair(kt + 2, na, nb);
+                uint32_t va[32], vb[32];
+                {
+                    const Lut la = make_lut(block_scale_finish<kMode>(ca.sr, mu));
+                    const Lut lb = make_lut(block_scale_finish<kMode>(cb.sr, mu));
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        lut_lookup8(la, ca.w[i], va + 4 * i);
+                        lut_lookup8(lb, cb.w[i], vb + 4 * i);
+                    }
+                }
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.w_empty[s], ph ^ 1u, abort, err));
+                if (!ok) break;
+                // word j of a row holds k = 2j (low half) and 2j + 1 (high half);
+                // the tile row k holds (n = 2p, n = 2p + 1) in one word
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int kk = 64 * q + 2 * j;
+                    sts32(tile + wt_offset(kk, p), __byte_perm(va[j], vb[j], 0x5410));
+                    sts32(tile + wt_offset(kk + 1, p), __byte_perm(va[j], vb[j], 0x7632));
+                }
+                ca = na;
+                cb = nb;
+            } else {
+                // rows kk of [A^T | A^T | 0], columns [64 e, 64 e + 64): two rows per thread
+                const int e = kt - kn_steps;
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.w_empty[s], ph ^ 1u, abort, err));
+                if (!ok) break;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int kk = 32 * q + lane + 128 * half;
+                    const int64_t k = k0 + kk;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int j0 = 64 * e + 8 * c;
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (k < K && j0 < 2 * r)
+                            v = __ldg(reinterpret_cast<const uint4 *>(At + k * r + (j0 % r)));
+                        sts128(tile + (uint32_t)kk * 128u + ((uint32_t)(c ^ (kk & 7)) << 4), v);
+                    }
+                }
+            }
+            // the tile is read by the tensor cores (async proxy)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.w_full[s]);
+        }
+        if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err));
+        if (ok) {
+            // Epilogue: warpgroup h stores accumulator h; thread = token row.
+            tc_fence_after();
+            const int64_t m = m0 + 128 * h + 32 * q + lane;
+            const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + 256u * (uint32_t)h;
+#pragma unroll 1
+            for (int c = 0; c < kGN / 32; ++c) {
+                uint32_t v[32];
+                tc_load32(base + 32u * c, v);
+                tc_wait_ld();
+                const int64_t k = k0 + 32 * c;
+                if (m < M && k < K) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(dx + m * K + k);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            w[t] = pack_bf16x2(__uint_as_float(v[8 * i + 2 * t]), __uint_as_float(v[8 * i + 2 * t + 1]));
+                        dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGTmemCols) : "memory");
+    }
+}
+
+// dst[C, R] = src[R, C]^T for bf16 (32 x 32 tiles through shared memory)
+__global__ void k_transpose_bf16(const __nv_bfloat16 *__restrict__ src, int64_t R, int64_t C,
+                                 __nv_bfloat16 *__restrict__ dst) {
+    __shared__ __nv_bfloat16 t[32][34];
+    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int64_t rr = r0 + i, cc = c0 + threadIdx.x;
+        if (rr < R && cc < C) t[i][threadIdx.x] = src[rr * C + cc];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int64_t cc = c0 + i, rr = r0 + threadIdx.x;
+        if (rr < R && cc < C) dst[cc * R + rr] = t[threadIdx.x][i];
+    }
+}
+
+template <int kMode>
+cudaError_t launch_bwd_mode(const CUtensorMap &mg, const CUtensorMap &mu, int64_t M, int64_t K, int64_t N,
+                            const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
+                            const __nv_bfloat16 *At, int r, int rp, __nv_bfloat16 *dx, unsigned *err,
+                            cudaStream_t stream) {
+    const size_t smem = sizeof(BwdSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_bwd<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((K + kGN - 1) / kGN), (unsigned)((M + kGM - 1) / kGM));
+    cfg.blockDim = dim3(kGThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
+    return cudaLaunchKernelEx(&cfg, k_gemm_bwd<kMode>, mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dx,
+                              err);
+}
+
+}  // namespace
+
+cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
+                                unsigned *err, cudaStream_t stream);
+int lora_rp(int r);
+
+// dst[C, R] = src[R, C]^T (bf16)
+cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int64_t R, int64_t C, __nv_bfloat16 *dst,
+                                  cudaStream_t stream) {
+    const dim3 grid((unsigned)((C + 31) / 32), (unsigned)((R + 31) / 32));
+    k_transpose_bf16<<<grid, dim3(32, 8), 0, stream>>>(src, R, C, dst);
+    return cudaGetLastError();
+}
+
+static int64_t align256(int64_t b) { return (b + 255) & ~(int64_t)255; }
+
+// Workspace: [u_hi | u_lo | 0] bf16 [M, RP], B^T bf16 [r, N], A^T bf16 [K, r].
+int64_t lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+    if (r <= 0) return 0;
+    return align256(M * lora_rp(r) * 2) + align256((int64_t)r * N * 2) + align256(K * (int64_t)r * 2);
+}
+
+cudaError_t launch_lora_linear_bwd_dx(const void *g, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
+                                      const uint8_t *q8, const float *scales, const float *offset, const void *A,
+                                      const void *B, int r, float s, void *dx, void *workspace, unsigned *err,
+                                      cudaStream_t stream) {
+    if (M > 0x7FFFFFFF || K > 0x7FFFFFFF || N > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const int rp = r > 0 ? lora_rp(r) : 0;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *u2 = ws;
+    auto *Bt = reinterpret_cast<__nv_bfloat16 *>(ws + align256(M * rp * 2));
+    auto *At = reinterpret_cast<__nv_bfloat16 *>(ws + align256(M * rp * 2) + align256((int64_t)r * N * 2));
+    CUtensorMap mg, mu;
+    cudaError_t e = make_map(&mg, g, M, N, kGK, kGM, true);
+    if (e != cudaSuccess) return e;
+    if (r > 0) {
+        e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(B), N, r, Bt, stream);
+        if (e != cudaSuccess) return e;
+        e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(A), r, K, At, stream);
+        if (e != cudaSuccess) return e;
+        // u2 = s g (B^T)^T = s g B as [u_hi | u_lo | 0]
+        e = launch_lora_down_tc(g, Bt, M, N, r, s, u2, rp, err, stream);
+        if (e != cudaSuccess) return e;
+        e = make_map(&mu, u2, M, rp, kGK, kGM, true);
+    } else {
+        e = make_map(&mu, g, M, N, kGK, kGM, true);  // unused: no extension steps
+    }
+    if (e != cudaSuccess) return e;
+    auto *dxp = static_cast<__nv_bfloat16 *>(dx);
+    if (q8 == nullptr) return launch_bwd_mode<2>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+    if (offset == nullptr)
+        return launch_bwd_mode<1>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+    return launch_bwd_mode<0>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+}
+
+}  // namespace nf4

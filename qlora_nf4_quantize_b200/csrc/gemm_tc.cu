@@ -33,11 +33,8 @@
 // every role leaves its loop, the MMA issuer drains its own MMAs, the TMA
 // producer drains its own loads, and tensor memory is released before the
 // CTA exits.  nf4_device_status() reports the expiry as NF4_ERR_TIMEOUT.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "mbarrier.cuh"
 #include "mma_util.cuh"
+#include "tc_util.cuh"
 
 namespace nf4 {
 namespace {
@@ -87,30 +84,6 @@ struct __align__(1024) SmemLayout {
     int abort;
 };
 
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
-            "r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major operand tile written by TMA with
-// 128-byte swizzle (rows of 128 bytes, 8-row groups 1024 bytes apart).
-__device__ __forceinline__ uint64_t smem_desc_sw128(const void *p) {
-    const uint64_t addr = smem_addr(p);
-    uint64_t d = 0;
-    d |= (addr >> 4) & 0x3FFFull;          // start address
-    d |= (uint64_t)1 << 16;                // leading byte offset (unused for swizzled K-major)
-    d |= (uint64_t)(1024 >> 4) << 32;      // stride byte offset: 8 rows x 128 B
-    d |= (uint64_t)1 << 46;                // descriptor version for tcgen05
-    d |= (uint64_t)2 << 61;                // SWIZZLE_128B
-    return d;
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -119,40 +92,6 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
         : "memory");
 }
-
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_store32(uint32_t taddr, const uint32_t v[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_load32(uint32_t taddr, uint32_t v[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
-          "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
-          "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // The packed codes (8 words) and block constant of one 64-wide k-step of
 // weight row n; all-zero-code words outside the matrix.
@@ -375,41 +314,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn(cudaError_t *st) {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn != nullptr) {
-        *st = cudaSuccess;
-        return fn;
-    }
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    *st = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
-    if (*st != cudaSuccess || q != cudaDriverEntryPointSuccess || p == nullptr) {
-        if (*st == cudaSuccess) *st = cudaErrorNotSupported;
-        return nullptr;
-    }
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    return fn;
-}
-
-// 2-D bf16 tensor [rows, cols] row-major with a box of box_cols x box_rows.
-// Operand maps (x, t): box 64 x 256 with 128-byte swizzle, out-of-range rows
-// read as zero.  Output map (y): box 128 x 256, no swizzle; stores clip.
-cudaError_t make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int box_cols, int box_rows,
-                     bool swizzle) {
-    cudaError_t st;
-    auto fn = get_encode_fn(&st);
-    if (fn == nullptr) return st;
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 template <int kMode>
 cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUtensorMap &my, int64_t M, int64_t K, int64_t N,
                         const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
@@ -472,16 +376,6 @@ struct __align__(1024) DownSmem {
 };
 static_assert(kDownStages * kDownRows * 128 >= 64 * kDownRows * 4, "partial tile fits in the x ring");
 
-__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -523,7 +417,7 @@ __global__ void __launch_bounds__(128, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const int64_t m0 = (int64_t)blockIdx.y * kDownRows;
-    const int kt_all = (int)(K / 64);
+    const int kt_all = (int)((K + 63) / 64);  // a partial last step reads zeros beyond K (TMA fill)
     const int kt_begin = (int)((int64_t)rank * kt_all / kDownSplit);
     const int kt_total = (int)((int64_t)(rank + 1) * kt_all / kDownSplit) - kt_begin;
     if (threadIdx.x == 0) {

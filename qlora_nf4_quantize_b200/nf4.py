@@ -65,6 +65,10 @@ def lib() -> ctypes.CDLL:
     L.nf4_lora_linear_fwd_noalloc.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, i32, f32, P, P]
     L.nf4_device_status.restype = i32
     L.nf4_device_status.argtypes = [P]
+    L.nf4_lora_linear_bwd_workspace_size.restype = i64
+    L.nf4_lora_linear_bwd_workspace_size.argtypes = [i64, i64, i64, i32]
+    L.nf4_lora_linear_bwd.restype = i32
+    L.nf4_lora_linear_bwd.argtypes = [P, P, i64, i64, i64, P, P, P, P, P, P, i32, f32, P, P, P, P, i64, P]
     L.nf4_merge_requantize.restype = i32
     L.nf4_merge_requantize.argtypes = [P, P, P, P, i64, i64, P, P, i32, f32, P, P, P]
     L.nf4_selftest_wait_timeout.restype = i32
@@ -225,6 +229,55 @@ def nf4_device_status(stream=None) -> int:
     st = lib().nf4_device_status(_stream(stream))
     _check("nf4_device_status", st)
     return st
+
+
+def nf4_lora_linear_bwd_workspace_size(M: int, N: int, K: int, r: int) -> int:
+    return int(lib().nf4_lora_linear_bwd_workspace_size(M, N, K, r))
+
+
+def nf4_lora_linear_bwd(g: torch.Tensor, x: Optional[torch.Tensor], packed: torch.Tensor,
+                        absmax_q: Optional[torch.Tensor], absmax2: torch.Tensor, offset: Optional[torch.Tensor],
+                        K: int, A: Optional[torch.Tensor] = None, B: Optional[torch.Tensor] = None,
+                        scaling: float = 1.0, want=("dx", "dA", "dB"), dx: Optional[torch.Tensor] = None,
+                        dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None):
+    """Backward of nf4_lora_linear_fwd: returns (dx bf16 [M, K], dA fp32 [r, K],
+    dB fp32 [N, r]), None for an output not in `want` (or without an adapter)."""
+    M, N = g.shape
+    _need(g, "g", torch.bfloat16)
+    r = 0
+    if A is not None and B is not None:
+        r = A.shape[0]
+        _need(A, "A", torch.bfloat16, r * K)
+        _need(B, "B", torch.bfloat16, N * r)
+    if "dx" in want:
+        if dx is None:
+            dx = torch.empty(M, K, dtype=torch.bfloat16, device=g.device)
+        _need(dx, "dx", torch.bfloat16, M * K)
+    else:
+        dx = None
+    if r > 0 and "dA" in want:
+        if dA is None:
+            dA = torch.empty(r, K, dtype=torch.float32, device=g.device)
+        _need(dA, "dA", torch.float32, r * K)
+    else:
+        dA = None
+    if r > 0 and "dB" in want:
+        if dB is None:
+            dB = torch.empty(N, r, dtype=torch.float32, device=g.device)
+        _need(dB, "dB", torch.float32, N * r)
+    else:
+        dB = None
+    if x is not None:
+        _need(x, "x", torch.bfloat16, M * K)
+    ws_bytes = nf4_lora_linear_bwd_workspace_size(M, N, K, r)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=g.device)
+    st = lib().nf4_lora_linear_bwd(_p(g), _p(x), M, K, N, _p(packed), _p(absmax_q), _p(absmax2), _p(offset), _p(A),
+                                   _p(B), r, float(scaling), _p(dx), _p(dA), _p(dB), _p(workspace),
+                                   0 if workspace is None else workspace.numel(), _stream(stream))
+    _check("nf4_lora_linear_bwd", st)
+    return dx, dA, dB
 
 
 def nf4_merge_requantize(packed: torch.Tensor, absmax_q: Optional[torch.Tensor], absmax2: torch.Tensor,

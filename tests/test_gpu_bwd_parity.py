@@ -1,0 +1,78 @@
+"""GPU parity of nf4_lora_linear_bwd (backward through the frozen base)
+against the oracle, with the matmul tolerance of the forward (max relative
+1e-2 with a 1e-2 rms floor, mean < 2e-3).
+
+"QLoRA: Mathematical Foundations ...", section "Gradient Computation":
+dx = g W~ + s (g B) A, dA = s (g B)^T x, dB = s g^T (x A^T)."""
+import numpy as np
+import pytest
+import torch
+
+import nf4_workloads as wl
+from conftest import MATMUL_MAX_REL, MATMUL_MEAN_REL, rel_error_stats
+
+pytestmark = pytest.mark.gpu
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def check(got: torch.Tensor, ref: np.ndarray):
+    mx, mean, fro = rel_error_stats(got.float().cpu().numpy().reshape(ref.shape), ref)
+    assert mx <= MATMUL_MAX_REL and mean < MATMUL_MEAN_REL, (mx, mean, fro)
+
+
+def inputs(M, K, N, r, seed, dq=True):
+    c = wl.LinearCase("bwd", M, K, N, r, 0.75, seed)
+    W, x, A, B = wl.linear_inputs(c)
+    g = torch.Generator().manual_seed(seed + 7)
+    dy = torch.randn(M, N, generator=g).to(torch.bfloat16)
+    return c, W, x, A, B, dy
+
+
+def run(nf4lib, oracle_mod, dev, M, K, N, r, seed, dq=True, rows=None, want=("dx", "dA", "dB")):
+    c, W, x, A, B, dy = inputs(M, K, N, r, seed, dq)
+    st = nf4lib.quantize_weight(W.to(dev), double_quant=dq)
+    dx, dA, dB = nf4lib.nf4_lora_linear_bwd(dy.to(dev), x.to(dev), st.packed, st.absmax_q, st.absmax2, st.offset, K,
+                                            A.to(dev), B.to(dev), c.scaling, want=want)
+    torch.cuda.synchronize()
+    packed = st.packed.cpu().numpy()
+    q8 = None if st.absmax_q is None else st.absmax_q.cpu().numpy()
+    sc = st.absmax2.cpu().numpy()
+    mu = None if st.offset is None else float(st.offset.cpu().numpy()[0])
+    ref = oracle_mod.lora_linear_bwd(bits(dy), bits(x), K, N, packed, q8, sc, mu, bits(A), bits(B), r, c.scaling,
+                                     rows=rows, want=want)
+    return dx, dA, dB, ref
+
+
+@pytest.mark.parametrize("M,K,N,r,dq", [(40, 192, 136, 16, True), (300, 512, 264, 64, True),
+                                        (256, 256, 128, 32, False), (17, 64, 8, 16, True),
+                                        (5, 320, 1000, 64, True), (600, 1024, 72, 16, True)])
+def test_bwd_small_shapes(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
+    dx, dA, dB, ref = run(nf4lib, oracle_mod, cuda_device, M, K, N, r, 300 + M + K + N, dq)
+    check(dx, ref["dx"])
+    check(dA, ref["dA"])
+    check(dB, ref["dB"])
+
+
+def test_bwd_dx_only_without_adapter(nf4lib, oracle_mod, cuda_device):
+    M, K, N = 130, 384, 200
+    c, W, x, A, B, dy = inputs(M, K, N, 16, 5)
+    st = nf4lib.quantize_weight(W.to(cuda_device))
+    dx, dA, dB = nf4lib.nf4_lora_linear_bwd(dy.to(cuda_device), None, st.packed, st.absmax_q, st.absmax2, st.offset,
+                                            K, want=("dx",))
+    torch.cuda.synchronize()
+    assert dA is None and dB is None
+    wb = nf4lib.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, N * K).view(N, K)
+    ref = torch.matmul(dy.to(cuda_device).float(), wb.float())  # library routine on the dequantized weight
+    check(dx, ref.cpu().numpy())
+
+
+def test_bwd_training_shape_sampled(nf4lib, oracle_mod, cuda_device):
+    c = wl.GEMM_TRAIN
+    rows = np.array([0, 1, 255, 256, 2047, 3000, 4095])
+    dx, dA, dB, ref = run(nf4lib, oracle_mod, cuda_device, c.M, c.K, c.N, c.r, c.seed, rows=rows)
+    check(dx[torch.as_tensor(rows)], ref["dx"])
+    check(dA, ref["dA"])
+    check(dB, ref["dB"])
