@@ -526,6 +526,39 @@ def run_suite(args):
                  peak_sustained=peaks["bf16_tflops_sustained"])
     torch.cuda.empty_cache()
 
+    # ---- backward through the frozen base: dx (fused NF4 GEMM) and the adapter gradients
+    for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
+        W, x, A, B = wl.linear_inputs(c)
+        g = torch.Generator().manual_seed(c.seed + 7)
+        dy = torch.randn(c.M, c.N, generator=g).to(torch.bfloat16).to(dev)
+        st = q.quantize_weight(W.to(dev))
+        xd, Ad, Bd = x.to(dev), A.to(dev), B.to(dev)
+        dxb = torch.empty(c.M, c.K, dtype=torch.bfloat16, device=dev)
+        dAb = torch.empty(c.r, c.K, device=dev)
+        dBb = torch.empty(c.N, c.r, device=dev)
+        wsb = torch.empty(q.nf4_lora_linear_bwd_workspace_size(c.M, c.N, c.K, c.r), dtype=torch.uint8, device=dev)
+
+        def f_dx():
+            q.nf4_lora_linear_bwd(dy, None, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
+                                  want=("dx",), dx=dxb, workspace=wsb)
+
+        def f_grads():
+            q.nf4_lora_linear_bwd(dy, xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
+                                  want=("dA", "dB"), dA=dAb, dB=dBb, workspace=wsb)
+
+        def f_all():
+            q.nf4_lora_linear_bwd(dy, xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
+                                  dx=dxb, dA=dAb, dB=dBb, workspace=wsb)
+        us_dx, us_gr, us_all = graph_us(f_dx, 3), graph_us(f_grads, 3), graph_us(f_all, 3)
+        q.nf4_device_status()
+        fl_dx = 2 * c.M * c.N * c.K + 2 * c.M * c.r * (c.N + c.K)
+        fl_gr = 2 * c.M * c.r * (c.N + c.K) * 2  # two down-projections + the two gradient products
+        emit(f"backward dx {c.name}", us_dx, fl_dx, "TFLOP/s", peak_sustained=peaks["bf16_tflops_sustained"])
+        emit(f"backward dA + dB {c.name}", us_gr, fl_gr, "TFLOP/s")
+        emit(f"backward dx + dA + dB {c.name}", us_all, fl_dx + fl_gr, "TFLOP/s")
+        del W, x, A, B, dy, st, xd, Ad, Bd, dxb, dAb, dBb, wsb
+        torch.cuda.empty_cache()
+
     # ---- merge the adapter into the quantized base and requantize (+ double
     # quantization of the new constants), and the error the requantization adds
     for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):

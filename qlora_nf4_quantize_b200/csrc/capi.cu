@@ -31,14 +31,11 @@ cudaError_t launch_merge_requantize(const uint8_t *packed, const uint8_t *q8, co
                                     float s, uint8_t *packed_out, float *absmax_out, cudaStream_t stream);
 int merge_max_rank();
 int64_t lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
-cudaError_t launch_lora_linear_bwd_dx(const void *g, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
-                                      const uint8_t *q8, const float *scales, const float *offset, const void *A,
-                                      const void *B, int r, float s, void *dx, void *workspace, unsigned *err,
-                                      cudaStream_t stream);
-cudaError_t launch_lora_grads(const void *g, const void *x, int64_t M, int64_t K, int64_t N, const void *A,
-                              const void *B, int r, float s, float *dA, float *dB, void *workspace,
-                              cudaStream_t stream);
-int64_t lora_grads_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+cudaError_t launch_lora_linear_bwd(const void *g, const void *x, int64_t M, int64_t K, int64_t N,
+                                   const uint8_t *packed, const uint8_t *q8, const float *scales,
+                                   const float *offset, const void *A, const void *B, int r, float s, void *dx,
+                                   float *dA, float *dB, void *workspace, unsigned *err, cudaStream_t stream,
+                                   int num_sms);
 }  // namespace nf4
 
 namespace {
@@ -180,8 +177,7 @@ nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N, c
 
 int64_t nf4_lora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     if (M < 0 || N < 0 || K < 0 || r <= 0) return 0;
-    const int64_t a = nf4::lora_bwd_workspace_bytes(M, N, K, r), b = nf4::lora_grads_workspace_bytes(M, N, K, r);
-    return a > b ? a : b;
+    return nf4::lora_bwd_workspace_bytes(M, N, K, r);
 }
 
 nf4_status nf4_lora_linear_bwd(const void *g, const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
@@ -208,16 +204,11 @@ nf4_status nf4_lora_linear_bwd(const void *g, const void *x, int64_t M, int64_t 
     cudaError_t st;
     unsigned *err = nf4::device_error_word(&st);
     if (st != cudaSuccess) return cuda_status(st);
-    if (dx) {
-        st = nf4::launch_lora_linear_bwd_dx(g, M, K, N, packed, absmax_q, absmax2, offset, lora ? A : nullptr,
-                                            lora ? B : nullptr, rr, scaling, dx, workspace, err, (cudaStream_t)stream);
-        if (st != cudaSuccess) return cuda_status(st);
-    }
-    if (dA || dB) {
-        st = nf4::launch_lora_grads(g, x, M, K, N, A, B, r, scaling, dA, dB, workspace, (cudaStream_t)stream);
-        if (st != cudaSuccess) return cuda_status(st);
-    }
-    return NF4_OK;
+    const int sms = sm_count(&st);
+    if (st != cudaSuccess) return cuda_status(st);
+    return cuda_status(nf4::launch_lora_linear_bwd(g, x, M, K, N, packed, absmax_q, absmax2, offset,
+                                                   lora ? A : nullptr, lora ? B : nullptr, rr, scaling, dx, dA, dB,
+                                                   workspace, err, (cudaStream_t)stream, sms));
 }
 
 nf4_status nf4_merge_requantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2,

@@ -340,8 +340,12 @@ cudaError_t launch_bwd_mode(const CUtensorMap &mg, const CUtensorMap &mu, int64_
 }  // namespace
 
 cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
-                                unsigned *err, cudaStream_t stream);
+                                unsigned *err, cudaStream_t stream, int split);
 int lora_rp(int r);
+int64_t grad_chunks(int64_t M, int64_t P);
+cudaError_t launch_lora_grad_product(const __nv_bfloat16 *X, int64_t P, const __nv_bfloat16 *T, int64_t ldt,
+                                     int64_t M, int r, float *part, float *out, int64_t sp, int64_t sj,
+                                     cudaStream_t stream);
 
 // dst[C, R] = src[R, C]^T (bf16)
 cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int64_t R, int64_t C, __nv_bfloat16 *dst,
@@ -353,43 +357,98 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int64_t R, int64_t C
 
 static int64_t align256(int64_t b) { return (b + 255) & ~(int64_t)255; }
 
-// Workspace: [u_hi | u_lo | 0] bf16 [M, RP], B^T bf16 [r, N], A^T bf16 [K, r].
-int64_t lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    if (r <= 0) return 0;
-    return align256(M * lora_rp(r) * 2) + align256((int64_t)r * N * 2) + align256(K * (int64_t)r * 2);
+namespace {
+
+// Workspace of the backward pass (all 256-byte aligned):
+//   u2 = [s g B hi | lo | 0]  bf16 [M, RP]   (dx extension and dA)
+//   t2 = [s x A^T hi | lo | 0] bf16 [M, RP]  (dB)
+//   B^T bf16 [r, N], A^T bf16 [K, r]
+//   fp32 partials of dB (chunks x N x 2r) and of dA (chunks x K x 2r)
+struct BwdWorkspace {
+    int64_t u2, t2, bt, at, part_b, part_a, total;
+};
+
+BwdWorkspace bwd_layout(int64_t M, int64_t N, int64_t K, int r) {
+    BwdWorkspace w{};
+    if (r <= 0) return w;
+    const int64_t rp = lora_rp(r);
+    w.u2 = 0;
+    w.t2 = w.u2 + align256(M * rp * 2);
+    w.bt = w.t2 + align256(M * rp * 2);
+    w.at = w.bt + align256((int64_t)r * N * 2);
+    w.part_b = w.at + align256(K * (int64_t)r * 2);
+    w.part_a = w.part_b + align256(grad_chunks(M, N) * N * 2 * r * 4);
+    w.total = w.part_a + align256(grad_chunks(M, K) * K * 2 * r * 4);
+    return w;
 }
 
-cudaError_t launch_lora_linear_bwd_dx(const void *g, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
-                                      const uint8_t *q8, const float *scales, const float *offset, const void *A,
-                                      const void *B, int r, float s, void *dx, void *workspace, unsigned *err,
-                                      cudaStream_t stream) {
+}  // namespace
+
+int64_t lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) { return bwd_layout(M, N, K, r).total; }
+
+// The whole backward pass (see include/nf4.h, nf4_lora_linear_bwd).  Launch
+// order: transposes, the down-projection(s), the dx GEMM (programmatic
+// dependent launch on the last down-projection, whose result it reads only in
+// its extension steps), then the two gradient products.
+cudaError_t launch_lora_linear_bwd(const void *g, const void *x, int64_t M, int64_t K, int64_t N,
+                                   const uint8_t *packed, const uint8_t *q8, const float *scales,
+                                   const float *offset, const void *A, const void *B, int r, float s, void *dx,
+                                   float *dA, float *dB, void *workspace, unsigned *err, cudaStream_t stream,
+                                   int num_sms) {
     if (M > 0x7FFFFFFF || K > 0x7FFFFFFF || N > 0x7FFFFFFF) return cudaErrorInvalidValue;
     const int rp = r > 0 ? lora_rp(r) : 0;
+    const BwdWorkspace L = bwd_layout(M, N, K, r);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    void *u2 = ws;
-    auto *Bt = reinterpret_cast<__nv_bfloat16 *>(ws + align256(M * rp * 2));
-    auto *At = reinterpret_cast<__nv_bfloat16 *>(ws + align256(M * rp * 2) + align256((int64_t)r * N * 2));
-    CUtensorMap mg, mu;
-    cudaError_t e = make_map(&mg, g, M, N, kGK, kGM, true);
-    if (e != cudaSuccess) return e;
+    auto *u2 = reinterpret_cast<__nv_bfloat16 *>(ws + L.u2);
+    auto *t2 = reinterpret_cast<__nv_bfloat16 *>(ws + L.t2);
+    auto *Bt = reinterpret_cast<__nv_bfloat16 *>(ws + L.bt);
+    auto *At = reinterpret_cast<__nv_bfloat16 *>(ws + L.at);
+    const auto *gp = static_cast<const __nv_bfloat16 *>(g);
+    const auto *xp = static_cast<const __nv_bfloat16 *>(x);
+    cudaError_t e = cudaSuccess;
+    // a long contraction over few 128-row tiles: split it over a 4-CTA cluster
+    auto split_for = [&](int64_t kdim) { return ((M + 127) / 128) * 4 <= num_sms && kdim >= 2048 ? 4 : 0; };
     if (r > 0) {
-        e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(B), N, r, Bt, stream);
-        if (e != cudaSuccess) return e;
-        e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(A), r, K, At, stream);
-        if (e != cudaSuccess) return e;
-        // u2 = s g (B^T)^T = s g B as [u_hi | u_lo | 0]
-        e = launch_lora_down_tc(g, Bt, M, N, r, s, u2, rp, err, stream);
-        if (e != cudaSuccess) return e;
-        e = make_map(&mu, u2, M, rp, kGK, kGM, true);
-    } else {
-        e = make_map(&mu, g, M, N, kGK, kGM, true);  // unused: no extension steps
+        const bool need_u = dx != nullptr || dA != nullptr;
+        if (need_u) {
+            e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(B), N, r, Bt, stream);
+            if (e != cudaSuccess) return e;
+        }
+        if (dx) {
+            e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(A), r, K, At, stream);
+            if (e != cudaSuccess) return e;
+        }
+        if (need_u) {  // u2 = s g (B^T)^T = s g B
+            e = launch_lora_down_tc(g, Bt, M, N, r, s, u2, rp, err, stream, split_for(N));
+            if (e != cudaSuccess) return e;
+        }
+        if (dB) {  // t2 = s x A^T
+            e = launch_lora_down_tc(x, A, M, K, r, s, t2, rp, err, stream, split_for(K));
+            if (e != cudaSuccess) return e;
+        }
     }
-    if (e != cudaSuccess) return e;
-    auto *dxp = static_cast<__nv_bfloat16 *>(dx);
-    if (q8 == nullptr) return launch_bwd_mode<2>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
-    if (offset == nullptr)
-        return launch_bwd_mode<1>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
-    return launch_bwd_mode<0>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+    if (dx) {
+        CUtensorMap mg, mu;
+        e = make_map(&mg, g, M, N, kGK, kGM, true);
+        if (e != cudaSuccess) return e;
+        e = r > 0 ? make_map(&mu, u2, M, rp, kGK, kGM, true) : make_map(&mu, g, M, N, kGK, kGM, true);
+        if (e != cudaSuccess) return e;
+        auto *dxp = static_cast<__nv_bfloat16 *>(dx);
+        if (q8 == nullptr) e = launch_bwd_mode<2>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+        else if (offset == nullptr)
+            e = launch_bwd_mode<1>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+        else e = launch_bwd_mode<0>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+        if (e != cudaSuccess) return e;
+    }
+    if (dB) {
+        e = launch_lora_grad_product(gp, N, t2, rp, M, r, reinterpret_cast<float *>(ws + L.part_b), dB, r, 1, stream);
+        if (e != cudaSuccess) return e;
+    }
+    if (dA) {
+        e = launch_lora_grad_product(xp, K, u2, rp, M, r, reinterpret_cast<float *>(ws + L.part_a), dA, 1, K, stream);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace nf4

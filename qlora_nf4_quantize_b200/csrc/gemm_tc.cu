@@ -339,14 +339,14 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUte
 // LoRA down-projection for large M on the tensor cores:
 //   t = s x A^T,  x [M, K] bf16,  A [r, K] bf16,  t as [t_hi | t_lo | 0] bf16
 // (same output as the warp-MMA kernel in lora_down.cu).  A thread-block
-// cluster of kDownSplit CTAs (1, 2 or 4) owns 128 rows of x and splits K: CTA c runs the
-// k-steps [c kt / kDownSplit, (c + 1) kt / kDownSplit) as
+// cluster of kSplit CTAs (1, 2 or 4) owns 128 rows of x and splits K: CTA c runs the
+// k-steps [c kt / kSplit, (c + 1) kt / kSplit) as
 // D[128, r] += X[128, k] A[r, k]^T with both operands brought by TMA (128-byte
 // swizzle, kDownStages-deep ring) and one thread issuing the MMAs (M = 128,
 // N = r, K = 16) into r fp32 columns of its tensor memory.  Each CTA then
 // stages its partial tile in shared memory, and CTA c finishes rows
-// [128 c / kDownSplit, 128 (c + 1) / kDownSplit) of the tile: it adds the
-// kDownSplit partials in rank order
+// [128 c / kSplit, 128 (c + 1) / kSplit) of the tile: it adds the
+// kSplit partials in rank order
 // through distributed shared memory (so the result does not depend on
 // timing), scales, and writes the hi/lo pair.
 // The kernel runs alongside the fused GEMM (programmatic dependent launch),
@@ -361,8 +361,7 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUte
 #endif
 constexpr int kDownStages = NF4_DOWN_STAGES;
 constexpr int kDownRows = 128;
-constexpr int kDownSplit = NF4_DOWN_SPLIT;  // cluster size along K
-static_assert(kDownSplit == 1 || kDownSplit == 2 || kDownSplit == 4, "128 rows split evenly over the cluster");
+constexpr int kDownSplit = NF4_DOWN_SPLIT;  // default cluster size along K
 
 template <int kR>
 struct __align__(1024) DownSmem {
@@ -399,7 +398,7 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
     return v;
 }
 
-template <int kR>
+template <int kR, int kSplit>
 __global__ void __launch_bounds__(128, 1)
     k_lora_down_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_a, int64_t M,
                    int64_t K, float scaling, __nv_bfloat16 *__restrict__ t2, int rp, unsigned *err) {
@@ -418,8 +417,8 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t rank = cluster_rank();
     const int64_t m0 = (int64_t)blockIdx.y * kDownRows;
     const int kt_all = (int)((K + 63) / 64);  // a partial last step reads zeros beyond K (TMA fill)
-    const int kt_begin = (int)((int64_t)rank * kt_all / kDownSplit);
-    const int kt_total = (int)((int64_t)(rank + 1) * kt_all / kDownSplit) - kt_begin;
+    const int kt_begin = (int)((int64_t)rank * kt_all / kSplit);
+    const int kt_total = (int)((int64_t)(rank + 1) * kt_all / kSplit) - kt_begin;
     if (threadIdx.x == 0) {
         for (int st = 0; st < kDownStages; ++st) {
             mbar_init(&S.full[st], 1);
@@ -508,16 +507,16 @@ __global__ void __launch_bounds__(128, 1)
     // finish rows [kRowsPer rank, kRowsPer (rank + 1)): thread t takes row
     // kRowsPer rank + t % kRowsPer and the kCw columns of group t / kRowsPer
     {
-        constexpr int kRowsPer = kDownRows / kDownSplit;
+        constexpr int kRowsPer = kDownRows / kSplit;
         constexpr int kCw = kR / (128 / kRowsPer);  // columns per thread (>= 4)
         static_assert(kCw % 4 == 0, "whole 4-column chunks");
         const int t = threadIdx.x;
         const int r_loc = kRowsPer * (int)rank + t % kRowsPer;
         const int64_t m = m0 + r_loc;
         const int cb = (t / kRowsPer) * kCw;
-        uint32_t base[kDownSplit];
+        uint32_t base[kSplit];
 #pragma unroll
-        for (int c = 0; c < kDownSplit; ++c) base[c] = map_rank(part + cb * kDownRows + r_loc, (uint32_t)c);
+        for (int c = 0; c < kSplit; ++c) base[c] = map_rank(part + cb * kDownRows + r_loc, (uint32_t)c);
 #pragma unroll 1
         for (int j0 = 0; j0 < kCw; j0 += 4) {
             float v[4];
@@ -525,7 +524,7 @@ __global__ void __launch_bounds__(128, 1)
             for (int j = 0; j < 4; ++j) {
                 float a = 0.0f;
 #pragma unroll
-                for (int c = 0; c < kDownSplit; ++c)
+                for (int c = 0; c < kSplit; ++c)
                     a += ld_cluster_f32(base[c] + (uint32_t)((j0 + j) * kDownRows * 4));
                 v[j] = a * scaling;
             }
@@ -555,25 +554,35 @@ __global__ void __launch_bounds__(128, 1)
     }
 }
 
-template <int kR>
+template <int kR, int kSplit>
 cudaError_t launch_down_tc(const CUtensorMap &mx, const CUtensorMap &ma, int64_t M, int64_t K, float s, void *t2,
                            int rp, unsigned *err, cudaStream_t stream) {
+    static_assert(kSplit == 1 || kSplit == 2 || kSplit == 4, "128 rows split evenly over the cluster");
     const size_t smem = sizeof(DownSmem<kR>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_lora_down_tc<kR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_lora_down_tc<kR, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kDownSplit, (unsigned)((M + kDownRows - 1) / kDownRows));
+    cfg.gridDim = dim3(kSplit, (unsigned)((M + kDownRows - 1) / kDownRows));
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kDownSplit;
+    attr[0].val.clusterDim.x = kSplit;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_lora_down_tc<kR>, mx, ma, M, K, s, static_cast<__nv_bfloat16 *>(t2), rp, err);
+    return cudaLaunchKernelEx(&cfg, k_lora_down_tc<kR, kSplit>, mx, ma, M, K, s, static_cast<__nv_bfloat16 *>(t2),
+                              rp, err);
+}
+
+template <int kR>
+cudaError_t launch_down_tc_split(const CUtensorMap &mx, const CUtensorMap &ma, int64_t M, int64_t K, float s,
+                                 void *t2, int rp, unsigned *err, cudaStream_t stream, int split) {
+    if (split == 4) return launch_down_tc<kR, 4>(mx, ma, M, K, s, t2, rp, err, stream);
+    return launch_down_tc<kR, kDownSplit>(mx, ma, M, K, s, t2, rp, err, stream);
 }
 
 }  // namespace
@@ -597,9 +606,12 @@ cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const
     return launch_mode<0>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
 }
 
-// Tensor-core LoRA down-projection (M > 16): see k_lora_down_tc.
+// Tensor-core LoRA down-projection: see k_lora_down_tc.  split: 0 = the
+// default (one CTA per 128 rows, the least SM time while a fused GEMM runs
+// alongside); 4 = K split over a 4-CTA cluster (a long contraction with
+// nothing running alongside).
 cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
-                                unsigned *err, cudaStream_t stream) {
+                                unsigned *err, cudaStream_t stream, int split) {
     if (M > 0x7FFFFFFF || K > 0x7FFFFFFF) return cudaErrorInvalidValue;
     CUtensorMap mx, ma;
     cudaError_t e = make_map(&mx, x, M, K, 64, kDownRows, true);
@@ -607,9 +619,9 @@ cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t
     e = make_map(&ma, A, r, K, 64, r, true);
     if (e != cudaSuccess) return e;
     switch (r) {
-        case 16: return launch_down_tc<16>(mx, ma, M, K, s, t2, rp, err, stream);
-        case 32: return launch_down_tc<32>(mx, ma, M, K, s, t2, rp, err, stream);
-        case 64: return launch_down_tc<64>(mx, ma, M, K, s, t2, rp, err, stream);
+        case 16: return launch_down_tc_split<16>(mx, ma, M, K, s, t2, rp, err, stream, split);
+        case 32: return launch_down_tc_split<32>(mx, ma, M, K, s, t2, rp, err, stream, split);
+        case 64: return launch_down_tc_split<64>(mx, ma, M, K, s, t2, rp, err, stream, split);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -12,7 +12,7 @@ cudaError_t launch_gemv(const void *x, int M, int64_t K, int64_t N, const uint8_
                         const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                         void *y, cudaStream_t stream, int num_sms);
 cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
-                                unsigned *err, cudaStream_t stream);
+                                unsigned *err, cudaStream_t stream, int split);
 cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                            const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                            void *y, cudaStream_t stream, int num_sms, unsigned *err_word);
@@ -46,7 +46,7 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
     if (r > 0) {
         // decode-size M: warp-MMA kernel; larger M: tensor-core kernel
         cudaError_t e = M <= kGemvMaxTokens ? launch_lora_down(x, A, M, K, r, scaling, workspace, stream)
-                                            : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream);
+                                            : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream, 0);
         if (e != cudaSuccess) return e;
     }
     if (M <= kGemvMaxTokens)

@@ -138,6 +138,10 @@ __global__ void k_grad_reduce(const float *__restrict__ part, int chunks, int64_
     out[p * sp + j * sj] = v;
 }
 
+}  // namespace
+
+// Token chunks of a gradient product over P columns (p-tiles x chunks ~ 296
+// CTAs; independent of the device so that workspace sizes are too).
 int64_t grad_chunks(int64_t M, int64_t P) {
     const int64_t ptiles = (P + kGP - 1) / kGP;
     int64_t c = (kGTargetCtas + ptiles - 1) / ptiles;
@@ -146,10 +150,11 @@ int64_t grad_chunks(int64_t M, int64_t P) {
     return c < 1 ? 1 : c;
 }
 
-int64_t align256g(int64_t b) { return (b + 255) & ~(int64_t)255; }
-
-cudaError_t launch_grad(const __nv_bfloat16 *X, int64_t P, const __nv_bfloat16 *T, int64_t ldt, int64_t M, int r,
-                        float *part, float *out, int64_t sp, int64_t sj, cudaStream_t stream) {
+// out[p sp + j sj] = sum_m X[m, p] (T2[m, j] + T2[m, r + j]) in fp32 (part:
+// grad_chunks(M, P) x P x 2r fp32 of scratch).
+cudaError_t launch_lora_grad_product(const __nv_bfloat16 *X, int64_t P, const __nv_bfloat16 *T, int64_t ldt,
+                                     int64_t M, int r, float *part, float *out, int64_t sp, int64_t sj,
+                                     cudaStream_t stream) {
     const int64_t chunks = grad_chunks(M, P);
     const int64_t m_chunk = ((M + chunks - 1) / chunks + kGMt - 1) / kGMt * kGMt;
     const dim3 grid((unsigned)((P + kGP - 1) / kGP), (unsigned)chunks);
@@ -164,61 +169,6 @@ cudaError_t launch_grad(const __nv_bfloat16 *X, int64_t P, const __nv_bfloat16 *
     const int64_t total = P * r;
     k_grad_reduce<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(part, (int)chunks, P, r, out, sp, sj);
     return cudaGetLastError();
-}
-
-}  // namespace
-
-int lora_rp(int r);
-cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
-                                unsigned *err, cudaStream_t stream);
-unsigned *device_error_word(cudaError_t *status);
-cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int64_t R, int64_t C, __nv_bfloat16 *dst,
-                                  cudaStream_t stream);
-
-// Workspace: t2 = [s x A^T hi | lo | 0] [M, RP], u2 likewise for s g B, B^T [r, N],
-// then the fp32 partials of dB and of dA.
-int64_t lora_grads_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    if (r <= 0) return 0;
-    const int64_t rp = lora_rp(r);
-    return 2 * align256g(M * rp * 2) + align256g((int64_t)r * N * 2) + align256g(grad_chunks(M, N) * N * 2 * r * 4) +
-           align256g(grad_chunks(M, K) * K * 2 * r * 4);
-}
-
-cudaError_t launch_lora_grads(const void *g, const void *x, int64_t M, int64_t K, int64_t N, const void *A,
-                              const void *B, int r, float s, float *dA, float *dB, void *workspace,
-                              cudaStream_t stream) {
-    const int rp = lora_rp(r);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    auto *t2 = reinterpret_cast<__nv_bfloat16 *>(ws);
-    auto *u2 = reinterpret_cast<__nv_bfloat16 *>(ws + align256g(M * rp * 2));
-    auto *Bt = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * align256g(M * rp * 2));
-    float *partB = reinterpret_cast<float *>(ws + 2 * align256g(M * rp * 2) + align256g((int64_t)r * N * 2));
-    float *partA = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(partB) +
-                                             align256g(grad_chunks(M, N) * N * 2 * r * 4));
-    cudaError_t e;
-    unsigned *err = device_error_word(&e);
-    if (e != cudaSuccess) return e;
-    // the tensor-core down-projection takes any M and any contraction length
-    // that is a multiple of 8 (TMA fills beyond the end with zeros)
-    auto down = [&](const void *xx, const void *aa, int64_t kk, void *out) -> cudaError_t {
-        return launch_lora_down_tc(xx, aa, M, kk, r, s, out, rp, err, stream);
-    };
-    if (dB) {
-        e = down(x, A, K, t2);  // s x A^T
-        if (e != cudaSuccess) return e;
-        e = launch_grad(static_cast<const __nv_bfloat16 *>(g), N, t2, rp, M, r, partB, dB, r, 1, stream);
-        if (e != cudaSuccess) return e;
-    }
-    if (dA) {
-        // B^T [r, N] so that the down-projection computes s g (B^T)^T = s g B
-        e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(B), N, r, Bt, stream);
-        if (e != cudaSuccess) return e;
-        e = down(g, Bt, N, u2);
-        if (e != cudaSuccess) return e;
-        e = launch_grad(static_cast<const __nv_bfloat16 *>(x), K, u2, rp, M, r, partA, dA, 1, K, stream);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
 }
 
 }  // namespace nf4
