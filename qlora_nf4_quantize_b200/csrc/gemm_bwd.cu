@@ -346,6 +346,9 @@ int64_t grad_chunks(int64_t M, int64_t P);
 cudaError_t launch_lora_grad_product(const __nv_bfloat16 *X, int64_t P, const __nv_bfloat16 *T, int64_t ldt,
                                      int64_t M, int r, float *part, float *out, int64_t sp, int64_t sj,
                                      cudaStream_t stream);
+cudaError_t launch_lora_grad_product_tc(const __nv_bfloat16 *X, int64_t P, const __nv_bfloat16 *T2, int rp, int64_t M,
+                                        int r, float *out, int64_t sp, int64_t sj, unsigned *err, cudaStream_t stream,
+                                        int num_sms);
 
 // dst[C, R] = src[R, C]^T (bf16)
 cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int64_t R, int64_t C, __nv_bfloat16 *dst,
@@ -356,6 +359,10 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16 *src, int64_t R, int64_t C
 }
 
 static int64_t align256(int64_t b) { return (b + 255) & ~(int64_t)255; }
+
+#ifndef NF4_GRAD_TC
+#define NF4_GRAD_TC 1
+#endif
 
 namespace {
 
@@ -440,12 +447,18 @@ cudaError_t launch_lora_linear_bwd(const void *g, const void *x, int64_t M, int6
         else e = launch_bwd_mode<0>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
         if (e != cudaSuccess) return e;
     }
+    // the adapter gradients: tensor-core products (NF4_GRAD_TC 0 selects the
+    // warp-MMA form, which needs the fp32 partial scratch)
     if (dB) {
-        e = launch_lora_grad_product(gp, N, t2, rp, M, r, reinterpret_cast<float *>(ws + L.part_b), dB, r, 1, stream);
+        e = NF4_GRAD_TC ? launch_lora_grad_product_tc(gp, N, t2, rp, M, r, dB, r, 1, err, stream, num_sms)
+                        : launch_lora_grad_product(gp, N, t2, rp, M, r, reinterpret_cast<float *>(ws + L.part_b), dB,
+                                                   r, 1, stream);
         if (e != cudaSuccess) return e;
     }
     if (dA) {
-        e = launch_lora_grad_product(xp, K, u2, rp, M, r, reinterpret_cast<float *>(ws + L.part_a), dA, 1, K, stream);
+        e = NF4_GRAD_TC ? launch_lora_grad_product_tc(xp, K, u2, rp, M, r, dA, 1, K, err, stream, num_sms)
+                        : launch_lora_grad_product(xp, K, u2, rp, M, r, reinterpret_cast<float *>(ws + L.part_a), dA,
+                                                   1, K, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -15,8 +15,8 @@
 // form).  Tiles of 32 token rows are double-buffered with cp.async.  Each
 // chunk writes its fp32 partial; a second kernel adds the chunks in index
 // order, so the result does not depend on timing.
-#include "mbarrier.cuh"
 #include "mma_util.cuh"
+#include "tc_util.cuh"
 
 namespace nf4 {
 namespace {
@@ -139,6 +139,248 @@ __global__ void k_grad_reduce(const float *__restrict__ part, int chunks, int64_
 }
 
 }  // namespace
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Tensor-core form (tcgen05): D[p, c] += X[m, p] T2[m, c] with M_mma = 128 p
+// columns of X, N_mma = RP columns of T2 ([T_hi | T_lo | 0]), K = token rows.
+// Both operands are read by TMA in their natural row-major form (boxes of 64
+// columns x 64 token rows, 128-byte swizzle) and handed to the MMA as
+// MN-major operands (instruction descriptor transpose bits): each 8-row x
+// 128-byte swizzle atom holds 64 consecutive columns of 8 tokens; atoms along
+// the columns are a box apart (leading byte offset 8 KB), atoms along the
+// tokens 1 KB apart (stride byte offset).  One thread issues TMA and MMA
+// (ring of kGStagesTc); a cluster of kSplit CTAs splits the token rows and
+// adds its fp32 partials in rank order through distributed shared memory; the
+// epilogue folds the hi and lo columns (c and c + r) and writes fp32.
+constexpr int kGStagesTc = 4;
+constexpr int kGBox = 64;                       // columns and token rows of one TMA box
+constexpr uint32_t kGBoxBytes = kGBox * kGBox * 2;  // 8 KB
+
+template <int kC>
+struct __align__(1024) GradSmem {
+    uint8_t a[kGStagesTc][2][kGBoxBytes];         // X: p 0-63, p 64-127
+    uint8_t b[kGStagesTc][kC / kGBox][kGBoxBytes];  // T2: c in boxes of 64
+    uint64_t full[kGStagesTc];
+    uint64_t empty[kGStagesTc];
+    uint64_t acc_full;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// MN-major operand in 128-byte swizzle atoms (8 rows along K x 64 elements
+// along M or N): leading byte offset = distance between atoms along M/N,
+// stride byte offset = distance between 8-row groups along K.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(const void *p, uint32_t lbo_bytes) {
+    const uint64_t addr = smem_addr(p);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;                      // start address
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next 64-column atom
+    d |= (uint64_t)(1024 >> 4) << 32;                   // stride byte offset: next 8 token rows
+    d |= (uint64_t)1 << 46;                             // descriptor version for tcgen05
+    d |= (uint64_t)2 << 61;                             // SWIZZLE_128B
+    return d;
+}
+
+__device__ __forceinline__ void cluster_sync_all_g() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int kR, int kSplit>
+__global__ void __launch_bounds__(128, 1)
+    k_grad_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_t, int64_t M,
+              int64_t P, float *__restrict__ out, int64_t sp, int64_t sj, unsigned *err) {
+    constexpr int kC = (2 * kR + 63) / 64 * 64;  // RP: columns of [T_hi | T_lo | 0]
+    constexpr int r = kR;
+    // D fp32, A bf16, B bf16, A and B MN-major (bits 15, 16), N = kC, M = 128
+    constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                                ((uint32_t)(kC >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+    constexpr uint32_t kStageBytes = (2 + kC / kGBox) * kGBoxBytes;
+    extern __shared__ uint8_t smem_raw[];
+    GradSmem<kC> &S =
+        *reinterpret_cast<GradSmem<kC> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    volatile int *abort = &S.abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t rank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    const int64_t p0 = (int64_t)blockIdx.y * 128;
+    const int kt_all = (int)((M + kGBox - 1) / kGBox);
+    const int kt_begin = (int)((int64_t)rank * kt_all / kSplit);
+    const int kt_total = (int)((int64_t)(rank + 1) * kt_all / kSplit) - kt_begin;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kGStagesTc; ++st) {
+            mbar_init(&S.full[st], 1);
+            mbar_init(&S.empty[st], 1);
+        }
+        mbar_init(&S.acc_full, 1);
+        S.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&S.tmem_base)),
+                     "r"((uint32_t)kC)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (threadIdx.x == 0 && kt_total > 0) {
+        bool ok = true;
+        auto issue = [&](int kt) -> bool {
+            const int st = kt % kGStagesTc;
+            const uint32_t ph = (uint32_t)(kt / kGStagesTc) & 1u;
+            if (!mbar_wait(&S.empty[st], ph ^ 1u, abort, err)) return false;
+            mbar_arrive_expect_tx(&S.full[st], kStageBytes);
+            const int m = (kt_begin + kt) * kGBox;
+            tma_load_2d(S.a[st][0], &tmap_x, &S.full[st], (int)p0, m);
+            tma_load_2d(S.a[st][1], &tmap_x, &S.full[st], (int)p0 + kGBox, m);
+#pragma unroll
+            for (int i = 0; i < kC / kGBox; ++i) tma_load_2d(S.b[st][i], &tmap_t, &S.full[st], kGBox * i, m);
+            return true;
+        };
+        int issued = 0;
+        for (; issued < kGStagesTc - 1 && issued < kt_total && ok; ++issued) ok = issue(issued);
+        for (int kt = 0; kt < kt_total && ok; ++kt) {
+            if (issued < kt_total) {
+                ok = issue(issued);
+                ++issued;
+                if (!ok) break;
+            }
+            const int st = kt % kGStagesTc;
+            if (!mbar_wait(&S.full[st], (uint32_t)(kt / kGStagesTc) & 1u, abort, err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint64_t ad = smem_desc_mn_sw128(S.a[st][0], kGBoxBytes);
+            const uint64_t bd = smem_desc_mn_sw128(S.b[st][0], kGBoxBytes);
+#pragma unroll
+            for (int kk = 0; kk < kGBox / 16; ++kk)  // 16 token rows = two 8-row atoms
+                tc_mma_ss(tmem, ad + (uint64_t)(kk * 2048 >> 4), bd + (uint64_t)(kk * 2048 >> 4), kIdesc,
+                          (kt | kk) != 0 ? 1u : 0u);
+            tc_commit(&S.empty[st]);
+        }
+        tc_commit(&S.acc_full);
+        for (int kt = issued - kGStagesTc < 0 ? 0 : issued - kGStagesTc; kt < issued; ++kt) {
+            unsigned long long t0 = global_ns();
+            while (!mbar_try_wait(&S.full[kt % kGStagesTc], (uint32_t)(kt / kGStagesTc) & 1u) &&
+                   global_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    }
+    __syncwarp();
+    // fold hi + lo into this CTA's partial tile, column-major [r][128] fp32, in
+    // the idle operand ring (every MMA that read it has completed)
+    float *part = reinterpret_cast<float *>(&S.a[0][0][0]);
+    const int row = 32 * warp + lane;
+    if (kt_total > 0 && __all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err))) {
+        tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+        for (int j0 = 0; j0 < r; j0 += 16) {
+            uint32_t hi[32], lo[32];
+            tc_load32(taddr + (uint32_t)(j0 & ~31), hi);
+            tc_load32(taddr + (uint32_t)((r + j0) & ~31), lo);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                part[(j0 + j) * 128 + row] =
+                    __uint_as_float(hi[(j0 & 31) + j]) + __uint_as_float(lo[((r + j0) & 31) + j]);
+        }
+    } else {
+        for (int j = 0; j < r; ++j) part[j * 128 + row] = 0.0f;
+    }
+    if constexpr (kSplit > 1) cluster_sync_all_g();
+    {
+        // CTA `rank` finishes rows [128 rank / kSplit, 128 (rank + 1) / kSplit):
+        // thread t takes row (t % rows) and every (128 / rows)-th column
+        constexpr int kRows = 128 / kSplit;
+        const int t = threadIdx.x;
+        const int rl = kRows * (int)rank + t % kRows;
+        const int64_t p = p0 + rl;
+        for (int j = t / kRows; j < r; j += 128 / kRows) {
+            float v = 0.0f;
+#pragma unroll
+            for (int c = 0; c < kSplit; ++c) {
+                uint32_t addr;
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                             : "=r"(addr)
+                             : "r"(smem_addr(part + j * 128 + rl)), "r"((uint32_t)c));
+                float x;
+                asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(addr) : "memory");
+                v += x;
+            }
+            if (p < P) out[p * sp + j * sj] = v;
+        }
+    }
+    if constexpr (kSplit > 1) cluster_sync_all_g();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)kC)
+                     : "memory");
+    }
+}
+
+template <int kR, int kSplit>
+cudaError_t launch_grad_tc_k(const CUtensorMap &mx, const CUtensorMap &mt, int64_t M, int64_t P, float *out,
+                             int64_t sp, int64_t sj, unsigned *err, cudaStream_t stream) {
+    constexpr int kC = (2 * kR + 63) / 64 * 64;
+    const size_t smem = sizeof(GradSmem<kC>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_grad_tc<kR, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kSplit, (unsigned)((P + 127) / 128));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kSplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_grad_tc<kR, kSplit>, mx, mt, M, P, out, sp, sj, err);
+}
+
+template <int kR>
+cudaError_t launch_grad_tc_r(const CUtensorMap &mx, const CUtensorMap &mt, int64_t M, int64_t P, float *out,
+                             int64_t sp, int64_t sj, unsigned *err, cudaStream_t stream, int split) {
+    if (split >= 4) return launch_grad_tc_k<kR, 4>(mx, mt, M, P, out, sp, sj, err, stream);
+    if (split == 2) return launch_grad_tc_k<kR, 2>(mx, mt, M, P, out, sp, sj, err, stream);
+    return launch_grad_tc_k<kR, 1>(mx, mt, M, P, out, sp, sj, err, stream);
+}
+
+}  // namespace
+
+// Tensor-core gradient product: out[p sp + j sj] = sum_m X[m, p] (T2[m, j] +
+// T2[m, r + j]); X bf16 [M, P] (P % 8 == 0), T2 bf16 [M, RP].
+cudaError_t launch_lora_grad_product_tc(const __nv_bfloat16 *X, int64_t P, const __nv_bfloat16 *T2, int rp, int64_t M,
+                                        int r, float *out, int64_t sp, int64_t sj, unsigned *err, cudaStream_t stream,
+                                        int num_sms) {
+    CUtensorMap mx, mt;
+    cudaError_t e = make_map(&mx, X, M, P, kGBox, kGBox, true);
+    if (e != cudaSuccess) return e;
+    e = make_map(&mt, T2, M, rp, kGBox, kGBox, true);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (P + 127) / 128;
+    const int split = tiles * 4 <= num_sms ? 4 : (tiles * 2 <= num_sms ? 2 : 1);
+    switch (r) {
+        case 16: return launch_grad_tc_r<16>(mx, mt, M, P, out, sp, sj, err, stream, split);
+        case 32: return launch_grad_tc_r<32>(mx, mt, M, P, out, sp, sj, err, stream, split);
+        case 64: return launch_grad_tc_r<64>(mx, mt, M, P, out, sp, sj, err, stream, split);
+        default: return cudaErrorInvalidValue;
+    }
+}
 
 // Token chunks of a gradient product over P columns (p-tiles x chunks ~ 296
 // CTAs; independent of the device so that workspace sizes are too).
