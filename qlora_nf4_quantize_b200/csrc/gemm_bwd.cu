@@ -11,20 +11,22 @@
 // Unlike the forward, the contraction runs along W's rows (n), across the
 // 64-blocks.  A CTA computes a 256 (tokens) x 256 (k) tile of dx as two MMA
 // accumulators of 128 tokens each (512 tensor-memory columns):
-//   D_h[m, k] += G[m, n] * WT[k, n],  M_mma = 128, N_mma = 256, K = 16
-//   G  = g tile (256 tokens x 64 n) brought by TMA with 128-byte swizzle;
-//   WT = the dequantized weight tile transposed (256 k x 64 n), written by
-//        two dequant warpgroups into shared memory in the same 128-byte
-//        swizzled K-major layout that TMA produces for G: a lane owns two
-//        rows n, n+1 and one 64-block of k, so it still dequantizes whole
-//        blocks with one register lookup table each (mma_util.cuh), and pairs
-//        the two rows' values of one k into one 32-bit word (one byte permute
-//        per two weights) for a conflict-free 32-bit shared store;
+//   D_h[m, k] += G[m, n] * W~[n, k],  M_mma = 128, N_mma = 256, K = 16
+//   G  = g tile (256 tokens x 64 n) brought by TMA with 128-byte swizzle,
+//        a K-major operand;
+//   W~ = the dequantized weight tile (64 n x 256 k) written by two dequant
+//        warpgroups into shared memory in its own row layout, as an MN-major
+//        operand (instruction descriptor transpose bit): 128-byte swizzle
+//        atoms of 8 rows n x 64 k, the four 64-k atoms of a row group 8 KB
+//        apart (leading byte offset), row groups 1 KB apart (stride byte
+//        offset).  A lane owns two rows and one 64-block, dequantizes it with
+//        one register lookup table (mma_util.cuh) and writes it with eight
+//        16-byte stores, conflict-free across the 8 rows of an atom;
 // both operands come from shared memory (SS MMA).  Each dequantized weight
 // feeds 256 tokens, as in the forward.  After the N / 64 weight steps, RP / 64
 // extension steps add the LoRA term the same way: G' = [u_hi | u_lo | 0]
 // (u scaled by s, as a bf16 hi/lo pair, from the down-projection kernel run
-// on g with B^T) and WT' = rows k of [A^T | A^T | 0].
+// on g with B^T) and W~' = rows of [A ; A ; 0] (A's own rows, no transpose).
 //
 // Warp roles (12 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
 // MMA issuer (one elected thread), warps 4..11 = two dequant warpgroups
@@ -46,10 +48,25 @@ constexpr uint32_t kGTmemCols = 512;
 constexpr uint32_t kGStageBytes = kGM * kGK * 2;  // also the WT tile: kGN x kGK bf16
 static_assert(kGM * kGK == kGN * kGK, "G and WT tiles have the same size");
 
-// UMMA instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both
-// K-major, N = 256, M = 128.
-constexpr uint32_t kGIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kGN >> 3) << 17) |
+// UMMA instruction descriptor, kind::f16: D fp32, A bf16 K-major, B bf16
+// MN-major (bit 16), N = 256, M = 128.
+constexpr uint32_t kGIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(kGN >> 3) << 17) |
                              ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t kGAtomCol = kGK * 128;  // bytes of one 64-k column of atoms (64 rows x 128 B)
+
+// MN-major operand in 128-byte swizzle atoms (8 rows along K x 64 elements
+// along N): leading byte offset = distance between atoms along N, stride byte
+// offset = distance between 8-row groups along K.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128_b(const void *p, uint32_t lbo_bytes) {
+    const uint64_t addr = smem_addr(p);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
 
 struct __align__(1024) BwdSmem {
     uint8_t g[kGStages][kGStageBytes];
@@ -88,13 +105,10 @@ __device__ __forceinline__ void load_block(const uint8_t *__restrict__ packed, c
     }
 }
 
-// byte offset of the 32-bit word (k-row kk, n-pair p) in a 128-byte swizzled tile
-__device__ __forceinline__ uint32_t wt_offset(int kk, int p) {
-    return (uint32_t)kk * 128u + ((uint32_t)((p >> 2) ^ (kk & 7)) << 4) + (uint32_t)(p & 3) * 4u;
-}
-
-__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+// byte offset of 16-byte chunk c (k = 8c .. 8c+7 of 64-k block a) of row n
+// (0..63) in the MN-major swizzled weight tile
+__device__ __forceinline__ uint32_t w_offset(int n, int a, int c) {
+    return (uint32_t)a * kGAtomCol + (uint32_t)n * 128u + ((uint32_t)(c ^ (n & 7)) << 4);
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
@@ -107,7 +121,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     k_gemm_bwd(const __grid_constant__ CUtensorMap tmap_g, const __grid_constant__ CUtensorMap tmap_u, int64_t M,
                int64_t K, int64_t N, const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
                const float *__restrict__ scales, const float *__restrict__ offset,
-               const __nv_bfloat16 *__restrict__ At, int r, int rp, __nv_bfloat16 *__restrict__ dx, unsigned *err) {
+               const __nv_bfloat16 *__restrict__ Al, int r, int rp, __nv_bfloat16 *__restrict__ dx, unsigned *err) {
     extern __shared__ uint8_t smem_raw[];
     BwdSmem &S = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int *abort = &S.abort;
@@ -177,12 +191,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 tc_fence_after();
                 const uint64_t a0 = smem_desc_sw128(S.g[s]);
                 const uint64_t a1 = smem_desc_sw128(S.g[s] + kGStageBytes / 2);  // tokens 128..255
-                const uint64_t bd = smem_desc_sw128(S.wt[s]);
+                const uint64_t bd = smem_desc_mn_sw128_b(S.wt[s], kGAtomCol);
 #pragma unroll
                 for (int kk = 0; kk < kGK / 16; ++kk) {
                     const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
-                    tc_mma_ss(tmem, a0 + 2ull * kk, bd + 2ull * kk, kGIdesc, acc);
-                    tc_mma_ss(tmem + 256u, a1 + 2ull * kk, bd + 2ull * kk, kGIdesc, acc);
+                    const uint64_t b = bd + (uint64_t)(kk * 2048 >> 4);  // 16 rows n = two atoms along K
+                    tc_mma_ss(tmem, a0 + 2ull * kk, b, kGIdesc, acc);
+                    tc_mma_ss(tmem + 256u, a1 + 2ull * kk, b, kGIdesc, acc);
                 }
                 any = true;
                 tc_commit(&S.g_empty[s]);
@@ -230,33 +245,31 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.w_empty[s], ph ^ 1u, abort, err));
                 if (!ok) break;
-                // word j of a row holds k = 2j (low half) and 2j + 1 (high half);
-                // the tile row k holds (n = 2p, n = 2p + 1) in one word
+                // word j of a row holds k = 2j (low half) and 2j + 1 (high half):
+                // chunk c = words 4c .. 4c + 3, rows 2p and 2p + 1 of the step
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int kk = 64 * q + 2 * j;
-                    sts32(tile + wt_offset(kk, p), __byte_perm(va[j], vb[j], 0x5410));
-                    sts32(tile + wt_offset(kk + 1, p), __byte_perm(va[j], vb[j], 0x7632));
+                for (int c = 0; c < 8; ++c) {
+                    sts128(tile + w_offset(2 * p, q, c), make_uint4(va[4 * c], va[4 * c + 1], va[4 * c + 2], va[4 * c + 3]));
+                    sts128(tile + w_offset(2 * p + 1, q, c),
+                           make_uint4(vb[4 * c], vb[4 * c + 1], vb[4 * c + 2], vb[4 * c + 3]));
                 }
                 ca = na;
                 cb = nb;
             } else {
-                // rows kk of [A^T | A^T | 0], columns [64 e, 64 e + 64): two rows per thread
+                // rows j of [A ; A ; 0] (row j -> A[j mod r] for j < 2r), columns
+                // k0 + 64 q .. + 63: rows 2p and 2p + 1 of the step
                 const int e = kt - kn_steps;
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.w_empty[s], ph ^ 1u, abort, err));
                 if (!ok) break;
+                const int64_t k = k0 + 64 * q;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int kk = 32 * q + lane + 128 * half;
-                    const int64_t k = k0 + kk;
+                for (int i = 0; i < 2; ++i) {
+                    const int j = 64 * e + 2 * p + i;
+                    const bool v = j < 2 * r && k < K;
+                    const uint4 *src = reinterpret_cast<const uint4 *>(Al + (int64_t)(v ? j % r : 0) * K + (v ? k : 0));
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int j0 = 64 * e + 8 * c;
-                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                        if (k < K && j0 < 2 * r)
-                            v = __ldg(reinterpret_cast<const uint4 *>(At + k * r + (j0 % r)));
-                        sts128(tile + (uint32_t)kk * 128u + ((uint32_t)(c ^ (kk & 7)) << 4), v);
-                    }
+                    for (int c = 0; c < 8; ++c)
+                        sts128(tile + w_offset(2 * p + i, q, c), v ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u));
                 }
             }
             // the tile is read by the tensor cores (async proxy)
@@ -318,7 +331,7 @@ __global__ void k_transpose_bf16(const __nv_bfloat16 *__restrict__ src, int64_t 
 template <int kMode>
 cudaError_t launch_bwd_mode(const CUtensorMap &mg, const CUtensorMap &mu, int64_t M, int64_t K, int64_t N,
                             const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
-                            const __nv_bfloat16 *At, int r, int rp, __nv_bfloat16 *dx, unsigned *err,
+                            const __nv_bfloat16 *Al, int r, int rp, __nv_bfloat16 *dx, unsigned *err,
                             cudaStream_t stream) {
     const size_t smem = sizeof(BwdSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_gemm_bwd<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -333,7 +346,7 @@ cudaError_t launch_bwd_mode(const CUtensorMap &mg, const CUtensorMap &mu, int64_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
-    return cudaLaunchKernelEx(&cfg, k_gemm_bwd<kMode>, mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dx,
+    return cudaLaunchKernelEx(&cfg, k_gemm_bwd<kMode>, mg, mu, M, K, N, packed, q8, scales, offset, Al, r, rp, dx,
                               err);
 }
 
@@ -369,10 +382,10 @@ namespace {
 // Workspace of the backward pass (all 256-byte aligned):
 //   u2 = [s g B hi | lo | 0]  bf16 [M, RP]   (dx extension and dA)
 //   t2 = [s x A^T hi | lo | 0] bf16 [M, RP]  (dB)
-//   B^T bf16 [r, N], A^T bf16 [K, r]
+//   B^T bf16 [r, N]
 //   fp32 partials of dB (chunks x N x 2r) and of dA (chunks x K x 2r)
 struct BwdWorkspace {
-    int64_t u2, t2, bt, at, part_b, part_a, total;
+    int64_t u2, t2, bt, part_b, part_a, total;
 };
 
 BwdWorkspace bwd_layout(int64_t M, int64_t N, int64_t K, int r) {
@@ -382,8 +395,7 @@ BwdWorkspace bwd_layout(int64_t M, int64_t N, int64_t K, int r) {
     w.u2 = 0;
     w.t2 = w.u2 + align256(M * rp * 2);
     w.bt = w.t2 + align256(M * rp * 2);
-    w.at = w.bt + align256((int64_t)r * N * 2);
-    w.part_b = w.at + align256(K * (int64_t)r * 2);
+    w.part_b = w.bt + align256((int64_t)r * N * 2);
     w.part_a = w.part_b + align256(grad_chunks(M, N) * N * 2 * r * 4);
     w.total = w.part_a + align256(grad_chunks(M, K) * K * 2 * r * 4);
     return w;
@@ -409,7 +421,7 @@ cudaError_t launch_lora_linear_bwd(const void *g, const void *x, int64_t M, int6
     auto *u2 = reinterpret_cast<__nv_bfloat16 *>(ws + L.u2);
     auto *t2 = reinterpret_cast<__nv_bfloat16 *>(ws + L.t2);
     auto *Bt = reinterpret_cast<__nv_bfloat16 *>(ws + L.bt);
-    auto *At = reinterpret_cast<__nv_bfloat16 *>(ws + L.at);
+    const auto *Al = static_cast<const __nv_bfloat16 *>(A);
     const auto *gp = static_cast<const __nv_bfloat16 *>(g);
     const auto *xp = static_cast<const __nv_bfloat16 *>(x);
     cudaError_t e = cudaSuccess;
@@ -419,10 +431,6 @@ cudaError_t launch_lora_linear_bwd(const void *g, const void *x, int64_t M, int6
         const bool need_u = dx != nullptr || dA != nullptr;
         if (need_u) {
             e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(B), N, r, Bt, stream);
-            if (e != cudaSuccess) return e;
-        }
-        if (dx) {
-            e = launch_transpose_bf16(static_cast<const __nv_bfloat16 *>(A), r, K, At, stream);
             if (e != cudaSuccess) return e;
         }
         if (need_u) {  // u2 = s g (B^T)^T = s g B
@@ -441,10 +449,10 @@ cudaError_t launch_lora_linear_bwd(const void *g, const void *x, int64_t M, int6
         e = r > 0 ? make_map(&mu, u2, M, rp, kGK, kGM, true) : make_map(&mu, g, M, N, kGK, kGM, true);
         if (e != cudaSuccess) return e;
         auto *dxp = static_cast<__nv_bfloat16 *>(dx);
-        if (q8 == nullptr) e = launch_bwd_mode<2>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+        if (q8 == nullptr) e = launch_bwd_mode<2>(mg, mu, M, K, N, packed, q8, scales, offset, Al, r, rp, dxp, err, stream);
         else if (offset == nullptr)
-            e = launch_bwd_mode<1>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
-        else e = launch_bwd_mode<0>(mg, mu, M, K, N, packed, q8, scales, offset, At, r, rp, dxp, err, stream);
+            e = launch_bwd_mode<1>(mg, mu, M, K, N, packed, q8, scales, offset, Al, r, rp, dxp, err, stream);
+        else e = launch_bwd_mode<0>(mg, mu, M, K, N, packed, q8, scales, offset, Al, r, rp, dxp, err, stream);
         if (e != cudaSuccess) return e;
     }
     // the adapter gradients: tensor-core products (NF4_GRAD_TC 0 selects the
