@@ -40,23 +40,14 @@ namespace nf4 {
 namespace {
 
 constexpr int kBN = 128;                   // weight rows per CTA (MMA M)
-constexpr int kBT = 256;                   // tokens per CTA (MMA N)
 constexpr int kBK = 64;                    // k per pipeline step
 #ifndef NF4_GEMM_STAGES
 #define NF4_GEMM_STAGES 4
 #endif
-constexpr int kStages = NF4_GEMM_STAGES;  // x tiles in shared memory and A tiles in tensor memory
-static_assert(256 + 32 * kStages <= 512, "tensor memory: 256 accumulator columns + 32 per A stage");
-// Dequant warpgroups: warpgroup h produces the k-steps with index % kWG == h.
+// Dequant warpgroups: warpgroup h produces the k-steps with index % WG == h.
 #ifndef NF4_GEMM_WG
 #define NF4_GEMM_WG 2
 #endif
-constexpr int kWG = NF4_GEMM_WG;
-constexpr int kThreads = 128 + 128 * kWG;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol = 0;            // accumulator: columns [0, 256)
-constexpr uint32_t kACol = 256;            // A stages: columns [256 + 32 s, +32)
-constexpr uint32_t kXStageBytes = kBT * kBK * 2;
 // Dequantization lookup per warpgroup: bit h set = warpgroup h uses the
 // shared-memory pair table (one shared load per two weights), clear = the
 // register lookup table (byte permutes on the integer pipe).  Mixing the two
@@ -66,17 +57,49 @@ constexpr uint32_t kXStageBytes = kBT * kBK * 2;
 #endif
 constexpr int kLutMask = NF4_GEMM_LUT_MASK;
 
-// UMMA instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both
-// K-major, N = 256, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBT >> 3) << 17) |
-                            ((uint32_t)(kBN >> 4) << 24);
+constexpr uint32_t pow2_at_least(uint32_t v) {
+    uint32_t p = 32;
+    while (p < v) p <<= 1;
+    return p;
+}
 
+// Token tile BT (MMA N), pipeline depth and dequant warpgroups of one
+// instantiation: BT = 256 for the large-M GEMM; BT = 16 serves decode-size M
+// when built with NF4_SMALL_M_TC=1 (one 128-row tile per CTA: 86 CTAs for an
+// 11008-row weight, and a k-step rate bound by the dequant warps' latency,
+// measured slower than the warp-MMA GEMV kernels, so not the default).
+template <int BT_, int STAGES_, int WG_>
+struct TileCfg {
+    static constexpr int BT = BT_, Stages = STAGES_, WG = WG_;
+    static constexpr int Threads = 128 + 128 * WG;
+    static constexpr uint32_t AccCols = BT < 32 ? 32 : BT;   // accumulator: columns [0, AccCols)
+    static constexpr uint32_t ACol = AccCols;                // A stages: columns [ACol + 32 s, +32)
+    static constexpr uint32_t TmemCols = pow2_at_least(AccCols + 32 * Stages);
+    static constexpr uint32_t XStageBytes = BT * kBK * 2;
+    // UMMA instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both
+    // K-major, N = BT, M = 128.
+    static constexpr uint32_t Idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BT >> 3) << 17) |
+                                      ((uint32_t)(kBN >> 4) << 24);
+    static_assert(TmemCols <= 512, "tensor memory: accumulator + 32 columns per A stage");
+    static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M = 128");
+};
+
+using CfgLarge = TileCfg<256, NF4_GEMM_STAGES, NF4_GEMM_WG>;
+#ifndef NF4_GEMV_TC_WG
+#define NF4_GEMV_TC_WG 3
+#endif
+#ifndef NF4_GEMV_TC_STAGES
+#define NF4_GEMV_TC_STAGES 6
+#endif
+using CfgSmall = TileCfg<16, NF4_GEMV_TC_STAGES, NF4_GEMV_TC_WG>;
+
+template <class C>
 struct __align__(1024) SmemLayout {
-    uint8_t x[kStages][kXStageBytes];
-    uint64_t x_full[kStages];
-    uint64_t x_empty[kStages];
-    uint64_t a_full[kStages];
-    uint64_t a_empty[kStages];
+    uint8_t x[C::Stages][C::XStageBytes];
+    uint64_t x_full[C::Stages];
+    uint64_t x_empty[C::Stages];
+    uint64_t a_full[C::Stages];
+    uint64_t a_empty[C::Stages];
     float2 pairs[kLutMask != 0 ? kPairTableFloat2 : 1];
     uint64_t acc_full;
     uint64_t drain;
@@ -84,12 +107,13 @@ struct __align__(1024) SmemLayout {
     int abort;
 };
 
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -146,15 +170,18 @@ __device__ __forceinline__ void lora_step(const __nv_bfloat16 *__restrict__ Bl, 
     }
 }
 
-template <int kMode>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kMode, class C>
+__global__ void __launch_bounds__(C::Threads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_t,
               const __grid_constant__ CUtensorMap tmap_y, int64_t M,
               int64_t K, int64_t N, const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
               const float *__restrict__ scales, const float *__restrict__ offset,
               const __nv_bfloat16 *__restrict__ Bl, int r, int rp, __nv_bfloat16 *__restrict__ y, unsigned *err) {
     extern __shared__ uint8_t smem_raw[];
-    SmemLayout &S = *reinterpret_cast<SmemLayout *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int kBT = C::BT, kStages = C::Stages, kWG = C::WG;
+    constexpr uint32_t kTmemCols = C::TmemCols, kAccCol = 0, kACol = C::ACol, kXStageBytes = C::XStageBytes;
+    SmemLayout<C> &S =
+        *reinterpret_cast<SmemLayout<C> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int *abort = &S.abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -226,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t bdesc = smem_desc_sw128(S.x[s]);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk) {
-                    tc_mma_ts(tmem + kAccCol, tmem + kACol + 32u * s + 8u * kk, bdesc + 2ull * kk,
+                    tc_mma_ts(tmem + kAccCol, tmem + kACol + 32u * s + 8u * kk, bdesc + 2ull * kk, C::Idesc,
                               (kt | kk) != 0 ? 1u : 0u);
                 }
                 any = true;
@@ -283,13 +310,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(&S.x[0][0]);
 #pragma unroll 1
-            for (int c = h; c < kBT / 32; c += kWG) {  // 32-token chunks of the tile
+            for (int c = h; c < (kBT + 31) / 32; c += kWG) {  // 32-token chunks of the tile
                 uint32_t v[32];
-                tc_load32(lane_base + kAccCol + 32u * c, v);
+                tc_load32(lane_base + kAccCol + 32u * c, v);  // the allocation holds >= 32 columns
                 tc_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    stage[(32 * c + i) * kBN + row_in_tile] = __float2bfloat16_rn(__uint_as_float(v[i]));
+                    if (32 * c + i < kBT)
+                        stage[(32 * c + i) * kBN + row_in_tile] = __float2bfloat16_rn(__uint_as_float(v[i]));
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
@@ -314,16 +342,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int kMode>
+template <int kMode, class C>
 cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUtensorMap &my, int64_t M, int64_t K, int64_t N,
                         const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
                         const __nv_bfloat16 *Bl, int r, int rp, __nv_bfloat16 *y, unsigned *err, cudaStream_t stream) {
-    const size_t smem = sizeof(SmemLayout) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = sizeof(SmemLayout<C>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<kMode, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBT - 1) / kBT));
-    cfg.blockDim = dim3(kThreads);
+    cfg.gridDim = dim3((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + C::BT - 1) / C::BT));
+    cfg.blockDim = dim3(C::Threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -331,8 +359,29 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUte
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
-    return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode>, mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, y,
+    return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode, C>, mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, y,
                               err);
+}
+
+template <class C>
+cudaError_t launch_cfg(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
+                       const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
+                       void *y, cudaStream_t stream, unsigned *err_word) {
+    CUtensorMap mx, mt, my;
+    cudaError_t e = make_map(&mx, x, M, K, kBK, C::BT, true);
+    if (e != cudaSuccess) return e;
+    if (r > 0) e = make_map(&mt, t2, M, rp, kBK, C::BT, true);
+    else e = make_map(&mt, x, M, K, kBK, C::BT, true);  // unused: no extension steps
+    if (e != cudaSuccess) return e;
+    e = make_map(&my, y, M, N, kBN, C::BT, false);
+    if (e != cudaSuccess) return e;
+    auto *Bl = static_cast<const __nv_bfloat16 *>(B);
+    auto *yp = static_cast<__nv_bfloat16 *>(y);
+    if (q8 == nullptr)
+        return launch_mode<2, C>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+    if (offset == nullptr)
+        return launch_mode<1, C>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+    return launch_mode<0, C>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -591,19 +640,9 @@ cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const
                            const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                            void *y, cudaStream_t stream, int /*num_sms*/, unsigned *err_word) {
     if (M > 0x7FFFFFFF || K > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    CUtensorMap mx, mt, my;
-    cudaError_t e = make_map(&mx, x, M, K, kBK, kBT, true);
-    if (e != cudaSuccess) return e;
-    if (r > 0) e = make_map(&mt, t2, M, rp, kBK, kBT, true);
-    else e = make_map(&mt, x, M, K, kBK, kBT, true);  // unused: no extension steps
-    if (e != cudaSuccess) return e;
-    e = make_map(&my, y, M, N, kBN, kBT, false);
-    if (e != cudaSuccess) return e;
-    auto *Bl = static_cast<const __nv_bfloat16 *>(B);
-    auto *yp = static_cast<__nv_bfloat16 *>(y);
-    if (q8 == nullptr) return launch_mode<2>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
-    if (offset == nullptr) return launch_mode<1>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
-    return launch_mode<0>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+    if (M <= CfgSmall::BT)
+        return launch_cfg<CfgSmall>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream, err_word);
+    return launch_cfg<CfgLarge>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream, err_word);
 }
 
 // Tensor-core LoRA down-projection: see k_lora_down_tc.  split: 0 = the

@@ -18,6 +18,9 @@ cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const
                            void *y, cudaStream_t stream, int num_sms, unsigned *err_word);
 
 constexpr int kGemvMaxTokens = 16;
+#ifndef NF4_SMALL_M_TC
+#define NF4_SMALL_M_TC 0
+#endif
 
 // Device error word: one per device, cleared by nf4_device_status().
 static __device__ unsigned g_error_word;
@@ -49,7 +52,9 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
                                             : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream, 0);
         if (e != cudaSuccess) return e;
     }
-    if (M <= kGemvMaxTokens)
+    // decode-size M: the warp-MMA GEMV kernels, or (built with
+    // NF4_SMALL_M_TC=1) the tcgen05 pipeline with a 16-token tile
+    if (M <= kGemvMaxTokens && !NF4_SMALL_M_TC)
         return launch_gemv(x, (int)M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms);
     return launch_gemm_tc(x, M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms,
                           err_word);
