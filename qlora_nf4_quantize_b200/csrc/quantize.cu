@@ -92,9 +92,9 @@ __device__ __forceinline__ void load8(const void *w, int64_t e0, int64_t n, floa
 }
 
 // One group = 8 consecutive elements, owned by one thread; the 8 lanes of a
-// lane group (lane / 8) own one 64-block.  A thread handles kUnroll groups per
-// iteration, 256 groups apart (so lane groups still cover whole blocks), and
-// issues all their loads before any arithmetic.
+// lane group (lane / 8) own one 64-block.  Consecutive groups of a thread are
+// a grid stride apart (a multiple of 8 groups, so lane groups still cover
+// whole blocks).
 template <bool kBf16>
 __device__ __forceinline__ void quantize_group(float v[8], int64_t g, int64_t e0, int64_t n, int lane,
                                                const float *s_t, const uint32_t *s_cell,
@@ -109,47 +109,59 @@ __device__ __forceinline__ void quantize_group(float v[8], int64_t g, int64_t e0
     if (e0 >= n) return;
     if ((lane & 7) == 0) absmax[g >> 3] = c1;
 
-    int code[8];
+    uint32_t word;  // byte j = code[2j] << 4 | code[2j+1], bytes 0..3
     if (c1 == 0.0f) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) code[i] = 7;
-    } else if (c1 < 0x1p-125f || c1 >= 0x1p125f) {
-        // c1 < 2^-125 or >= 2^125: 1/c1 may overflow or be subnormal, so
-        // the 2^-22 error bound of the fast path would not hold
-#pragma unroll
-        for (int i = 0; i < 8; ++i) code[i] = exact_code(v[i], c1, s_t);
+        word = 0x77777777u;
     } else {
-        const float rc = __frcp_rn(c1);
-        bool amb = false;
+        bool amb = true;  // take the exact path
+        word = 0;
+        if (c1 >= 0x1p-125f && c1 < 0x1p125f) {
+            // (outside this range 1/c1 may overflow or be subnormal, so the
+            // 2^-22 error bound of the fast path would not hold)
+            const float rc = __frcp_rn(c1);
+            uint64_t rc2, k64, kmagic;
+            asm("mov.b64 %0, {%1, %1};" : "=l"(rc2) : "f"(rc));
+            asm("mov.b64 %0, {%1, %1};" : "=l"(k64) : "f"(64.0f));
+            asm("mov.b64 %0, {%1, %1};" : "=l"(kmagic) : "f"(12582976.0f));  // 1.5 * 2^23 + 64
+            float dmin = 1.0f;  // smallest |q - t| of the group
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float q = __fmul_rn(v[i], rc);
-            const float f = __fmaf_rn(q, 64.0f, 12582976.0f);  // 1.5 * 2^23 + 64: RN(64 q) + 64 in the low bits
-            // RN(64 q) + 64 is in [0, 128] for finite inputs; the byte mask
-            // keeps any input inside the 256-entry table
-            const uint32_t e = s_cell[__float_as_uint(f) & 0xFFu];
-            const float t = __uint_as_float(e);
-            code[i] = (int)(e & 15u) + ((q > t) ? 1 : 0);
-            amb |= fabsf(q - t) <= kAmbiguity;
+            for (int i = 0; i < 8; i += 2) {
+                // q = RN(w * RN(1/c1)) and RN(64 q) + 64 in the low bits of
+                // f = RN(64 q + 1.5 * 2^23 + 64), two elements per packed op
+                uint64_t vv, qq, ff;
+                asm("mov.b64 %0, {%1, %2};" : "=l"(vv) : "f"(v[i]), "f"(v[i + 1]));
+                asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(qq) : "l"(vv), "l"(rc2));
+                asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(ff) : "l"(qq), "l"(k64), "l"(kmagic));
+                float q[2], f[2];
+                asm("mov.b64 {%0, %1}, %2;" : "=f"(q[0]), "=f"(q[1]) : "l"(qq));
+                asm("mov.b64 {%0, %1}, %2;" : "=f"(f[0]), "=f"(f[1]) : "l"(ff));
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    // RN(64 q) + 64 is in [0, 128] for finite inputs; the byte
+                    // mask keeps any input inside the 256-entry table
+                    const uint32_t e = s_cell[__float_as_uint(f[j]) & 0xFFu];
+                    const float t = __uint_as_float(e);
+                    const uint32_t code = (e & 15u) + ((q[j] > t) ? 1u : 0u);
+                    const int el = i + j;  // element 2m in the high nibble of byte m
+                    word += code << (8 * (el >> 1) + ((el & 1) ? 0 : 4));
+                    dmin = fminf(dmin, fabsf(q[j] - t));
+                }
+            }
+            amb = dmin <= kAmbiguity;  // rare: some quotient is within 2^-18 of a threshold
         }
-        if (amb) {  // rare: some quotient is within 2^-18 of a threshold
+        if (amb) {
+            word = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) code[i] = exact_code(v[i], c1, s_t);
+            for (int i = 0; i < 8; ++i)
+                word += (uint32_t)exact_code(v[i], c1, s_t) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
         }
     }
-    // byte j = code[2j] << 4 | code[2j+1]; word = bytes 0..3
-    uint32_t b[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) b[j] = (uint32_t)(code[2 * j] * 16 + code[2 * j + 1]);
-    const uint32_t word = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     if (e0 + 8 <= n) {
         reinterpret_cast<uint32_t *>(packed)[g] = word;
     } else {
         for (int j = 0; 2 * j < (int)(n - e0); ++j) packed[(e0 >> 1) + j] = (uint8_t)(word >> (8 * j));
     }
 }
-
-constexpr int kUnroll = 1;
 
 template <bool kBf16>
 __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restrict__ w, int64_t n,
@@ -161,20 +173,13 @@ __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restri
 
     const int lane = threadIdx.x & 31;
     const int64_t ngroups = (n + 7) >> 3;
-    constexpr int64_t kSpan = (int64_t)kQuantThreads * kUnroll;  // groups per CTA iteration
+    const int64_t stride = (int64_t)gridDim.x * kQuantThreads;
     // the trip count depends only on blockIdx, so whole warps stay converged
-    for (int64_t base = (int64_t)blockIdx.x * kSpan; base < ngroups; base += (int64_t)gridDim.x * kSpan) {
-        float v[kUnroll][8];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t g = base + u * kQuantThreads + threadIdx.x;
-            load8<kBf16>(w, g << 3, n, v[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t g = base + u * kQuantThreads + threadIdx.x;
-            quantize_group<kBf16>(v[u], g, g << 3, n, lane, s_t, s_cell, packed, absmax);
-        }
+    for (int64_t base = (int64_t)blockIdx.x * kQuantThreads; base < ngroups; base += stride) {
+        const int64_t g = base + threadIdx.x;
+        float v[8];
+        load8<kBf16>(w, g << 3, n, v);
+        quantize_group<kBf16>(v, g, g << 3, n, lane, s_t, s_cell, packed, absmax);
     }
 }
 
@@ -184,7 +189,7 @@ cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed
                             cudaStream_t stream, int num_sms) {
     if (n == 0) return cudaSuccess;
     int64_t ngroups = (n + 7) / 8;
-    int64_t span = (int64_t)kQuantThreads * kUnroll;
+    int64_t span = (int64_t)kQuantThreads;
     int64_t want = (ngroups + span - 1) / span;
     int64_t cap = (int64_t)num_sms * 8;
     int grid = (int)(want < cap ? want : cap);
