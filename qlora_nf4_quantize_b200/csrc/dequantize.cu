@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kDeqThreads) k_dequantize(const uint8_t *__res
                                                              const float *__restrict__ offset, int64_t n,
                                                              void *__restrict__ out) {
     __shared__ float s_q[16];
+    pdl_wait_then_release();
     if (threadIdx.x < 16) s_q[threadIdx.x] = c_levels[threadIdx.x];
     __syncthreads();
     const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
@@ -88,9 +89,11 @@ __global__ void __launch_bounds__(kDeqThreads) k_dequantize(const uint8_t *__res
 template <int kMode>
 cudaError_t launch_mode(const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
                         int64_t n, void *out, bool bf16, int grid, cudaStream_t stream) {
-    if (bf16) k_dequantize<kMode, true><<<grid, kDeqThreads, 0, stream>>>(packed, q8, scales, offset, n, out);
-    else k_dequantize<kMode, false><<<grid, kDeqThreads, 0, stream>>>(packed, q8, scales, offset, n, out);
-    return cudaGetLastError();
+    if (bf16)
+        return launch_pdl(k_dequantize<kMode, true>, dim3(grid), dim3(kDeqThreads), 0, stream, 1, packed, q8, scales,
+                          offset, n, out);
+    return launch_pdl(k_dequantize<kMode, false>, dim3(grid), dim3(kDeqThreads), 0, stream, 1, packed, q8, scales,
+                      offset, n, out);
 }
 
 }  // namespace

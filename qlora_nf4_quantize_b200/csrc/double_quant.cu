@@ -44,6 +44,7 @@ __device__ __forceinline__ int biased_exp(float v) {
 __global__ void __launch_bounds__(1024) k_dq_chunk_sums(const float *__restrict__ c1, int64_t nb,
                                                          double *__restrict__ chunk_sums) {
     __shared__ double s_run[kRunsPerChunk];
+    pdl_wait_then_release();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
     const int64_t d = (int64_t)blockIdx.x * kRunsPerChunk + warp;
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c
                                                       float *__restrict__ offset) {
     extern __shared__ double s_tree[];  // 2 * nchunks doubles when centring
     __shared__ float s_mu;
+    pdl_wait_then_release();
     if (offset != nullptr) {
         for (int64_t j = threadIdx.x; j < nchunks; j += blockDim.x) s_tree[j] = chunk_sums[j];
         __syncthreads();
@@ -180,8 +182,8 @@ cudaError_t launch_double_quantize(const float *absmax, int64_t nb, uint8_t *cod
     const int64_t nchunks = dq_chunk_count(nb);
     size_t smem = 0;
     if (offset != nullptr) {
-        k_dq_chunk_sums<<<(unsigned)nchunks, 1024, 0, stream>>>(absmax, nb, chunk_sums);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(k_dq_chunk_sums, dim3((unsigned)nchunks), dim3(1024), 0, stream, 1, absmax, nb,
+                                   chunk_sums);
         if (e != cudaSuccess) return e;
         smem = (size_t)(2 * nchunks) * sizeof(double);
         if (smem > 48 * 1024) {
@@ -192,8 +194,8 @@ cudaError_t launch_double_quantize(const float *absmax, int64_t nb, uint8_t *cod
     int64_t want = (nd + 7) / 8;
     int64_t cap = (int64_t)num_sms * 4;
     int grid = (int)(want < cap ? want : cap);
-    k_dq_quantize<<<grid, 256, smem, stream>>>(absmax, nb, chunk_sums, nchunks, codes, absmax2, offset);
-    return cudaGetLastError();
+    return launch_pdl(k_dq_quantize, dim3(grid), dim3(256), smem, stream, 1, absmax, nb,
+                      static_cast<const double *>(chunk_sums), nchunks, codes, absmax2, offset);
 }
 
 }  // namespace nf4

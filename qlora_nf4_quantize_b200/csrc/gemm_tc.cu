@@ -189,6 +189,12 @@ __global__ void __launch_bounds__(C::Threads, 1)
     const int64_t m0 = (int64_t)blockIdx.y * kBT;
     const int kw_steps = (int)(K / kBK);
     const int kt_total = kw_steps + (r > 0 ? rp / kBK : 0);
+    // Programmatic dependent launch.  With an adapter the grid before this one
+    // is the down-projection, which releases it only after its own
+    // predecessor completed: x and W may be read at once, t only after the
+    // wait in the extension steps.  Without one, wait before reading anything.
+    if (r <= 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -358,7 +364,7 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUte
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode, C>, mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, y,
                               err);
 }
@@ -459,8 +465,9 @@ __global__ void __launch_bounds__(128, 1)
     DownSmem<kR> &S =
         *reinterpret_cast<DownSmem<kR> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int *abort = &S.abort;
-    // the fused linear launched next may start now; it waits for t itself
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // the fused linear launched next may start once every CTA is past this
+    // point; it reads x and W at once and waits for t itself
+    pdl_wait_then_release();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -611,20 +618,9 @@ cudaError_t launch_down_tc(const CUtensorMap &mx, const CUtensorMap &ma, int64_t
     cudaError_t e = cudaFuncSetAttribute(k_lora_down_tc<kR, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kSplit, (unsigned)((M + kDownRows - 1) / kDownRows));
-    cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kSplit;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_lora_down_tc<kR, kSplit>, mx, ma, M, K, s, static_cast<__nv_bfloat16 *>(t2),
-                              rp, err);
+    return launch_pdl(k_lora_down_tc<kR, kSplit>, dim3(kSplit, (unsigned)((M + kDownRows - 1) / kDownRows)),
+                      dim3(128), smem, stream, (unsigned)kSplit, mx, ma, M, K, s, static_cast<__nv_bfloat16 *>(t2), rp,
+                      err);
 }
 
 template <int kR>

@@ -93,6 +93,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32, NF4_GEMV_MINB) k_gemv(const _
                                                           const __nv_bfloat16 *__restrict__ t2, int rp,
                                                           __nv_bfloat16 *__restrict__ y) {
     constexpr bool kSmemLut = kLutSel != 0;
+    // programmatic dependent launch: see k_gemm_tc (x and W at once when the
+    // down-projection precedes; otherwise wait before reading anything)
+    if (r <= 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ float s_part[kGemvWarps][MT][NT][4][32];
     extern __shared__ float2 s_pairs[];  // kPairTableFloat2 entries when kSmemLut
     if constexpr (kSmemLut) {
@@ -341,6 +345,9 @@ __global__ void __launch_bounds__(kPWarps * 32, 1)
              const __nv_bfloat16 *__restrict__ Bl, int r, const __nv_bfloat16 *__restrict__ t2, int rp,
              __nv_bfloat16 *__restrict__ y, int depth, int my_tiles_max) {
     extern __shared__ __align__(16) uint8_t s_dyn[];
+    // programmatic dependent launch: see k_gemm_tc
+    if (r <= 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr bool kSmemLut = kLut != 0;
     const GemvPLayout L = gemv_p_layout(M, K, rp, NT, kSmemLut, depth, my_tiles_max);
     uint4 *xs = reinterpret_cast<uint4 *>(s_dyn + L.x_off);
@@ -598,7 +605,7 @@ cudaError_t launch_gemv_p(const void *x, int M, int64_t K, int64_t N, const uint
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = r > 0 ? 1 : 0;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k_gemv_p<kMode, NT, kLut>, static_cast<const __nv_bfloat16 *>(x), M, K, N,
                               packed, q8, scales, offset, static_cast<const __nv_bfloat16 *>(B), r,
                               static_cast<const __nv_bfloat16 *>(t2), rp, static_cast<__nv_bfloat16 *>(y), depth,
@@ -678,7 +685,7 @@ cudaError_t launch_gemv_mode(const void *x, int M, int64_t K, int64_t N, const u
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = r > 0 ? 1 : 0;  // overlap with the down-projection that precedes it
+    cfg.numAttrs = 1;
     cfg.dynamicSmemBytes = kGemvSmemLut ? kPairTableFloat2 * sizeof(float2) : 0;
     if (M <= 8)
         return cudaLaunchKernelEx(&cfg, k_gemv<kMode, 1, 1, kGemvLut>, xp, M, K, N, packed, q8, scales, offset, bp,

@@ -18,9 +18,9 @@
 // partial tiles in shared memory in warp order; then every CTA takes a slice
 // of the 16 x r outputs and sums the CTAs' partials in rank order through
 // distributed shared memory, so the result is independent of timing.  The
-// kernel triggers programmatic dependent launch at entry: the fused linear
-// that follows starts streaming the weight at once and waits for t only where
-// it reads it (griddepcontrol.wait).
+// kernel releases the fused linear that follows (programmatic dependent
+// launch) as soon as its own predecessor has completed: the linear starts
+// streaming the weight at once and waits for t only where it reads it.
 #include <cooperative_groups.h>
 
 #include "mma_util.cuh"
@@ -42,7 +42,10 @@ __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat
     extern __shared__ float s_dyn[];  // [kDownWarps][NT][4][32] warp partials, then [NT * 128] CTA partial
     auto s_part = reinterpret_cast<float (*)[NT][4][32]>(s_dyn);
     float *s_cta = s_dyn + kDownWarps * NT * 4 * 32;  // this CTA's partial tile, fragment order
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // the fused linear launched next may start once every CTA is past this
+    // point (it reads x and W before waiting for t, so this grid releases it
+    // only after its own predecessor has completed)
+    pdl_wait_then_release();
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -121,19 +124,8 @@ cudaError_t launch_down(cudaStream_t stream, const __nv_bfloat16 *x, const __nv_
         cudaError_t e = cudaFuncSetAttribute(k_lora_down<kR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.dynamicSmemBytes = smem;
-    cfg.gridDim = dim3(kDownCtas);
-    cfg.blockDim = dim3(kDownWarps * 32);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kDownCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_lora_down<kR>, x, A, M, K, s, t2, rp);
+    return launch_pdl(k_lora_down<kR>, dim3(kDownCtas), dim3(kDownWarps * 32), smem, stream, kDownCtas, x, A, M, K,
+                      s, t2, rp);
 }
 
 }  // namespace

@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restri
                                                              float *__restrict__ absmax) {
     __shared__ float s_t[16];
     __shared__ uint32_t s_cell[kCellTable];
+    pdl_wait_then_release();
     build_tables(s_t, s_cell);
 
     const int lane = threadIdx.x & 31;
@@ -193,9 +194,8 @@ cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed
     int64_t want = (ngroups + span - 1) / span;
     int64_t cap = (int64_t)num_sms * 8;
     int grid = (int)(want < cap ? want : cap);
-    if (bf16) k_quantize<true><<<grid, kQuantThreads, 0, stream>>>(w, n, packed, absmax);
-    else k_quantize<false><<<grid, kQuantThreads, 0, stream>>>(w, n, packed, absmax);
-    return cudaGetLastError();
+    if (bf16) return launch_pdl(k_quantize<true>, dim3(grid), dim3(kQuantThreads), 0, stream, 1, w, n, packed, absmax);
+    return launch_pdl(k_quantize<false>, dim3(grid), dim3(kQuantThreads), 0, stream, 1, w, n, packed, absmax);
 }
 
 }  // namespace nf4
