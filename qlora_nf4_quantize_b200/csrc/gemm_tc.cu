@@ -44,6 +44,9 @@ constexpr int kBK = 64;                    // k per pipeline step
 #ifndef NF4_GEMM_STAGES
 #define NF4_GEMM_STAGES 4
 #endif
+#ifndef NF4_GEMM_SUB
+#define NF4_GEMM_SUB 1
+#endif
 // Dequant warpgroups: warpgroup h produces the k-steps with index % WG == h.
 #ifndef NF4_GEMM_WG
 #define NF4_GEMM_WG 2
@@ -56,6 +59,10 @@ constexpr int kBK = 64;                    // k per pipeline step
 #define NF4_GEMM_LUT_MASK 0
 #endif
 constexpr int kLutMask = NF4_GEMM_LUT_MASK;
+// k-steps of packed codes each dequant thread keeps in flight
+#ifndef NF4_GEMM_PF
+#define NF4_GEMM_PF 1
+#endif
 
 constexpr uint32_t pow2_at_least(uint32_t v) {
     uint32_t p = 32;
@@ -68,14 +75,24 @@ constexpr uint32_t pow2_at_least(uint32_t v) {
 // when built with NF4_SMALL_M_TC=1 (one 128-row tile per CTA: 86 CTAs for an
 // 11008-row weight, and a k-step rate bound by the dequant warps' latency,
 // measured slower than the warp-MMA GEMV kernels, so not the default).
-template <int BT_, int STAGES_, int WG_>
+constexpr uint32_t AccColsFor(int bt) { return bt < 32 ? 32u : (uint32_t)bt; }
+
+template <int BT_, int STAGES_, int WG_, int SUB_>
 struct TileCfg {
     static constexpr int BT = BT_, Stages = STAGES_, WG = WG_;
+    // k-steps of 64 per pipeline stage: the stage's barriers, its TMA
+    // transaction and its MMA issue are shared by SUB k-steps
+    static constexpr int Sub = SUB_;
     static constexpr int Threads = 128 + 128 * WG;
-    static constexpr uint32_t AccCols = BT < 32 ? 32 : BT;   // accumulator: columns [0, AccCols)
-    static constexpr uint32_t ACol = AccCols;                // A stages: columns [ACol + 32 s, +32)
-    static constexpr uint32_t TmemCols = pow2_at_least(AccCols + 32 * Stages);
-    static constexpr uint32_t XStageBytes = BT * kBK * 2;
+    // two CTAs per SM when both fit (registers at 128 per thread, tensor
+    // memory at 256 columns each)
+    static constexpr int MinBlocks = (Threads <= 256 && AccColsFor(BT_) + 32 * SUB_ * STAGES_ <= 256) ? 2 : 1;
+    static constexpr uint32_t AccCols = AccColsFor(BT);     // accumulator: columns [0, AccCols)
+    // A of k-step j of stage s: columns [ACol + 32 (Sub s + j), +32)
+    static constexpr uint32_t ACol = AccCols;
+    static constexpr uint32_t TmemCols = pow2_at_least(AccCols + 32 * Sub * Stages);
+    static constexpr uint32_t XSubBytes = BT * kBK * 2;     // one 64-wide k-step of x
+    static constexpr uint32_t XStageBytes = Sub * XSubBytes;
     // UMMA instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both
     // K-major, N = BT, M = 128.
     static constexpr uint32_t Idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BT >> 3) << 17) |
@@ -84,22 +101,27 @@ struct TileCfg {
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M = 128");
 };
 
-using CfgLarge = TileCfg<256, NF4_GEMM_STAGES, NF4_GEMM_WG>;
+#ifndef NF4_GEMM_BT
+#define NF4_GEMM_BT 256
+#endif
+using CfgLarge = TileCfg<NF4_GEMM_BT, NF4_GEMM_STAGES, NF4_GEMM_WG, NF4_GEMM_SUB>;
 #ifndef NF4_GEMV_TC_WG
 #define NF4_GEMV_TC_WG 3
 #endif
 #ifndef NF4_GEMV_TC_STAGES
 #define NF4_GEMV_TC_STAGES 6
 #endif
-using CfgSmall = TileCfg<16, NF4_GEMV_TC_STAGES, NF4_GEMV_TC_WG>;
+using CfgSmall = TileCfg<16, NF4_GEMV_TC_STAGES, NF4_GEMV_TC_WG, 1>;
 
 template <class C>
 struct __align__(1024) SmemLayout {
     uint8_t x[C::Stages][C::XStageBytes];
-    uint64_t x_full[C::Stages];
-    uint64_t x_empty[C::Stages];
-    uint64_t a_full[C::Stages];
-    uint64_t a_empty[C::Stages];
+    // full[s]: the x tile has landed (one arrival with its transaction
+    // bytes) and the dequant warpgroup has stored the weight tile (128
+    // arrivals); empty[s]: the MMAs that read stage s have completed (one
+    // commit), awaited by the TMA producer and the dequant warpgroups alike
+    uint64_t full[C::Stages];
+    uint64_t empty[C::Stages];
     float2 pairs[kLutMask != 0 ? kPairTableFloat2 : 1];
     uint64_t acc_full;
     uint64_t drain;
@@ -148,7 +170,7 @@ template <int kMode>
 __device__ __forceinline__ void dequant_step(const StepCodes &sc, float mu, uint32_t out[32]) {
     const Lut lut = make_lut(block_scale_finish<kMode>(sc.sr, mu));
 #pragma unroll
-    for (int s = 0; s < 16; ++s) lut_lookup4(lut, sc.w[s >> 1] >> ((s & 1) * 16), out[2 * s], out[2 * s + 1]);
+    for (int i = 0; i < 8; ++i) lut_lookup8(lut, sc.w[i], out + 4 * i);
 }
 
 template <int kMode>
@@ -171,15 +193,16 @@ __device__ __forceinline__ void lora_step(const __nv_bfloat16 *__restrict__ Bl, 
 }
 
 template <int kMode, class C>
-__global__ void __launch_bounds__(C::Threads, 1)
+__global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_t,
               const __grid_constant__ CUtensorMap tmap_y, int64_t M,
               int64_t K, int64_t N, const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
               const float *__restrict__ scales, const float *__restrict__ offset,
               const __nv_bfloat16 *__restrict__ Bl, int r, int rp, __nv_bfloat16 *__restrict__ y, unsigned *err) {
     extern __shared__ uint8_t smem_raw[];
-    constexpr int kBT = C::BT, kStages = C::Stages, kWG = C::WG;
-    constexpr uint32_t kTmemCols = C::TmemCols, kAccCol = 0, kACol = C::ACol, kXStageBytes = C::XStageBytes;
+    constexpr int kBT = C::BT, kStages = C::Stages, kWG = C::WG, kSub = C::Sub;
+    constexpr uint32_t kTmemCols = C::TmemCols, kAccCol = 0, kACol = C::ACol, kXSubBytes = C::XSubBytes,
+                       kXStageBytes = C::XStageBytes;
     SmemLayout<C> &S =
         *reinterpret_cast<SmemLayout<C> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int *abort = &S.abort;
@@ -189,6 +212,7 @@ __global__ void __launch_bounds__(C::Threads, 1)
     const int64_t m0 = (int64_t)blockIdx.y * kBT;
     const int kw_steps = (int)(K / kBK);
     const int kt_total = kw_steps + (r > 0 ? rp / kBK : 0);
+    const int kg_total = (kt_total + kSub - 1) / kSub;  // pipeline stages (groups of kSub k-steps)
     // Programmatic dependent launch.  With an adapter the grid before this one
     // is the down-projection, which releases it only after its own
     // predecessor completed: x and W may be read at once, t only after the
@@ -198,10 +222,8 @@ __global__ void __launch_bounds__(C::Threads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&S.x_full[s], 1);
-            mbar_init(&S.x_empty[s], 1);
-            mbar_init(&S.a_full[s], 128);
-            mbar_init(&S.a_empty[s], 1);
+            mbar_init(&S.full[s], 1 + 128);
+            mbar_init(&S.empty[s], 1);
         }
         mbar_init(&S.acc_full, 1);
         mbar_init(&S.drain, 1);
@@ -225,48 +247,71 @@ __global__ void __launch_bounds__(C::Threads, 1)
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             int issued = 0;
-            for (int kt = 0; kt < kt_total; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+            for (int g = 0; g < kg_total; ++g) {
+                const int s = g % kStages;
+                const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+                const int kt0 = g * kSub;
+                const int nsub = kt_total - kt0 < kSub ? kt_total - kt0 : kSub;
                 // the t workspace is written by the down-projection kernel
                 // launched just before (programmatic dependent launch)
-                if (kt == kw_steps) asm volatile("griddepcontrol.wait;" ::: "memory");
-                if (!mbar_wait(&S.x_empty[s], ph ^ 1u, abort, err)) break;
-                mbar_arrive_expect_tx(&S.x_full[s], kXStageBytes);
-                if (kt < kw_steps) tma_load_2d(S.x[s], &tmap_x, &S.x_full[s], kt * kBK, (int)m0);
-                else tma_load_2d(S.x[s], &tmap_t, &S.x_full[s], (kt - kw_steps) * kBK, (int)m0);
-                issued = kt + 1;
+                if (kt0 <= kw_steps && kw_steps < kt0 + nsub) asm volatile("griddepcontrol.wait;" ::: "memory");
+                if (!mbar_wait(&S.empty[s], ph ^ 1u, abort, err)) break;
+                mbar_arrive_expect_tx(&S.full[s], (uint32_t)nsub * kXSubBytes);
+                for (int j = 0; j < nsub; ++j) {
+                    const int kt = kt0 + j;
+                    uint8_t *dst = S.x[s] + j * kXSubBytes;
+                    if (kt < kw_steps) tma_load_2d(dst, &tmap_x, &S.full[s], kt * kBK, (int)m0);
+                    else tma_load_2d(dst, &tmap_t, &S.full[s], (kt - kw_steps) * kBK, (int)m0);
+                }
+                issued = g + 1;
             }
             // drain: every issued load has landed before the CTA may exit
-            for (int kt = issued - kStages < 0 ? 0 : issued - kStages; kt < issued; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+            for (int g = issued - kStages < 0 ? 0 : issued - kStages; g < issued; ++g) {
+                const int s = g % kStages;
+                const uint32_t ph = (uint32_t)(g / kStages) & 1u;
                 unsigned long long t0 = global_ns();
-                while (!mbar_try_wait(&S.x_full[s], ph) && global_ns() - t0 < kWaitLimitNs) {
+                while (!mbar_try_wait(&S.full[s], ph) && global_ns() - t0 < kWaitLimitNs) {
                 }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            bool any = false;
-            for (int kt = 0; kt < kt_total; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
-                if (!mbar_wait(&S.x_full[s], ph, abort, err)) break;
-                if (!mbar_wait(&S.a_full[s], ph, abort, err)) break;
-                tc_fence_after();
-                const uint64_t bdesc = smem_desc_sw128(S.x[s]);
+            bool any = false, stop = false;
+            // Stage s: x tile at descriptor xdesc0 + (s * kXStageBytes) / 16
+            // (the start-address field counts 16-byte units and the sum is
+            // the stage's own address), weight k-step j at tensor-memory
+            // column kACol + 32 (kSub s + j).  Unrolled over the stages, so
+            // every offset is a constant and the issue loop stays short.
+            const uint64_t xdesc0 = smem_desc_sw128(S.x[0]);
+            for (int g0 = 0; !stop && g0 < kg_total; g0 += kStages) {
+                const uint32_t ph = (uint32_t)(g0 / kStages) & 1u;
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk) {
-                    tc_mma_ts(tmem + kAccCol, tmem + kACol + 32u * s + 8u * kk, bdesc + 2ull * kk, C::Idesc,
-                              (kt | kk) != 0 ? 1u : 0u);
+                for (int s = 0; s < kStages; ++s) {
+                    const int g = g0 + s;
+                    if (g >= kg_total) break;
+                    if (!mbar_wait(&S.full[s], ph, abort, err)) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int j = 0; j < kSub; ++j) {
+                        const int kt = g * kSub + j;
+                        if (kSub == 1 || kt < kt_total) {
+                            const uint64_t bdesc = xdesc0 + (uint64_t)((s * kXStageBytes + j * kXSubBytes) >> 4);
+                            const uint32_t acol = tmem + kACol + 32u * (uint32_t)(kSub * s + j);
+                            tc_mma_ts(tmem + kAccCol, acol, bdesc, C::Idesc, kt != 0 ? 1u : 0u);
+#pragma unroll
+                            for (int kk = 1; kk < kBK / 16; ++kk)
+                                tc_mma_ts(tmem + kAccCol, acol + 8u * kk, bdesc + 2ull * kk, C::Idesc, 1u);
+                        }
+                    }
+                    any = true;
+                    tc_commit(&S.empty[s]);
                 }
-                any = true;
-                tc_commit(&S.x_empty[s]);
-                tc_commit(&S.a_empty[s]);
-                if (kt == kt_total - 1) tc_commit(&S.acc_full);
             }
+            if (any && !stop) tc_commit(&S.acc_full);
             if (any && *abort) {  // drain our own MMAs before tensor memory is released
                 tc_commit(&S.drain);
                 unsigned long long t0 = global_ns();
@@ -284,29 +329,56 @@ __global__ void __launch_bounds__(C::Threads, 1)
         const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         bool ok = true;
-        // software pipeline: the codes of this warpgroup's next k-step are in
-        // flight while the current one is converted
-        StepCodes cur, nxt;
-        if (h < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, h, nvalid, cur);
-        for (int kt = h; kt < kt_total; kt += kWG) {
-            const int s = kt % kStages;
-            const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
-            uint32_t v[32];
-            if (kt < kw_steps) {
-                if (kt + kWG < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, kt + kWG, nvalid, nxt);
-                if ((kLutMask >> h) & 1) dequant_step_smem<kMode>(cur, mu, S.pairs + (lane & 15), v);
-                else dequant_step<kMode>(cur, mu, v);
-                cur = nxt;
-            } else {
-                lora_step(Bl, r, n, nvalid, kt - kw_steps, v);
+        // software pipeline: the codes of this warpgroup's next kPF stages
+        // (kSub k-steps each) are in flight while the current one is
+        // converted.  The register sets form a ring of kPF + 1 stages,
+        // indexed at compile time by unrolling kPF + 1 stages, so no set is
+        // copied (a copy would wait for its load).
+        constexpr int kPF = NF4_GEMM_PF;
+        StepCodes ring[kPF + 1][kSub];
+        auto load_group = [&](int g, StepCodes(&set)[kSub]) {
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) {
+                const int kt = g * kSub + j;
+                if (kt < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, kt, nvalid, set[j]);
             }
-            // warp-uniform outcome: the tcgen05.st below is a warp-wide instruction
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.a_empty[s], ph ^ 1u, abort, err));
-            if (!ok) break;
-            tc_store32(lane_base + kACol + 32u * s, v);
-            tc_wait_st();
-            tc_fence_before();
-            mbar_arrive(&S.a_full[s]);
+        };
+#pragma unroll
+        for (int i = 0; i < kPF; ++i) {
+            const int g = h + i * kWG;
+            if (g < kg_total) load_group(g, ring[i]);
+        }
+        for (int g0 = h; ok && g0 < kg_total; g0 += (kPF + 1) * kWG) {
+#pragma unroll
+            for (int i = 0; i <= kPF; ++i) {
+                const int g = g0 + i * kWG;
+                if (g >= kg_total) break;
+                const int s = g % kStages;
+                const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+                if (g + kPF * kWG < kg_total) load_group(g + kPF * kWG, ring[(i + kPF) % (kPF + 1)]);
+#pragma unroll
+                for (int j = 0; j < kSub; ++j) {
+                    const int kt = g * kSub + j;
+                    if (kt >= kt_total) break;
+                    uint32_t v[32];
+                    if (kt < kw_steps) {
+                        if ((kLutMask >> h) & 1) dequant_step_smem<kMode>(ring[i][j], mu, S.pairs + (lane & 15), v);
+                        else dequant_step<kMode>(ring[i][j], mu, v);
+                    } else {
+                        lora_step(Bl, r, n, nvalid, kt - kw_steps, v);
+                    }
+                    if (j == 0) {
+                        // warp-uniform outcome: the tcgen05.st below is a warp-wide instruction
+                        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.empty[s], ph ^ 1u, abort, err));
+                        if (!ok) break;
+                    }
+                    tc_store32(lane_base + kACol + 32u * (uint32_t)(kSub * s + j), v);
+                    tc_wait_st();
+                }
+                if (!ok) break;
+                tc_fence_before();
+                mbar_arrive(&S.full[s]);
+            }
         }
         if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err));
         if (ok) {

@@ -27,9 +27,21 @@ struct Lut {
 };
 
 __device__ __forceinline__ Lut make_lut(float c) {
+    // P[j] = (RNE_bf16(RN(q[2j] c)), RNE_bf16(RN(q[2j+1] c))): the two
+    // products are one packed f32x2 multiply (each half rounded to nearest,
+    // as two binary32 multiplies)
+    uint64_t cc;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
     uint32_t P[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) P[j] = pack_bf16x2(__fmul_rn(c_levels[2 * j], c), __fmul_rn(c_levels[2 * j + 1], c));
+    for (int j = 0; j < 8; ++j) {
+        uint64_t qq, d;
+        asm("mov.b64 %0, {%1, %2};" : "=l"(qq) : "f"(c_levels[2 * j]), "f"(c_levels[2 * j + 1]));
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(qq), "l"(cc));
+        float lo, hi;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+        P[j] = pack_bf16x2(lo, hi);
+    }
     Lut t;
     t.L0 = __byte_perm(P[0], P[1], 0x6420); t.H0 = __byte_perm(P[0], P[1], 0x7531);
     t.L1 = __byte_perm(P[2], P[3], 0x6420); t.H1 = __byte_perm(P[2], P[3], 0x7531);
