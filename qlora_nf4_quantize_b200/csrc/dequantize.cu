@@ -12,9 +12,9 @@
 // warp's load is 128 contiguous bytes) and 16 output bytes for bf16 (one
 // 128-bit store; the warp's store is 512 contiguous bytes).  All kSeg loads of
 // a lane (codes and block constants) are issued before any arithmetic; up to
-// 8 CTAs of 256 threads per SM.  Eight segments per iteration (a 4096 x 4096
-// weight read in one round trip per warp) measured slower than four: 9.8
-// against 9.6 us to bf16, 24.0 against 21.3 us to fp32.
+// 8 CTAs of 256 threads per SM are resident, and the grid may hold more (see
+// launch_mode for the shape).  Eight segments per iteration (a 4096 x 4096
+// weight read in one round trip per warp) measured slower than four.
 // Codes are looked up in a 16-entry shared-memory copy of the table (16
 // distinct words in 16 banks: conflict-free for any code pattern).
 #include "nf4_device.cuh"
@@ -23,12 +23,6 @@ namespace nf4 {
 namespace {
 
 constexpr int kDeqThreads = 256;
-#ifndef NF4_DEQ_SEG
-#define NF4_DEQ_SEG 4
-#endif
-constexpr int kSeg = NF4_DEQ_SEG;        // segments per lane per iteration
-constexpr int kWarpElems = kSeg * 256;   // elements per warp per iteration
-static_assert(16384 % kWarpElems == 0, "a warp iteration stays in one group of 256 blocks");
 
 template <int kMode, bool kBf16Out>
 __device__ __forceinline__ void store8(void *out, int64_t e0, const float v[8]) {
@@ -46,12 +40,14 @@ __device__ __forceinline__ void store8(void *out, int64_t e0, const float v[8]) 
     }
 }
 
-template <int kMode, bool kBf16Out>
-__global__ void __launch_bounds__(kDeqThreads, 8) k_dequantize(const uint8_t *__restrict__ packed,
+template <int kMode, bool kBf16Out, int kSeg>
+__global__ void __launch_bounds__(kDeqThreads, 2048 / kDeqThreads) k_dequantize(const uint8_t *__restrict__ packed,
                                                              const uint8_t *__restrict__ q8,
                                                              const float *__restrict__ scales,
                                                              const float *__restrict__ offset, int64_t n,
                                                              void *__restrict__ out) {
+    constexpr int kWarpElems = kSeg * 256;  // elements per warp per iteration
+    static_assert(16384 % kWarpElems == 0, "a warp iteration stays in one group of 256 blocks");
     __shared__ float s_q[16];
     pdl_wait_then_release();
     if (threadIdx.x < 16) s_q[threadIdx.x] = c_levels[threadIdx.x];
@@ -105,14 +101,32 @@ __global__ void __launch_bounds__(kDeqThreads, 8) k_dequantize(const uint8_t *__
     }
 }
 
+template <int kMode, int kSeg>
+cudaError_t launch_seg(const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset, int64_t n,
+                       void *out, bool bf16, int ctas_per_sm, int num_sms, cudaStream_t stream) {
+    const int64_t witers = (n + kSeg * 256 - 1) / (kSeg * 256);
+    const int64_t want = (witers + (kDeqThreads / 32) - 1) / (kDeqThreads / 32);
+    const int64_t cap = (int64_t)num_sms * ctas_per_sm;
+    const int grid = (int)(want < cap ? want : cap);
+    if (bf16)
+        return launch_pdl(k_dequantize<kMode, true, kSeg>, dim3(grid), dim3(kDeqThreads), 0, stream, 1, packed, q8,
+                          scales, offset, n, out);
+    return launch_pdl(k_dequantize<kMode, false, kSeg>, dim3(grid), dim3(kDeqThreads), 0, stream, 1, packed, q8,
+                      scales, offset, n, out);
+}
+
+// Launch shape, measured on B200 (4096 x 4096 and 14336 x 4096 weights): a
+// bf16 output of up to 2^25 elements runs 2 segments per lane and iteration
+// with the grid capped at 16 CTAs per SM (about 1.7 iterations per warp, so
+// CTAs that finish early are followed by the rest); larger outputs and fp32
+// runs 4 segments with the grid capped at 32 CTAs per SM.  Both shapes beat
+// 4 segments at 8 CTAs per SM (a single resident wave) by 5-11 %.
 template <int kMode>
 cudaError_t launch_mode(const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
-                        int64_t n, void *out, bool bf16, int grid, cudaStream_t stream) {
-    if (bf16)
-        return launch_pdl(k_dequantize<kMode, true>, dim3(grid), dim3(kDeqThreads), 0, stream, 1, packed, q8, scales,
-                          offset, n, out);
-    return launch_pdl(k_dequantize<kMode, false>, dim3(grid), dim3(kDeqThreads), 0, stream, 1, packed, q8, scales,
-                      offset, n, out);
+                        int64_t n, void *out, bool bf16, int num_sms, cudaStream_t stream) {
+    if (bf16 && n <= (int64_t(1) << 25))
+        return launch_seg<kMode, 2>(packed, q8, scales, offset, n, out, bf16, 16, num_sms, stream);
+    return launch_seg<kMode, 4>(packed, q8, scales, offset, n, out, bf16, 32, num_sms, stream);
 }
 
 }  // namespace
@@ -120,13 +134,9 @@ cudaError_t launch_mode(const uint8_t *packed, const uint8_t *q8, const float *s
 cudaError_t launch_dequantize(const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
                               int64_t n, void *out, bool bf16, cudaStream_t stream, int num_sms) {
     if (n == 0) return cudaSuccess;
-    int64_t witers = (n + kWarpElems - 1) / kWarpElems;
-    int64_t want = (witers + (kDeqThreads / 32) - 1) / (kDeqThreads / 32);
-    int64_t cap = (int64_t)num_sms * 8;
-    int grid = (int)(want < cap ? want : cap);
-    if (q8 == nullptr) return launch_mode<2>(packed, q8, scales, offset, n, out, bf16, grid, stream);
-    if (offset == nullptr) return launch_mode<1>(packed, q8, scales, offset, n, out, bf16, grid, stream);
-    return launch_mode<0>(packed, q8, scales, offset, n, out, bf16, grid, stream);
+    if (q8 == nullptr) return launch_mode<2>(packed, q8, scales, offset, n, out, bf16, num_sms, stream);
+    if (offset == nullptr) return launch_mode<1>(packed, q8, scales, offset, n, out, bf16, num_sms, stream);
+    return launch_mode<0>(packed, q8, scales, offset, n, out, bf16, num_sms, stream);
 }
 
 }  // namespace nf4

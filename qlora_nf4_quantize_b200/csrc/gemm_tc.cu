@@ -42,14 +42,14 @@ namespace {
 constexpr int kBN = 128;                   // weight rows per CTA (MMA M)
 constexpr int kBK = 64;                    // k per pipeline step
 #ifndef NF4_GEMM_STAGES
-#define NF4_GEMM_STAGES 4
+#define NF4_GEMM_STAGES 6
 #endif
 #ifndef NF4_GEMM_SUB
 #define NF4_GEMM_SUB 1
 #endif
 // Dequant warpgroups: warpgroup h produces the k-steps with index % WG == h.
 #ifndef NF4_GEMM_WG
-#define NF4_GEMM_WG 2
+#define NF4_GEMM_WG 3
 #endif
 // Dequantization lookup per warpgroup: bit h set = warpgroup h uses the
 // shared-memory pair table (one shared load per two weights), clear = the
