@@ -28,11 +28,13 @@
 // (u scaled by s, as a bf16 hi/lo pair, from the down-projection kernel run
 // on g with B^T) and W~' = rows of [A ; A ; 0] (A's own rows, no transpose).
 //
-// Warp roles (12 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
-// MMA issuer (one elected thread), warps 4..11 = two dequant warpgroups
-// (warpgroup h produces the k-steps with index % 2 == h) and, at the end, the
-// epilogue (warpgroup h stores accumulator h: tcgen05.ld, bf16, 64-byte row
-// segments).  Every mbarrier wait is bounded as in the forward GEMM.
+// Warp roles (16 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
+// MMA issuer (one elected thread), warps 4..15 = three dequant warpgroups
+// (warpgroup h produces the k-steps with index % 3 == h) and, at the end, the
+// epilogue (16 units of one accumulator and 32 columns spread over the
+// warpgroups: tcgen05.ld, bf16, 64-byte row segments).  One full and one
+// empty barrier per stage; every mbarrier wait is bounded as in the forward
+// GEMM.
 #include "mma_util.cuh"
 #include "tc_util.cuh"
 
@@ -43,7 +45,12 @@ constexpr int kGM = 256;       // tokens per CTA (two accumulators of 128)
 constexpr int kGN = 256;       // output columns k per CTA (MMA N)
 constexpr int kGK = 64;        // contraction (n) per pipeline step
 constexpr int kGStages = 3;
-constexpr int kGThreads = 128 + 256;
+// dequant warpgroups: warpgroup h produces the k-steps with index % kGWG == h
+#ifndef NF4_BWD_WG
+#define NF4_BWD_WG 3
+#endif
+constexpr int kGWG = NF4_BWD_WG;
+constexpr int kGThreads = 128 + 128 * kGWG;
 constexpr uint32_t kGTmemCols = 512;
 constexpr uint32_t kGStageBytes = kGM * kGK * 2;  // also the WT tile: kGN x kGK bf16
 static_assert(kGM * kGK == kGN * kGK, "G and WT tiles have the same size");
@@ -71,10 +78,12 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128_b(const void *p, uint32_t
 struct __align__(1024) BwdSmem {
     uint8_t g[kGStages][kGStageBytes];
     uint8_t wt[kGStages][kGStageBytes];
-    uint64_t g_full[kGStages];
-    uint64_t g_empty[kGStages];
-    uint64_t w_full[kGStages];
-    uint64_t w_empty[kGStages];
+    // full[s]: the g tile has landed (one arrival with its transaction bytes)
+    // and the producing warpgroup has written the weight tile (one arrival
+    // per warp); empty[s]: the MMAs that read stage s have completed (one
+    // commit), awaited by the TMA producer and the dequant warpgroups alike
+    uint64_t full[kGStages];
+    uint64_t empty[kGStages];
     uint64_t acc_full;
     uint64_t drain;
     uint32_t tmem_base;
@@ -134,10 +143,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGStages; ++s) {
-            mbar_init(&S.g_full[s], 1);
-            mbar_init(&S.g_empty[s], 1);
-            mbar_init(&S.w_full[s], 4);  // one arrival per warp of the producing warpgroup
-            mbar_init(&S.w_empty[s], 1);
+            mbar_init(&S.full[s], 1 + 4);
+            mbar_init(&S.empty[s], 1);
         }
         mbar_init(&S.acc_full, 1);
         mbar_init(&S.drain, 1);
@@ -166,15 +173,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 // u is written by the down-projection kernel launched just
                 // before (programmatic dependent launch)
                 if (kt == kn_steps) asm volatile("griddepcontrol.wait;" ::: "memory");
-                if (!mbar_wait(&S.g_empty[s], ph ^ 1u, abort, err)) break;
-                mbar_arrive_expect_tx(&S.g_full[s], kGStageBytes);
-                if (kt < kn_steps) tma_load_2d(S.g[s], &tmap_g, &S.g_full[s], kt * kGK, (int)m0);
-                else tma_load_2d(S.g[s], &tmap_u, &S.g_full[s], (kt - kn_steps) * kGK, (int)m0);
+                if (!mbar_wait(&S.empty[s], ph ^ 1u, abort, err)) break;
+                mbar_arrive_expect_tx(&S.full[s], kGStageBytes);
+                if (kt < kn_steps) tma_load_2d(S.g[s], &tmap_g, &S.full[s], kt * kGK, (int)m0);
+                else tma_load_2d(S.g[s], &tmap_u, &S.full[s], (kt - kn_steps) * kGK, (int)m0);
                 issued = kt + 1;
             }
             for (int kt = issued - kGStages < 0 ? 0 : issued - kGStages; kt < issued; ++kt) {
                 unsigned long long t0 = global_ns();
-                while (!mbar_try_wait(&S.g_full[kt % kGStages], (uint32_t)(kt / kGStages) & 1u) &&
+                while (!mbar_try_wait(&S.full[kt % kGStages], (uint32_t)(kt / kGStages) & 1u) &&
                        global_ns() - t0 < kWaitLimitNs) {
                 }
             }
@@ -186,8 +193,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             for (int kt = 0; kt < kt_total; ++kt) {
                 const int s = kt % kGStages;
                 const uint32_t ph = (uint32_t)(kt / kGStages) & 1u;
-                if (!mbar_wait(&S.g_full[s], ph, abort, err)) break;
-                if (!mbar_wait(&S.w_full[s], ph, abort, err)) break;
+                if (!mbar_wait(&S.full[s], ph, abort, err)) break;
                 tc_fence_after();
                 const uint64_t a0 = smem_desc_sw128(S.g[s]);
                 const uint64_t a1 = smem_desc_sw128(S.g[s] + kGStageBytes / 2);  // tokens 128..255
@@ -200,8 +206,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     tc_mma_ss(tmem + 256u, a1 + 2ull * kk, b, kGIdesc, acc);
                 }
                 any = true;
-                tc_commit(&S.g_empty[s]);
-                tc_commit(&S.w_empty[s]);
+                tc_commit(&S.empty[s]);
                 if (kt == kt_total - 1) tc_commit(&S.acc_full);
             }
             if (any && *abort) {  // drain our own MMAs before tensor memory is released
@@ -214,7 +219,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     } else if (warp >= 4) {
         // ---------------- dequant warpgroups (transposed tiles), then epilogue ----------------
         const int q = warp & 3;         // k-block of the tile / tensor-memory lane quarter
-        const int h = (warp - 4) >> 2;  // warpgroup: k-steps with index % 2 == h
+        const int h = (warp - 4) >> 2;  // warpgroup: k-steps with index % kGWG == h
         const int p = lane;             // n-pair: rows 2p, 2p + 1 of the step
         const int64_t kb = (k0 >> 6) + q;  // this lane's k-block of W
         const bool kvalid = kb * 64 < K;
@@ -227,39 +232,42 @@ __global__ void __launch_bounds__(kGThreads, 1)
             load_block<kMode>(packed, q8, scales, n + 1, K, kb, kvalid && n + 1 < N, x1);
         };
         if (h < kn_steps) load_pair(h, ca, cb);
-        for (int kt = h; kt < kt_total; kt += 2) {
+        for (int kt = h; kt < kt_total; kt += kGWG) {
             const int s = kt % kGStages;
             const uint32_t ph = (uint32_t)(kt / kGStages) & 1u;
             const uint32_t tile = smem_addr(S.wt[s]);
             if (kt < kn_steps) {
-                if (kt + 2 < kn_steps) load_pair(kt + 2, na, nb);
-                uint32_t va[32], vb[32];
+                if (kt + kGWG < kn_steps) load_pair(kt + kGWG, na, nb);
+                // word j of a row holds k = 2j (low half) and 2j + 1 (high half):
+                // chunk c = words 4c .. 4c + 3; row 2p is dequantized before the
+                // wait for the stage and stored after it, then row 2p + 1
+                uint32_t v[32];
                 {
                     const Lut la = make_lut(block_scale_finish<kMode>(ca.sr, mu));
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) lut_lookup8(la, ca.w[i], v + 4 * i);
+                }
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.empty[s], ph ^ 1u, abort, err));
+                if (!ok) break;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    sts128(tile + w_offset(2 * p, q, c), make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
+                {
                     const Lut lb = make_lut(block_scale_finish<kMode>(cb.sr, mu));
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        lut_lookup8(la, ca.w[i], va + 4 * i);
-                        lut_lookup8(lb, cb.w[i], vb + 4 * i);
-                    }
+                    for (int i = 0; i < 8; ++i) lut_lookup8(lb, cb.w[i], v + 4 * i);
                 }
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.w_empty[s], ph ^ 1u, abort, err));
-                if (!ok) break;
-                // word j of a row holds k = 2j (low half) and 2j + 1 (high half):
-                // chunk c = words 4c .. 4c + 3, rows 2p and 2p + 1 of the step
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    sts128(tile + w_offset(2 * p, q, c), make_uint4(va[4 * c], va[4 * c + 1], va[4 * c + 2], va[4 * c + 3]));
+                for (int c = 0; c < 8; ++c)
                     sts128(tile + w_offset(2 * p + 1, q, c),
-                           make_uint4(vb[4 * c], vb[4 * c + 1], vb[4 * c + 2], vb[4 * c + 3]));
-                }
+                           make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
                 ca = na;
                 cb = nb;
             } else {
                 // rows j of [A ; A ; 0] (row j -> A[j mod r] for j < 2r), columns
                 // k0 + 64 q .. + 63: rows 2p and 2p + 1 of the step
                 const int e = kt - kn_steps;
-                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.w_empty[s], ph ^ 1u, abort, err));
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.empty[s], ph ^ 1u, abort, err));
                 if (!ok) break;
                 const int64_t k = k0 + 64 * q;
 #pragma unroll
@@ -275,16 +283,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
             // the tile is read by the tensor cores (async proxy)
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S.w_full[s]);
+            if (lane == 0) mbar_arrive(&S.full[s]);
         }
         if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err));
         if (ok) {
-            // Epilogue: warpgroup h stores accumulator h; thread = token row.
+            // Epilogue: 16 units (accumulator a of 128 tokens, 32-column chunk
+            // c), unit a * 8 + c stored by warpgroup (a * 8 + c) % kGWG;
+            // thread = token row.
             tc_fence_after();
-            const int64_t m = m0 + 128 * h + 32 * q + lane;
-            const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + 256u * (uint32_t)h;
 #pragma unroll 1
-            for (int c = 0; c < kGN / 32; ++c) {
+            for (int u = h; u < 2 * (kGN / 32); u += kGWG) {
+                const int a = u / (kGN / 32), c = u % (kGN / 32);
+                const int64_t m = m0 + 128 * a + 32 * q + lane;
+                const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + 256u * (uint32_t)a;
                 uint32_t v[32];
                 tc_load32(base + 32u * c, v);
                 tc_wait_ld();
