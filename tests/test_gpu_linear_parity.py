@@ -93,7 +93,9 @@ def test_gemv_without_lora_equals_matmul_on_dequantized(nf4lib, cuda_device):
 
 # ---------------------------------------------------------------- tensor-core GEMM (M > 16)
 @pytest.mark.parametrize("M,K,N,r,dq", [(17, 64, 8, 0, True), (100, 192, 136, 16, True), (256, 256, 128, 64, True),
-                                        (300, 320, 264, 32, False), (513, 128, 256, 16, True)])
+                                        (300, 320, 264, 32, False), (513, 128, 256, 16, True),
+                                        # 13 and 7 pipeline steps: the stage ring wraps, ragged last round
+                                        (70, 768, 72, 32, True), (140, 448, 264, 0, False)])
 def test_gemm_small_shapes_full_output(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
     c = wl.LinearCase("gemm small", M, K, N, r, 0.75, 57 + M + K + N)
     W, x, A, B = wl.linear_inputs(c, with_lora=r > 0)
@@ -122,6 +124,20 @@ def test_gemm_full_size_sampled_rows(nf4lib, oracle_mod, cuda_device, case, nrow
     nf4lib.nf4_device_status()
     rows = sampled_rows(case.M, nrows, case.seed)
     ref = oracle_linear(oracle_mod, st, x, A, B, case.r, case.scaling, rows=rows)
+    check(y[torch.from_numpy(rows).to(cuda_device)], ref)
+
+
+def test_gemm_partial_last_wave(nf4lib, oracle_mod, cuda_device):
+    """150 tiles of 128 x 256 on 148 SMs (a second, nearly empty wave); the
+    sampled rows include the last 8 tokens, which meet the last tiles."""
+    c = wl.LinearCase("gemm partial wave", 512, 1024, 9600, 16, 0.5, 4242)
+    W, x, A, B = wl.linear_inputs(c)
+    st = quantize_on_gpu(nf4lib, W, cuda_device)
+    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, c.N,
+                                   A.to(cuda_device), B.to(cuda_device), c.scaling)
+    nf4lib.nf4_device_status()
+    rows = np.unique(np.concatenate([sampled_rows(c.M, 8, c.seed), np.arange(c.M - 8, c.M)])).astype(np.int64)
+    ref = oracle_linear(oracle_mod, st, x, A, B, c.r, c.scaling, rows=rows)
     check(y[torch.from_numpy(rows).to(cuda_device)], ref)
 
 
