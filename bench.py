@@ -446,216 +446,227 @@ def run_suite(args):
         line.update(extra)
         print(json.dumps(line), flush=True)
 
+    sections = set(args.sections.split(",")) if args.sections else None
+
+    def want(name):
+        return sections is None or name in sections
+
     rot = [0]
 
     def nxt(c):
         rot[0] += 1
         return rot[0] % c
 
-    # ---- projection 4096x4096 bf16: quantize, double-quantize, dequantize (with / without DQ)
-    wp = wl.weight_case(wl.PROJECTION).to(dev).reshape(-1)
-    n, C = wp.numel(), 6
-    nb = n // BLOCK
-    Ws = [wp.clone() for _ in range(C)]
-    sts = [q.quantize_weight(w) for w in Ws]
-    raw = [q.nf4_quantize(w) for w in Ws[:C]]  # (packed, fp32 absmax): the no-DQ state
-    absb = [torch.empty(nb, device=dev) for _ in range(C)]
-    outs = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(C)]
-    outs32 = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(C)]
-    q8s = [torch.empty(nb, dtype=torch.uint8, device=dev) for _ in range(C)]
-    c2s = [torch.empty(-(-nb // DQ_BLOCK), device=dev) for _ in range(C)]
-    offs = [torch.empty(1, device=dev) for _ in range(C)]
-    ws = torch.empty(q.nf4_double_quantize_workspace_size(nb), dtype=torch.uint8, device=dev)
+    if want("projection"):
+        # ---- projection 4096x4096 bf16: quantize, double-quantize, dequantize (with / without DQ)
+        wp = wl.weight_case(wl.PROJECTION).to(dev).reshape(-1)
+        n, C = wp.numel(), 6
+        nb = n // BLOCK
+        Ws = [wp.clone() for _ in range(C)]
+        sts = [q.quantize_weight(w) for w in Ws]
+        raw = [q.nf4_quantize(w) for w in Ws[:C]]  # (packed, fp32 absmax): the no-DQ state
+        absb = [torch.empty(nb, device=dev) for _ in range(C)]
+        outs = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(C)]
+        outs32 = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(C)]
+        q8s = [torch.empty(nb, dtype=torch.uint8, device=dev) for _ in range(C)]
+        c2s = [torch.empty(-(-nb // DQ_BLOCK), device=dev) for _ in range(C)]
+        offs = [torch.empty(1, device=dev) for _ in range(C)]
+        ws = torch.empty(q.nf4_double_quantize_workspace_size(nb), dtype=torch.uint8, device=dev)
 
-    def f_quant():
-        k = nxt(C)
-        q.nf4_quantize(Ws[k], packed=sts[k].packed, absmax=absb[k])
-
-    def f_dq():
-        k = nxt(C)
-        q.nf4_double_quantize(absb[k], absmax_q=q8s[k], absmax2=c2s[k], offset=offs[k], workspace=ws)
-
-    def f_deq(dq, f32):
-        def f():
+        def f_quant():
             k = nxt(C)
-            o = outs32[k] if f32 else outs[k]
-            if dq:
-                st = sts[k]
-                q.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, n,
-                                 torch.float32 if f32 else torch.bfloat16, out=o)
-            else:
-                q.nf4_dequantize(raw[k][0], None, raw[k][1], None, n, torch.float32 if f32 else torch.bfloat16,
-                                 out=o)
-        return f
+            q.nf4_quantize(Ws[k], packed=sts[k].packed, absmax=absb[k])
 
-    proj = "projection 4096x4096 bf16"
-    emit(f"quantize {proj}", graph_us(f_quant, 20), quantize_bytes(n), "GB/s")
-    emit(f"double_quantize {nb} constants", graph_us(f_dq, 20), dq_bytes(nb), "GB/s")
-    emit(f"dequantize {proj} -> bf16, DQ", graph_us(f_deq(True, False), 20), dequant_bytes(n), "GB/s")
-    emit(f"dequantize {proj} -> fp32, DQ", graph_us(f_deq(True, True), 20), dequant_bytes(n, 4), "GB/s")
-    nodq_b = n // 2 + nb * 4 + n * 2
-    emit(f"dequantize {proj} -> bf16, no DQ (fp32 c1)", graph_us(f_deq(False, False), 20), nodq_b, "GB/s",
-         bytes_per_param=round(nodq_b / n - 2, 6))
-    del Ws, sts, raw, absb, outs, outs32, q8s, c2s, offs
-    torch.cuda.empty_cache()
+        def f_dq():
+            k = nxt(C)
+            q.nf4_double_quantize(absb[k], absmax_q=q8s[k], absmax2=c2s[k], offset=offs[k], workspace=ws)
 
-    # ---- fused linear: decode GEMV and tensor-core GEMM, with / without DQ
-    def linear_case(c, dq, copies, reps):
-        W, x, A, B = wl.linear_inputs(c)
-        Wd = W.to(dev)
-        stl = [q.quantize_weight(Wd, double_quant=dq) for _ in range(copies)]
-        del W, Wd
-        xd, Ad, Bd = x.to(dev), A.to(dev), B.to(dev)
-        y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
-        wsl = torch.empty(max(1, q.nf4_lora_linear_workspace_size(c.M, c.r)), dtype=torch.uint8, device=dev)
+        def f_deq(dq, f32):
+            def f():
+                k = nxt(C)
+                o = outs32[k] if f32 else outs[k]
+                if dq:
+                    st = sts[k]
+                    q.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, n,
+                                     torch.float32 if f32 else torch.bfloat16, out=o)
+                else:
+                    q.nf4_dequantize(raw[k][0], None, raw[k][1], None, n, torch.float32 if f32 else torch.bfloat16,
+                                     out=o)
+            return f
 
-        def f():
-            st = stl[nxt(copies)]
-            q.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, Ad, Bd, c.scaling,
-                                  y=y, workspace=wsl)
-        us = graph_us(f, reps)
-        q.nf4_device_status()
-        wb = c.N * c.K // 2 + (c.N * c.K // BLOCK) * (1 if dq else 4) + (-(-(c.N * c.K // BLOCK) // DQ_BLOCK) * 4 + 4
-                                                                          if dq else 0)
-        byts = wb + c.M * c.K * 2 + c.r * c.K * 2 + c.N * c.r * 2 + c.M * c.N * 2
-        return us, byts
-
-    for c in wl.GEMV_CASES:
-        for dq in (True, False):
-            us, byts = linear_case(c, dq, 8, 20)
-            emit(f"{c.name}{'' if dq else ', no DQ'}", us, byts, "GB/s",
-                 tflops=round(linear_flops(c.M, c.K, c.N, c.r) / (us * 1e-6) / 1e12, 3))
-    for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
-        for dq in (True, False):
-            us, _ = linear_case(c, dq, 1, 5)
-            emit(f"{c.name}{'' if dq else ', no DQ'}", us, linear_flops(c.M, c.K, c.N, c.r), "TFLOP/s",
-                 peak_sustained=peaks["bf16_tflops_sustained"])
-    torch.cuda.empty_cache()
-
-    # ---- backward through the frozen base: dx (fused NF4 GEMM) and the adapter gradients
-    for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
-        W, x, A, B = wl.linear_inputs(c)
-        g = torch.Generator().manual_seed(c.seed + 7)
-        dy = torch.randn(c.M, c.N, generator=g).to(torch.bfloat16).to(dev)
-        st = q.quantize_weight(W.to(dev))
-        xd, Ad, Bd = x.to(dev), A.to(dev), B.to(dev)
-        dxb = torch.empty(c.M, c.K, dtype=torch.bfloat16, device=dev)
-        dAb = torch.empty(c.r, c.K, device=dev)
-        dBb = torch.empty(c.N, c.r, device=dev)
-        wsb = torch.empty(q.nf4_lora_linear_bwd_workspace_size(c.M, c.N, c.K, c.r), dtype=torch.uint8, device=dev)
-
-        def f_dx():
-            q.nf4_lora_linear_bwd(dy, None, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
-                                  want=("dx",), dx=dxb, workspace=wsb)
-
-        def f_grads():
-            q.nf4_lora_linear_bwd(dy, xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
-                                  want=("dA", "dB"), dA=dAb, dB=dBb, workspace=wsb)
-
-        def f_all():
-            q.nf4_lora_linear_bwd(dy, xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
-                                  dx=dxb, dA=dAb, dB=dBb, workspace=wsb)
-        us_dx, us_gr, us_all = graph_us(f_dx, 3), graph_us(f_grads, 3), graph_us(f_all, 3)
-        q.nf4_device_status()
-        fl_dx = 2 * c.M * c.N * c.K + 2 * c.M * c.r * (c.N + c.K)
-        fl_gr = 2 * c.M * c.r * (c.N + c.K) * 2  # two down-projections + the two gradient products
-        emit(f"backward dx {c.name}", us_dx, fl_dx, "TFLOP/s", peak_sustained=peaks["bf16_tflops_sustained"])
-        emit(f"backward dA + dB {c.name}", us_gr, fl_gr, "TFLOP/s")
-        emit(f"backward dx + dA + dB {c.name}", us_all, fl_dx + fl_gr, "TFLOP/s")
-        del W, x, A, B, dy, st, xd, Ad, Bd, dxb, dAb, dBb, wsb
+        proj = "projection 4096x4096 bf16"
+        emit(f"quantize {proj}", graph_us(f_quant, 20), quantize_bytes(n), "GB/s")
+        emit(f"double_quantize {nb} constants", graph_us(f_dq, 20), dq_bytes(nb), "GB/s")
+        emit(f"dequantize {proj} -> bf16, DQ", graph_us(f_deq(True, False), 20), dequant_bytes(n), "GB/s")
+        emit(f"dequantize {proj} -> fp32, DQ", graph_us(f_deq(True, True), 20), dequant_bytes(n, 4), "GB/s")
+        nodq_b = n // 2 + nb * 4 + n * 2
+        emit(f"dequantize {proj} -> bf16, no DQ (fp32 c1)", graph_us(f_deq(False, False), 20), nodq_b, "GB/s",
+             bytes_per_param=round(nodq_b / n - 2, 6))
+        del Ws, sts, raw, absb, outs, outs32, q8s, c2s, offs
         torch.cuda.empty_cache()
 
-    # ---- merge the adapter into the quantized base and requantize (+ double
-    # quantization of the new constants), and the error the requantization adds
-    for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
-        W, _, A, B = wl.linear_inputs(c)
-        Wd, Ad, Bd = W.to(dev), A.to(dev), B.to(dev)
-        st = q.quantize_weight(Wd)
-        m = c.N * c.K
-        pk = torch.empty(m // 2, dtype=torch.uint8, device=dev)
-        ab = torch.empty(m // BLOCK, device=dev)
+    if want("linear"):
+        # ---- fused linear: decode GEMV and tensor-core GEMM, with / without DQ
+        def linear_case(c, dq, copies, reps):
+            W, x, A, B = wl.linear_inputs(c)
+            Wd = W.to(dev)
+            stl = [q.quantize_weight(Wd, double_quant=dq) for _ in range(copies)]
+            del W, Wd
+            xd, Ad, Bd = x.to(dev), A.to(dev), B.to(dev)
+            y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+            wsl = torch.empty(max(1, q.nf4_lora_linear_workspace_size(c.M, c.r)), dtype=torch.uint8, device=dev)
 
-        def f_merge():
-            q.nf4_merge_requantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N, c.K, Ad, Bd, c.scaling,
-                                   packed_out=pk, absmax_out=ab)
-        us = graph_us(f_merge, 3)
-        byts = dequant_bytes(m, 0) + c.r * c.K * 2 + c.N * c.r * 2 + m // 2 + (m // BLOCK) * 4
-        merged = q.merge_and_requantize(st, Ad, Bd, c.scaling)
-        w_base = q.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, m, torch.float32).view(c.N, c.K)
-        w_new = q.nf4_dequantize(merged.packed, merged.absmax_q, merged.absmax2, merged.offset, m,
-                                 torch.float32).view(c.N, c.K)
-        delta = c.scaling * (Bd.float() @ Ad.float())
-        w_exact = w_base + delta
-        rms = lambda t: float(t.pow(2).mean().sqrt())
-        emit(f"merge + requantize {c.N}x{c.K} r={c.r}", us, byts, "GB/s",
-             fma_per_s=round(m * c.r / (us * 1e-6) / 1e12, 3), fma_unit="T fma/s (fp32 chain)",
-             base_quant_rel_rms=round(rms(w_base - Wd.float()) / rms(Wd.float()), 6),
-             requant_rel_rms=round(rms(w_new - w_exact) / rms(w_exact), 6),
-             adapter_rel_rms=round(rms(delta) / rms(w_base), 6),
-             adapter_retained=round(float(((w_new - w_base) * delta).sum() / (delta * delta).sum()), 4))
-        del W, Wd, Ad, Bd, st, pk, ab, merged, w_base, w_new, delta, w_exact
+            def f():
+                st = stl[nxt(copies)]
+                q.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, Ad, Bd, c.scaling,
+                                      y=y, workspace=wsl)
+            us = graph_us(f, reps)
+            q.nf4_device_status()
+            wb = c.N * c.K // 2 + (c.N * c.K // BLOCK) * (1 if dq else 4) + (-(-(c.N * c.K // BLOCK) // DQ_BLOCK) * 4 + 4
+                                                                              if dq else 0)
+            byts = wb + c.M * c.K * 2 + c.r * c.K * 2 + c.N * c.r * 2 + c.M * c.N * 2
+            return us, byts
+
+        for c in wl.GEMV_CASES:
+            for dq in (True, False):
+                us, byts = linear_case(c, dq, 8, 20)
+                emit(f"{c.name}{'' if dq else ', no DQ'}", us, byts, "GB/s",
+                     tflops=round(linear_flops(c.M, c.K, c.N, c.r) / (us * 1e-6) / 1e12, 3))
+        for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
+            for dq in (True, False):
+                us, _ = linear_case(c, dq, 1, 5)
+                emit(f"{c.name}{'' if dq else ', no DQ'}", us, linear_flops(c.M, c.K, c.N, c.r), "TFLOP/s",
+                     peak_sustained=peaks["bf16_tflops_sustained"])
         torch.cuda.empty_cache()
 
-    # ---- one 8B-shaped decoder layer, M = 4096 tokens, r = 64, s = 0.25:
-    # fused NF4 + LoRA against bf16 x W^T + s (x A^T) B^T on cuBLAS
-    M, r, sc = 4096, 64, 0.25
-    t_nf4 = t_bf16 = 0.0
-    flops = 0
-    for idx, (name, N, K) in enumerate(wl.LAYER_8B):
-        W = wl.sweep_weight(0, idx).to(dev)
-        g = torch.Generator().manual_seed(wl.sweep_seed(0, idx) + 1)
-        x = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
-        A = (torch.randn(r, K, generator=g) * 0.01).to(torch.bfloat16).to(dev)
-        B = (torch.randn(N, r, generator=g) * 0.01).to(torch.bfloat16).to(dev)
-        st = q.quantize_weight(W)
-        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        wsl = torch.empty(q.nf4_lora_linear_workspace_size(M, r), dtype=torch.uint8, device=dev)
-        Wt, At, Bt = W.t(), A.t(), B.t()
+    if want("backward"):
+        # ---- backward through the frozen base: dx (fused NF4 GEMM) and the adapter gradients
+        for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
+            W, x, A, B = wl.linear_inputs(c)
+            g = torch.Generator().manual_seed(c.seed + 7)
+            dy = torch.randn(c.M, c.N, generator=g).to(torch.bfloat16).to(dev)
+            st = q.quantize_weight(W.to(dev))
+            xd, Ad, Bd = x.to(dev), A.to(dev), B.to(dev)
+            dxb = torch.empty(c.M, c.K, dtype=torch.bfloat16, device=dev)
+            dAb = torch.empty(c.r, c.K, device=dev)
+            dBb = torch.empty(c.N, c.r, device=dev)
+            wsb = torch.empty(q.nf4_lora_linear_bwd_workspace_size(c.M, c.N, c.K, c.r), dtype=torch.uint8, device=dev)
 
-        def f_nf4():
-            q.nf4_lora_linear_fwd(x, st.packed, st.absmax_q, st.absmax2, st.offset, N, A, B, sc, y=y, workspace=wsl)
+            def f_dx():
+                q.nf4_lora_linear_bwd(dy, None, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
+                                      want=("dx",), dx=dxb, workspace=wsb)
 
-        def f_bf16():
-            yb = torch.matmul(x, Wt)
-            torch.addmm(yb, torch.matmul(x, At), Bt, alpha=sc, out=y)
+            def f_grads():
+                q.nf4_lora_linear_bwd(dy, xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
+                                      want=("dA", "dB"), dA=dAb, dB=dBb, workspace=wsb)
 
-        a_us, b_us = graph_us(f_nf4, 3), graph_us(f_bf16, 3)
-        fl = linear_flops(M, K, N, r)
-        emit(f"layer {name} {N}x{K} M={M} r={r}: fused NF4+LoRA", a_us, fl, "TFLOP/s",
-             bf16_lora_us=round(b_us, 3), ratio_nf4_over_bf16=round(a_us / b_us, 4))
-        t_nf4, t_bf16, flops = t_nf4 + a_us, t_bf16 + b_us, flops + fl
-        del W, x, A, B, st, y, wsl
-    emit(f"8B decoder layer (7 linears) M={M} r={r}: fused NF4+LoRA", t_nf4, flops, "TFLOP/s",
-         bf16_lora_us=round(t_bf16, 3), overhead_vs_bf16=round(t_nf4 / t_bf16 - 1, 4),
-         note="forward linears only; the pages' 25-40 % slowdown figure is per training step")
-    torch.cuda.empty_cache()
+            def f_all():
+                q.nf4_lora_linear_bwd(dy, xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.K, Ad, Bd, c.scaling,
+                                      dx=dxb, dA=dAb, dB=dBb, workspace=wsb)
+            us_dx, us_gr, us_all = graph_us(f_dx, 3), graph_us(f_grads, 3), graph_us(f_all, 3)
+            q.nf4_device_status()
+            fl_dx = 2 * c.M * c.N * c.K + 2 * c.M * c.r * (c.N + c.K)
+            fl_gr = 2 * c.M * c.r * (c.N + c.K) * 2  # two down-projections + the two gradient products
+            emit(f"backward dx {c.name}", us_dx, fl_dx, "TFLOP/s", peak_sustained=peaks["bf16_tflops_sustained"])
+            emit(f"backward dA + dB {c.name}", us_gr, fl_gr, "TFLOP/s")
+            emit(f"backward dx + dA + dB {c.name}", us_all, fl_dx + fl_gr, "TFLOP/s")
+            del W, x, A, B, dy, st, xd, Ad, Bd, dxb, dAb, dBb, wsb
+            torch.cuda.empty_cache()
 
-    # ---- 8B-shaped whole-model sweep: quantize + DQ + dequantize of every
-    # linear weight, layer by layer (layer 0's seeded weights stand in for all
-    # 32 layers: the same shapes and work; 224 weights, 6.98e9 parameters)
-    Wl = [wl.sweep_weight(0, idx).to(dev).reshape(-1) for idx in range(len(wl.LAYER_8B))]
-    bufs = []
-    for w in Wl:
-        m = w.numel()
-        mb = m // BLOCK
-        bufs.append((torch.empty(m // 2, dtype=torch.uint8, device=dev), torch.empty(mb, device=dev),
-                     torch.empty(mb, dtype=torch.uint8, device=dev), torch.empty(-(-mb // DQ_BLOCK), device=dev),
-                     torch.empty(1, device=dev),
-                     torch.empty(q.nf4_double_quantize_workspace_size(mb), dtype=torch.uint8, device=dev),
-                     torch.empty(m, dtype=torch.bfloat16, device=dev)))
+    if want("merge"):
+        # ---- merge the adapter into the quantized base and requantize (+ double
+        # quantization of the new constants), and the error the requantization adds
+        for c in (wl.GEMM_TRAIN, wl.GEMM_70B_MLP):
+            W, _, A, B = wl.linear_inputs(c)
+            Wd, Ad, Bd = W.to(dev), A.to(dev), B.to(dev)
+            st = q.quantize_weight(Wd)
+            m = c.N * c.K
+            pk = torch.empty(m // 2, dtype=torch.uint8, device=dev)
+            ab = torch.empty(m // BLOCK, device=dev)
 
-    def f_layer():
-        for w, (pk, ab, q8, c2, off, wsd, out) in zip(Wl, bufs):
+            def f_merge():
+                q.nf4_merge_requantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N, c.K, Ad, Bd, c.scaling,
+                                       packed_out=pk, absmax_out=ab)
+            us = graph_us(f_merge, 3)
+            byts = dequant_bytes(m, 0) + c.r * c.K * 2 + c.N * c.r * 2 + m // 2 + (m // BLOCK) * 4
+            merged = q.merge_and_requantize(st, Ad, Bd, c.scaling)
+            w_base = q.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, m, torch.float32).view(c.N, c.K)
+            w_new = q.nf4_dequantize(merged.packed, merged.absmax_q, merged.absmax2, merged.offset, m,
+                                     torch.float32).view(c.N, c.K)
+            delta = c.scaling * (Bd.float() @ Ad.float())
+            w_exact = w_base + delta
+            rms = lambda t: float(t.pow(2).mean().sqrt())
+            emit(f"merge + requantize {c.N}x{c.K} r={c.r}", us, byts, "GB/s",
+                 fma_per_s=round(m * c.r / (us * 1e-6) / 1e12, 3), fma_unit="T fma/s (fp32 chain)",
+                 base_quant_rel_rms=round(rms(w_base - Wd.float()) / rms(Wd.float()), 6),
+                 requant_rel_rms=round(rms(w_new - w_exact) / rms(w_exact), 6),
+                 adapter_rel_rms=round(rms(delta) / rms(w_base), 6),
+                 adapter_retained=round(float(((w_new - w_base) * delta).sum() / (delta * delta).sum()), 4))
+            del W, Wd, Ad, Bd, st, pk, ab, merged, w_base, w_new, delta, w_exact
+            torch.cuda.empty_cache()
+
+    if want("layer"):
+        # ---- one 8B-shaped decoder layer, M = 4096 tokens, r = 64, s = 0.25:
+        # fused NF4 + LoRA against bf16 x W^T + s (x A^T) B^T on cuBLAS
+        M, r, sc = 4096, 64, 0.25
+        t_nf4 = t_bf16 = 0.0
+        flops = 0
+        for idx, (name, N, K) in enumerate(wl.LAYER_8B):
+            W = wl.sweep_weight(0, idx).to(dev)
+            g = torch.Generator().manual_seed(wl.sweep_seed(0, idx) + 1)
+            x = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
+            A = (torch.randn(r, K, generator=g) * 0.01).to(torch.bfloat16).to(dev)
+            B = (torch.randn(N, r, generator=g) * 0.01).to(torch.bfloat16).to(dev)
+            st = q.quantize_weight(W)
+            y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            wsl = torch.empty(q.nf4_lora_linear_workspace_size(M, r), dtype=torch.uint8, device=dev)
+            Wt, At, Bt = W.t(), A.t(), B.t()
+
+            def f_nf4():
+                q.nf4_lora_linear_fwd(x, st.packed, st.absmax_q, st.absmax2, st.offset, N, A, B, sc, y=y, workspace=wsl)
+
+            def f_bf16():
+                yb = torch.matmul(x, Wt)
+                torch.addmm(yb, torch.matmul(x, At), Bt, alpha=sc, out=y)
+
+            a_us, b_us = graph_us(f_nf4, 3), graph_us(f_bf16, 3)
+            fl = linear_flops(M, K, N, r)
+            emit(f"layer {name} {N}x{K} M={M} r={r}: fused NF4+LoRA", a_us, fl, "TFLOP/s",
+                 bf16_lora_us=round(b_us, 3), ratio_nf4_over_bf16=round(a_us / b_us, 4))
+            t_nf4, t_bf16, flops = t_nf4 + a_us, t_bf16 + b_us, flops + fl
+            del W, x, A, B, st, y, wsl
+        emit(f"8B decoder layer (7 linears) M={M} r={r}: fused NF4+LoRA", t_nf4, flops, "TFLOP/s",
+             bf16_lora_us=round(t_bf16, 3), overhead_vs_bf16=round(t_nf4 / t_bf16 - 1, 4),
+             note="forward linears only; the pages' 25-40 % slowdown figure is per training step")
+        torch.cuda.empty_cache()
+
+    if want("sweep"):
+        # ---- 8B-shaped whole-model sweep: quantize + DQ + dequantize of every
+        # linear weight, layer by layer (layer 0's seeded weights stand in for all
+        # 32 layers: the same shapes and work; 224 weights, 6.98e9 parameters)
+        Wl = [wl.sweep_weight(0, idx).to(dev).reshape(-1) for idx in range(len(wl.LAYER_8B))]
+        bufs = []
+        for w in Wl:
             m = w.numel()
-            q.nf4_quantize(w, packed=pk, absmax=ab)
-            q.nf4_double_quantize(ab, absmax_q=q8, absmax2=c2, offset=off, workspace=wsd)
-            q.nf4_dequantize(pk, q8, c2, off, m, torch.bfloat16, out=out)
+            mb = m // BLOCK
+            bufs.append((torch.empty(m // 2, dtype=torch.uint8, device=dev), torch.empty(mb, device=dev),
+                         torch.empty(mb, dtype=torch.uint8, device=dev), torch.empty(-(-mb // DQ_BLOCK), device=dev),
+                         torch.empty(1, device=dev),
+                         torch.empty(q.nf4_double_quantize_workspace_size(mb), dtype=torch.uint8, device=dev),
+                         torch.empty(m, dtype=torch.bfloat16, device=dev)))
 
-    layer_us = graph_us(f_layer, 4)
-    per_layer = sum(quantize_bytes(w.numel()) + dq_bytes(w.numel() // BLOCK) + dequant_bytes(w.numel()) for w in Wl)
-    L = wl.N_LAYERS_8B
-    emit(f"8B-shaped sweep: quantize + DQ + dequantize, {L} layers x 7 linears", layer_us * L, per_layer * L,
-         "GB/s", params=sum(w.numel() for w in Wl) * L, seconds=round(layer_us * L * 1e-6, 4))
+        def f_layer():
+            for w, (pk, ab, q8, c2, off, wsd, out) in zip(Wl, bufs):
+                m = w.numel()
+                q.nf4_quantize(w, packed=pk, absmax=ab)
+                q.nf4_double_quantize(ab, absmax_q=q8, absmax2=c2, offset=off, workspace=wsd)
+                q.nf4_dequantize(pk, q8, c2, off, m, torch.bfloat16, out=out)
+
+        layer_us = graph_us(f_layer, 4)
+        per_layer = sum(quantize_bytes(w.numel()) + dq_bytes(w.numel() // BLOCK) + dequant_bytes(w.numel()) for w in Wl)
+        L = wl.N_LAYERS_8B
+        emit(f"8B-shaped sweep: quantize + DQ + dequantize, {L} layers x 7 linears", layer_us * L, per_layer * L,
+             "GB/s", params=sum(w.numel() for w in Wl) * L, seconds=round(layer_us * L * 1e-6, 4))
 
 
 def main(argv=None):
@@ -665,6 +676,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sections", default="",
+                    help="with --suite: comma-separated subset of projection,linear,backward,merge,layer,sweep")
     ap.add_argument("--suite", action="store_true",
                     help="time every call in isolation (no-DQ variant, sweep, decoder layer); one line each")
     args = ap.parse_args(argv)
