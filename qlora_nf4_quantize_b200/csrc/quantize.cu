@@ -12,10 +12,10 @@
 // codes as one 32-bit word (4 packed bytes), a warp 128 contiguous bytes.
 //
 // Division-free exact code selection: instead of the per-element IEEE
-// division, each element uses q = RN(w * RN(1 / c1)), which is within 2^-22
-// of x = RN(w / c1).  A 129-cell table indexed by round(64 q) gives the code
-// below the cell and the (at most one) threshold inside the cell widened by
-// 2^-18; code = base + (q > t).  When |q - t| <= 2^-18 the decision could
+// division, each element uses q = RN(w * rc), rc the reciprocal of c1 to
+// within 1 ulp, which is within 2^-22 of x = RN(w / c1).  A 129-cell table
+// indexed by round(64 q) gives the code below the cell and the (at most one)
+// threshold inside the cell widened by 2^-18; code = base + (q > t).  When |q - t| <= 2^-18 the decision could
 // differ from the exact one and the element falls back to __fdiv_rn and a
 // full threshold count.  Each table word stores the threshold's bits with the
 // low 4 mantissa bits replaced by the base code (a perturbation below 2^-20,
@@ -29,6 +29,9 @@ constexpr float kAmbiguity = 0x1p-18f;
 constexpr int kCells = 129;       // cells 0..128 cover q in [-1, 1]
 constexpr int kCellTable = 256;   // indexed by the low byte of RN(64 q) + 64 (+ 1.5 * 2^23)
 constexpr int kQuantThreads = 256;
+#ifndef NF4_QUANT_RCP_APPROX
+#define NF4_QUANT_RCP_APPROX 1
+#endif
 
 __device__ __forceinline__ int exact_code(float w, float c1, const float *s_t) {
     return code_of_quotient(__fdiv_rn(w, c1), s_t);
@@ -118,15 +121,25 @@ __device__ __forceinline__ void quantize_group(float v[8], int64_t g, int64_t e0
         if (c1 >= 0x1p-125f && c1 < 0x1p125f) {
             // (outside this range 1/c1 may overflow or be subnormal, so the
             // 2^-22 error bound of the fast path would not hold)
+#if NF4_QUANT_RCP_APPROX
+            // hardware reciprocal, at most 1 ulp from 1 / c1 (PTX rcp.approx):
+            // |q - x| stays below 2^-22 (2^-23 + 2 half-ulps of rounding for
+            // |w / c1| <= 1), the bound the 2^-18 margin covers
+            float rc;
+            asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(c1));
+#else
             const float rc = __frcp_rn(c1);
+#endif
             uint64_t rc2, k64, kmagic;
             asm("mov.b64 %0, {%1, %1};" : "=l"(rc2) : "f"(rc));
             asm("mov.b64 %0, {%1, %1};" : "=l"(k64) : "f"(64.0f));
             asm("mov.b64 %0, {%1, %1};" : "=l"(kmagic) : "f"(12582976.0f));  // 1.5 * 2^23 + 64
             float dmin = 1.0f;  // smallest |q - t| of the group
+            // pairs (6, 7), (4, 5), (2, 3), (0, 1): codes enter the word most
+            // significant nibble first (byte m = code[2m] << 4 | code[2m+1])
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-                // q = RN(w * RN(1/c1)) and RN(64 q) + 64 in the low bits of
+            for (int i = 6; i >= 0; i -= 2) {
+                // q = RN(w * rc) and RN(64 q) + 64 in the low bits of
                 // f = RN(64 q + 1.5 * 2^23 + 64), two elements per packed op
                 uint64_t vv, qq, ff;
                 asm("mov.b64 %0, {%1, %2};" : "=l"(vv) : "f"(v[i]), "f"(v[i + 1]));
@@ -142,8 +155,7 @@ __device__ __forceinline__ void quantize_group(float v[8], int64_t g, int64_t e0
                     const uint32_t e = s_cell[__float_as_uint(f[j]) & 0xFFu];
                     const float t = __uint_as_float(e);
                     const uint32_t code = (e & 15u) + ((q[j] > t) ? 1u : 0u);
-                    const int el = i + j;  // element 2m in the high nibble of byte m
-                    word += code << (8 * (el >> 1) + ((el & 1) ? 0 : 4));
+                    word = (word << 4) | code;
                     dmin = fminf(dmin, fabsf(q[j] - t));
                 }
             }
