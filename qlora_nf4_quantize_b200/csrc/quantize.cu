@@ -32,6 +32,10 @@ constexpr int kQuantThreads = 256;
 #ifndef NF4_QUANT_RCP_APPROX
 #define NF4_QUANT_RCP_APPROX 1
 #endif
+// CTAs per SM in the grid; 0 = the number resident at once (occupancy query)
+#ifndef NF4_QUANT_CTAS_PER_SM
+#define NF4_QUANT_CTAS_PER_SM 0
+#endif
 
 __device__ __forceinline__ int exact_code(float w, float c1, const float *s_t) {
     return code_of_quotient(__fdiv_rn(w, c1), s_t);
@@ -204,7 +208,16 @@ cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed
     int64_t ngroups = (n + 7) / 8;
     int64_t span = (int64_t)kQuantThreads;
     int64_t want = (ngroups + span - 1) / span;
-    int64_t cap = (int64_t)num_sms * 8;
+    // one wave: as many CTAs as are resident at once (registers bound it to
+    // 5 per SM), so that no SM idles while a second, partial wave finishes
+    int per_sm = NF4_QUANT_CTAS_PER_SM;
+    if (per_sm <= 0) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &per_sm, bf16 ? k_quantize<true> : k_quantize<false>, kQuantThreads, 0);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+    }
+    int64_t cap = (int64_t)num_sms * per_sm;
     int grid = (int)(want < cap ? want : cap);
     if (bf16) return launch_pdl(k_quantize<true>, dim3(grid), dim3(kQuantThreads), 0, stream, 1, w, n, packed, absmax);
     return launch_pdl(k_quantize<false>, dim3(grid), dim3(kQuantThreads), 0, stream, 1, w, n, packed, absmax);
