@@ -75,6 +75,17 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128_b(const void *p, uint32_t
     return d;
 }
 
+// One lane of the (converged) warp, the same every time (the lowest).
+__device__ __forceinline__ bool elect_one_lane() {
+    uint32_t p;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(p));
+    return p != 0;
+}
+
 struct __align__(1024) BwdSmem {
     uint8_t g[kGStages][kGStageBytes];
     uint8_t wt[kGStages][kGStageBytes];
@@ -165,20 +176,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
     if (warp == 0) {
         // ---------------- TMA producer: g tiles, then [u_hi | u_lo] tiles ----------------
-        if (lane == 0) {
-            int issued = 0;
-            for (int kt = 0; kt < kt_total; ++kt) {
-                const int s = kt % kGStages;
-                const uint32_t ph = (uint32_t)(kt / kGStages) & 1u;
-                // u is written by the down-projection kernel launched just
-                // before (programmatic dependent launch)
-                if (kt == kn_steps) asm volatile("griddepcontrol.wait;" ::: "memory");
-                if (!mbar_wait(&S.empty[s], ph ^ 1u, abort, err)) break;
+        // (the whole warp runs the loop; one elected lane issues the copies)
+        const bool leader = elect_one_lane();
+        int issued = 0;
+        for (int kt = 0; kt < kt_total; ++kt) {
+            const int s = kt % kGStages;
+            const uint32_t ph = (uint32_t)(kt / kGStages) & 1u;
+            // u is written by the down-projection kernel launched just
+            // before (programmatic dependent launch)
+            if (kt == kn_steps) asm volatile("griddepcontrol.wait;" ::: "memory");
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.empty[s], ph ^ 1u, abort, err))) break;
+            if (leader) {
                 mbar_arrive_expect_tx(&S.full[s], kGStageBytes);
                 if (kt < kn_steps) tma_load_2d(S.g[s], &tmap_g, &S.full[s], kt * kGK, (int)m0);
                 else tma_load_2d(S.g[s], &tmap_u, &S.full[s], (kt - kn_steps) * kGK, (int)m0);
-                issued = kt + 1;
             }
+            __syncwarp();
+            issued = kt + 1;
+        }
+        if (leader) {
             for (int kt = issued - kGStages < 0 ? 0 : issued - kGStages; kt < issued; ++kt) {
                 unsigned long long t0 = global_ns();
                 while (!mbar_try_wait(&S.full[kt % kGStages], (uint32_t)(kt / kGStages) & 1u) &&
@@ -186,35 +202,42 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
             }
         }
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        if (lane == 0) {
+        // (the whole warp runs the loop; one elected lane issues the MMAs)
+        const bool leader = elect_one_lane();
+        {
             bool any = false;
             for (int kt = 0; kt < kt_total; ++kt) {
                 const int s = kt % kGStages;
                 const uint32_t ph = (uint32_t)(kt / kGStages) & 1u;
-                if (!mbar_wait(&S.full[s], ph, abort, err)) break;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.full[s], ph, abort, err))) break;
                 tc_fence_after();
-                const uint64_t a0 = smem_desc_sw128(S.g[s]);
-                const uint64_t a1 = smem_desc_sw128(S.g[s] + kGStageBytes / 2);  // tokens 128..255
-                const uint64_t bd = smem_desc_mn_sw128_b(S.wt[s], kGAtomCol);
+                if (leader) {
+                    const uint64_t a0 = smem_desc_sw128(S.g[s]);
+                    const uint64_t a1 = smem_desc_sw128(S.g[s] + kGStageBytes / 2);  // tokens 128..255
+                    const uint64_t bd = smem_desc_mn_sw128_b(S.wt[s], kGAtomCol);
 #pragma unroll
-                for (int kk = 0; kk < kGK / 16; ++kk) {
-                    const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
-                    const uint64_t b = bd + (uint64_t)(kk * 2048 >> 4);  // 16 rows n = two atoms along K
-                    tc_mma_ss(tmem, a0 + 2ull * kk, b, kGIdesc, acc);
-                    tc_mma_ss(tmem + 256u, a1 + 2ull * kk, b, kGIdesc, acc);
+                    for (int kk = 0; kk < kGK / 16; ++kk) {
+                        const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
+                        const uint64_t b = bd + (uint64_t)(kk * 2048 >> 4);  // 16 rows n = two atoms along K
+                        tc_mma_ss(tmem, a0 + 2ull * kk, b, kGIdesc, acc);
+                        tc_mma_ss(tmem + 256u, a1 + 2ull * kk, b, kGIdesc, acc);
+                    }
+                    tc_commit(&S.empty[s]);
+                    if (kt == kt_total - 1) tc_commit(&S.acc_full);
                 }
+                __syncwarp();
                 any = true;
-                tc_commit(&S.empty[s]);
-                if (kt == kt_total - 1) tc_commit(&S.acc_full);
             }
-            if (any && *abort) {  // drain our own MMAs before tensor memory is released
+            if (leader && any && *abort) {  // drain our own MMAs before tensor memory is released
                 tc_commit(&S.drain);
                 unsigned long long t0 = global_ns();
                 while (!mbar_try_wait(&S.drain, 0) && global_ns() - t0 < kWaitLimitNs) {
                 }
             }
+            __syncwarp();
         }
     } else if (warp >= 4) {
         // ---------------- dequant warpgroups (transposed tiles), then epilogue ----------------

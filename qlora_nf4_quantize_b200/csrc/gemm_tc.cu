@@ -139,6 +139,18 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         : "memory");
 }
 
+// One lane of the (converged) warp, the same every time: elect.sync picks
+// the lowest active lane.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(p));
+    return p != 0;
+}
+
 // The packed codes (8 words) and block constant of one 64-wide k-step of
 // weight row n; all-zero-code words outside the matrix.
 struct StepCodes {
@@ -245,17 +257,19 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
-        if (lane == 0) {
-            int issued = 0;
-            for (int g = 0; g < kg_total; ++g) {
-                const int s = g % kStages;
-                const uint32_t ph = (uint32_t)(g / kStages) & 1u;
-                const int kt0 = g * kSub;
-                const int nsub = kt_total - kt0 < kSub ? kt_total - kt0 : kSub;
-                // the t workspace is written by the down-projection kernel
-                // launched just before (programmatic dependent launch)
-                if (kt0 <= kw_steps && kw_steps < kt0 + nsub) asm volatile("griddepcontrol.wait;" ::: "memory");
-                if (!mbar_wait(&S.empty[s], ph ^ 1u, abort, err)) break;
+        // (the whole warp runs the loop; one elected lane issues the copies)
+        const bool leader = elect_one();
+        int issued = 0;
+        for (int g = 0; g < kg_total; ++g) {
+            const int s = g % kStages;
+            const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+            const int kt0 = g * kSub;
+            const int nsub = kt_total - kt0 < kSub ? kt_total - kt0 : kSub;
+            // the t workspace is written by the down-projection kernel
+            // launched just before (programmatic dependent launch)
+            if (kt0 <= kw_steps && kw_steps < kt0 + nsub) asm volatile("griddepcontrol.wait;" ::: "memory");
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.empty[s], ph ^ 1u, abort, err))) break;
+            if (leader) {
                 mbar_arrive_expect_tx(&S.full[s], (uint32_t)nsub * kXSubBytes);
                 for (int j = 0; j < nsub; ++j) {
                     const int kt = kt0 + j;
@@ -263,9 +277,12 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                     if (kt < kw_steps) tma_load_2d(dst, &tmap_x, &S.full[s], kt * kBK, (int)m0);
                     else tma_load_2d(dst, &tmap_t, &S.full[s], (kt - kw_steps) * kBK, (int)m0);
                 }
-                issued = g + 1;
             }
-            // drain: every issued load has landed before the CTA may exit
+            __syncwarp();
+            issued = g + 1;
+        }
+        // drain: every issued load has landed before the CTA may exit
+        if (leader) {
             for (int g = issued - kStages < 0 ? 0 : issued - kStages; g < issued; ++g) {
                 const int s = g % kStages;
                 const uint32_t ph = (uint32_t)(g / kStages) & 1u;
@@ -274,27 +291,31 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                 }
             }
         }
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            bool any = false, stop = false;
-            // Stage s: x tile at descriptor xdesc0 + (s * kXStageBytes) / 16
-            // (the start-address field counts 16-byte units and the sum is
-            // the stage's own address), weight k-step j at tensor-memory
-            // column kACol + 32 (kSub s + j).  Unrolled over the stages, so
-            // every offset is a constant and the issue loop stays short.
-            const uint64_t xdesc0 = smem_desc_sw128(S.x[0]);
-            for (int g0 = 0; !stop && g0 < kg_total; g0 += kStages) {
-                const uint32_t ph = (uint32_t)(g0 / kStages) & 1u;
+        // The whole warp runs the loop (its values stay warp-uniform); one
+        // elected lane issues the MMAs and the commits.
+        const bool leader = elect_one();
+        bool any = false, stop = false;
+        // Stage s: x tile at descriptor xdesc0 + (s * kXStageBytes) / 16
+        // (the start-address field counts 16-byte units and the sum is
+        // the stage's own address), weight k-step j at tensor-memory
+        // column kACol + 32 (kSub s + j).  Unrolled over the stages, so
+        // every offset is a constant and the issue loop stays short.
+        const uint64_t xdesc0 = smem_desc_sw128(S.x[0]);
+        for (int g0 = 0; !stop && g0 < kg_total; g0 += kStages) {
+            const uint32_t ph = (uint32_t)(g0 / kStages) & 1u;
 #pragma unroll
-                for (int s = 0; s < kStages; ++s) {
-                    const int g = g0 + s;
-                    if (g >= kg_total) break;
-                    if (!mbar_wait(&S.full[s], ph, abort, err)) {
-                        stop = true;
-                        break;
-                    }
-                    tc_fence_after();
+            for (int s = 0; s < kStages; ++s) {
+                const int g = g0 + s;
+                if (g >= kg_total) break;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.full[s], ph, abort, err))) {
+                    stop = true;
+                    break;
+                }
+                tc_fence_after();
+                if (leader) {
 #pragma unroll
                     for (int j = 0; j < kSub; ++j) {
                         const int kt = g * kSub + j;
@@ -307,10 +328,13 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                                 tc_mma_ts(tmem + kAccCol, acol + 8u * kk, bdesc + 2ull * kk, C::Idesc, 1u);
                         }
                     }
-                    any = true;
                     tc_commit(&S.empty[s]);
                 }
+                __syncwarp();
+                any = true;
             }
+        }
+        if (leader) {
             if (any && !stop) tc_commit(&S.acc_full);
             if (any && *abort) {  // drain our own MMAs before tensor memory is released
                 tc_commit(&S.drain);
@@ -319,6 +343,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                 }
             }
         }
+        __syncwarp();
     } else if (warp >= 4) {
         // ---------------- dequant warpgroups, then epilogue ----------------
         const int q = warp & 3;         // tensor-memory lane quarter
