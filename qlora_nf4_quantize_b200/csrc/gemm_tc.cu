@@ -193,15 +193,30 @@ __device__ __forceinline__ void dequant_step_smem(const StepCodes &sc, float mu,
     for (int s = 0; s < 16; ++s) pair_lookup4(tbl_lane, sc.w[s >> 1] >> ((s & 1) * 16), c, out[2 * s], out[2 * s + 1]);
 }
 
-// 64 columns [64 e, 64 e + 64) of the row n of [B | B | 0] (bf16 pairs).
+// 64 columns [64 e, 64 e + 64) of the row n of [B | B | 0] (bf16 pairs):
+// column j is B[n, j mod r] for j < 2r, else 0.  The row is read with
+// 16-byte loads (rows of 2r bytes, 16-byte aligned: r = 16, 32, 64); since 64 is a
+// multiple of r, column 64 e + 2c takes word c mod (r / 2) of the row.
+template <int R>
+__device__ __forceinline__ void lora_step_r(const __nv_bfloat16 *__restrict__ Bl, int64_t n, bool valid, int e,
+                                            uint32_t out[32]) {
+    // the row's R / 2 words go straight into out[0 .. R/2); the rest repeat
+    // them ([B | B]) or are zero (columns >= 2r)
+    const uint4 *src = reinterpret_cast<const uint4 *>(Bl + (valid ? n : 0) * R);
+#pragma unroll
+    for (int i = 0; i < R / 8; ++i) {
+        const uint4 u = valid ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+        out[4 * i] = u.x; out[4 * i + 1] = u.y; out[4 * i + 2] = u.z; out[4 * i + 3] = u.w;
+    }
+#pragma unroll
+    for (int c = R / 2; c < 32; ++c) out[c] = (64 * e + 2 * c < 2 * R) ? out[c % (R / 2)] : 0u;
+}
+
 __device__ __forceinline__ void lora_step(const __nv_bfloat16 *__restrict__ Bl, int r, int64_t n, bool valid,
                                           int e, uint32_t out[32]) {
-    const uint32_t *row = reinterpret_cast<const uint32_t *>(Bl + (valid ? n : 0) * r);
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-        const int j = 64 * e + 2 * c;
-        out[c] = (valid && j < 2 * r) ? __ldg(row + ((j % r) >> 1)) : 0u;
-    }
+    if (r == 16) lora_step_r<16>(Bl, n, valid, e, out);
+    else if (r == 32) lora_step_r<32>(Bl, n, valid, e, out);
+    else lora_step_r<64>(Bl, n, valid, e, out);
 }
 
 template <int kMode, class C>
