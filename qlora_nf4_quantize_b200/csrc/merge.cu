@@ -19,11 +19,11 @@
 // columns 8 l .. 8 l + 7, so every value of A read from shared memory feeds 8
 // rows (64 fma per 2 vector loads and 8 broadcast loads); the 8 lanes
 // 8 m .. 8 m + 7 own one 64-block of each row, whose absmax is a 3-step
-// shuffle.  The merged weight never leaves registers.  packed_out may alias
+// shuffle, and the codes come from the quantizer's exact selection.  The merged weight never leaves registers.  packed_out may alias
 // packed (every thread reads its 4 code bytes before it writes them), and
 // absmax_out may alias fp32 constants (a block's 8 lanes have read its
 // constant before the shuffles that precede its write).
-#include "nf4_device.cuh"
+#include "nf4_encode.cuh"
 
 namespace nf4 {
 namespace {
@@ -44,7 +44,8 @@ __global__ void __launch_bounds__(kMergeThreads)
     // sit 512 bytes apart, so consecutive lanes read consecutive 16 bytes
     float *sA = s_dyn;                      // [r][2][32][4]
     float *sB = s_dyn + r * kMergeCols;     // [64][r]
-    __shared__ float s_t[15];
+    __shared__ float s_t[16];
+    __shared__ uint32_t s_cell[kCellTable];
     __shared__ float s_lv[16];
     const int64_t k0 = (int64_t)blockIdx.x * kMergeCols;
     const int64_t n0 = (int64_t)blockIdx.y * kMergeRows;
@@ -60,8 +61,7 @@ __global__ void __launch_bounds__(kMergeThreads)
         sB[i] = n < N ? __bfloat162float(B[n * r + j]) : 0.0f;
     }
     if (threadIdx.x < 16) s_lv[threadIdx.x] = c_levels[threadIdx.x];
-    fill_thresholds(s_t);
-    __syncthreads();
+    build_code_tables(s_t, s_cell);  // (synchronises the CTA: sA, sB, s_lv ready too)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
@@ -114,12 +114,8 @@ __global__ void __launch_bounds__(kMergeThreads)
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
         if (!valid) continue;
-        uint32_t out = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const int code = amax == 0.0f ? 7 : code_of_quotient(__fdiv_rn(w[t], amax), s_t);
-            out |= (uint32_t)code << (8 * (t >> 1) + ((t & 1) ? 0 : 4));
-        }
+        // codes of RN(W' / c1) (nf4_encode.cuh: division-free, exact)
+        const uint32_t out = encode8(w, amax, s_t, s_cell);
         *reinterpret_cast<uint32_t *>(packed_out + (e >> 1)) = out;
         if ((lane & 7) == 0) absmax_out[e >> 6] = amax;
     }

@@ -11,57 +11,18 @@
 // 3-step xor-shuffle max inside that lane group.  Each thread writes its 8
 // codes as one 32-bit word (4 packed bytes), a warp 128 contiguous bytes.
 //
-// Division-free exact code selection: instead of the per-element IEEE
-// division, each element uses q = RN(w * rc), rc the reciprocal of c1 to
-// within 1 ulp, which is within 2^-22 of x = RN(w / c1).  A 129-cell table
-// indexed by round(64 q) gives the code below the cell and the (at most one)
-// threshold inside the cell widened by 2^-18; code = base + (q > t).  When |q - t| <= 2^-18 the decision could
-// differ from the exact one and the element falls back to __fdiv_rn and a
-// full threshold count.  Each table word stores the threshold's bits with the
-// low 4 mantissa bits replaced by the base code (a perturbation below 2^-20,
-// covered by the 2^-18 margin).
-#include "nf4_device.cuh"
+// The code selection itself (division-free, exact) is encode8 in
+// nf4_encode.cuh.
+#include "nf4_encode.cuh"
 
 namespace nf4 {
 namespace {
 
-constexpr float kAmbiguity = 0x1p-18f;
-constexpr int kCells = 129;       // cells 0..128 cover q in [-1, 1]
-constexpr int kCellTable = 256;   // indexed by the low byte of RN(64 q) + 64 (+ 1.5 * 2^23)
 constexpr int kQuantThreads = 256;
-#ifndef NF4_QUANT_RCP_APPROX
-#define NF4_QUANT_RCP_APPROX 1
-#endif
 // CTAs per SM in the grid; 0 = the number resident at once (occupancy query)
 #ifndef NF4_QUANT_CTAS_PER_SM
 #define NF4_QUANT_CTAS_PER_SM 0
 #endif
-
-__device__ __forceinline__ int exact_code(float w, float c1, const float *s_t) {
-    return code_of_quotient(__fdiv_rn(w, c1), s_t);
-}
-
-// Fill the thresholds and the cell table in shared memory (once per CTA).
-__device__ void build_tables(float *s_t, uint32_t *s_cell) {
-    int tid = threadIdx.x;
-    fill_thresholds(s_t);
-    __syncthreads();
-    if (tid >= kCells && tid < kCellTable) s_cell[tid] = 0x40800000u | 15u;  // never reached by finite q
-    if (tid < kCells) {
-        // cell tid holds q with RN(64 q) = tid - 64, i.e. q in [lo, hi]
-        float lo = ((float)tid - 64.5f) * 0.015625f;
-        float hi = ((float)tid - 63.5f) * 0.015625f;
-        int base = 0;
-        uint32_t word = 0x40800000u;  // 4.0f: no threshold near this cell
-        for (int i = 0; i < 15; ++i) {
-            float t = s_t[i];
-            if (t < lo - kAmbiguity) ++base;
-            else if (t <= hi + kAmbiguity) word = __float_as_uint(t);
-        }
-        s_cell[tid] = (word & ~15u) | (uint32_t)base;
-    }
-    __syncthreads();
-}
 
 template <bool kBf16>
 __device__ __forceinline__ void load8(const void *w, int64_t e0, int64_t n, float v[8]) {
@@ -116,62 +77,7 @@ __device__ __forceinline__ void quantize_group(float v[8], int64_t g, int64_t e0
     if (e0 >= n) return;
     if ((lane & 7) == 0) absmax[g >> 3] = c1;
 
-    uint32_t word;  // byte j = code[2j] << 4 | code[2j+1], bytes 0..3
-    if (c1 == 0.0f) {
-        word = 0x77777777u;
-    } else {
-        bool amb = true;  // take the exact path
-        word = 0;
-        if (c1 >= 0x1p-125f && c1 < 0x1p125f) {
-            // (outside this range 1/c1 may overflow or be subnormal, so the
-            // 2^-22 error bound of the fast path would not hold)
-#if NF4_QUANT_RCP_APPROX
-            // hardware reciprocal, at most 1 ulp from 1 / c1 (PTX rcp.approx):
-            // |q - x| stays below 2^-22 (2^-23 + 2 half-ulps of rounding for
-            // |w / c1| <= 1), the bound the 2^-18 margin covers
-            float rc;
-            asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(c1));
-#else
-            const float rc = __frcp_rn(c1);
-#endif
-            uint64_t rc2, k64, kmagic;
-            asm("mov.b64 %0, {%1, %1};" : "=l"(rc2) : "f"(rc));
-            asm("mov.b64 %0, {%1, %1};" : "=l"(k64) : "f"(64.0f));
-            asm("mov.b64 %0, {%1, %1};" : "=l"(kmagic) : "f"(12582976.0f));  // 1.5 * 2^23 + 64
-            float dmin = 1.0f;  // smallest |q - t| of the group
-            // pairs (6, 7), (4, 5), (2, 3), (0, 1): codes enter the word most
-            // significant nibble first (byte m = code[2m] << 4 | code[2m+1])
-#pragma unroll
-            for (int i = 6; i >= 0; i -= 2) {
-                // q = RN(w * rc) and RN(64 q) + 64 in the low bits of
-                // f = RN(64 q + 1.5 * 2^23 + 64), two elements per packed op
-                uint64_t vv, qq, ff;
-                asm("mov.b64 %0, {%1, %2};" : "=l"(vv) : "f"(v[i]), "f"(v[i + 1]));
-                asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(qq) : "l"(vv), "l"(rc2));
-                asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(ff) : "l"(qq), "l"(k64), "l"(kmagic));
-                float q[2], f[2];
-                asm("mov.b64 {%0, %1}, %2;" : "=f"(q[0]), "=f"(q[1]) : "l"(qq));
-                asm("mov.b64 {%0, %1}, %2;" : "=f"(f[0]), "=f"(f[1]) : "l"(ff));
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    // RN(64 q) + 64 is in [0, 128] for finite inputs; the byte
-                    // mask keeps any input inside the 256-entry table
-                    const uint32_t e = s_cell[__float_as_uint(f[j]) & 0xFFu];
-                    const float t = __uint_as_float(e);
-                    const uint32_t code = (e & 15u) + ((q[j] > t) ? 1u : 0u);
-                    word = (word << 4) | code;
-                    dmin = fminf(dmin, fabsf(q[j] - t));
-                }
-            }
-            amb = dmin <= kAmbiguity;  // rare: some quotient is within 2^-18 of a threshold
-        }
-        if (amb) {
-            word = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                word += (uint32_t)exact_code(v[i], c1, s_t) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
-        }
-    }
+    const uint32_t word = encode8(v, c1, s_t, s_cell);  // byte j = code[2j] << 4 | code[2j+1]
     if (e0 + 8 <= n) {
         reinterpret_cast<uint32_t *>(packed)[g] = word;
     } else {
@@ -186,7 +92,7 @@ __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restri
     __shared__ float s_t[16];
     __shared__ uint32_t s_cell[kCellTable];
     pdl_wait_then_release();
-    build_tables(s_t, s_cell);
+    build_code_tables(s_t, s_cell);
 
     const int lane = threadIdx.x & 31;
     const int64_t ngroups = (n + 7) >> 3;
