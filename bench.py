@@ -348,6 +348,7 @@ def oracle_dequant_rate(wp, budget_s):
     packed, c1 = oracle.quantize(bits)
     codes, c2, mu = oracle.double_quantize(c1)
     n = bits.size
+    oracle.dequantize(packed, codes, c2, mu, n, "bf16")  # first call: one-time setup, untimed
     reps, t0 = 0, time.perf_counter()
     while True:
         oracle.dequantize(packed, codes, c2, mu, n, "bf16")
@@ -358,28 +359,82 @@ def oracle_dequant_rate(wp, budget_s):
     return reps * dequant_bytes(n) / el / 1e9, reps, el
 
 
+def _oracle_slice_worker(job):
+    """One host process: the oracle's dequant of one slice of the quantized
+    state (whole runs of 256 blocks), repeated for budget_s seconds."""
+    packed, codes, c2, mu, n, budget_s = job
+    import oracle
+    oracle.dequantize(packed, codes, c2, mu, n, "bf16")  # first call: one-time setup, untimed
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.dequantize(packed, codes, c2, mu, n, "bf16")
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return reps, n, el
+
+
+def oracle_dequant_rate_cores(wp, budget_s, cores):
+    """The oracle's dequant on `cores` host processes at once (spawned, each a
+    slice of the weight on run boundaries); returns (GB/s, bytes moved)."""
+    import multiprocessing as mp
+    import torch
+    import oracle
+    bits = wp.contiguous().view(torch.int16).numpy().view(np.uint16).ravel()
+    packed, c1 = oracle.quantize(bits)
+    codes, c2, mu = oracle.double_quantize(c1)
+    n = bits.size
+    run = BLOCK * DQ_BLOCK
+    runs = -(-n // run)
+    jobs = []
+    for i in range(cores):
+        r0, r1 = runs * i // cores, runs * (i + 1) // cores
+        e0, e1 = r0 * run, min(r1 * run, n)
+        if e1 <= e0:
+            continue
+        jobs.append((packed[e0 // 2:(e1 + 1) // 2].copy(), codes[e0 // BLOCK:-(-e1 // BLOCK)].copy(),
+                     c2[r0:r1].copy(), mu, e1 - e0, budget_s))
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(len(jobs)) as pool:
+        res = pool.map(_oracle_slice_worker, jobs)
+    # the processes run side by side for the same budget: rates add up
+    return sum(reps * dequant_bytes(m) / el for reps, m, el in res) / 1e9, len(jobs)
+
+
+def host_cores():
+    """Host cores the oracle may use (the host is shared: at most 16)."""
+    return max(1, min(16, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)))
+
+
 def cpu_baseline(wp, budget_s=10.0):
-    gbs, reps, el = oracle_dequant_rate(wp, budget_s)
-    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"oracle nf4 dequantize (bf16 out) of the full 4096x4096 projection weight, {reps} passes "
-                      f"in {el:.1f} s, single thread"}
+    gbs1, reps, el = oracle_dequant_rate(wp, budget_s * 0.4)
+    cores = host_cores()
+    gbs, used = oracle_dequant_rate_cores(wp, budget_s * 0.6, cores) if cores > 1 else (gbs1, 1)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": used, "kind": "oracle", "value_1core": round(gbs1, 4),
+            "sample": f"oracle nf4 dequantize (bf16 out) of the 4096x4096 projection weight: {used} host processes "
+                      f"on slices of whole 256-block runs for {budget_s * 0.6:.0f} s; single thread {reps} full "
+                      f"passes in {el:.1f} s (value_1core)"}
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
+    import torch
     import nf4_workloads as wl
+    import oracle
     wp = wl.weight((4096, 4096), 0.02, wl.PROJECTION["seed"], "bf16", outliers=True)
-    for _ in range(args.warmup):
-        oracle_dequant_rate(wp, 0.0)
+    bits = wp.contiguous().view(torch.int16).numpy().view(np.uint16).ravel()
+    packed, c1 = oracle.quantize(bits)
+    codes, c2, mu = oracle.double_quantize(c1)
+    n = bits.size
+    for _ in range(max(1, args.warmup)):
+        oracle.dequantize(packed, codes, c2, mu, n, "bf16")
     t0 = time.perf_counter()
-    gbs = []
     for _ in range(args.steps):
-        g, _, _ = oracle_dequant_rate(wp, 0.0)
-        gbs.append(g)
+        oracle.dequantize(packed, codes, c2, mu, n, "bf16")
     el = time.perf_counter() - t0
-    n = wp.numel()
     value = args.steps * dequant_bytes(n) / el / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
@@ -387,7 +442,8 @@ def run_reference(args):
             "config": {"workload": "projection 4096x4096 bf16 (0.1% x10 outliers): NF4 dequantize (bf16 out), "
                                    "CPU oracle (plain C, single thread)", "parallelism": "rank 0 only"},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{args.steps} full dequantize passes of the projection weight"},
+                             "sample": f"{args.steps} full dequantize passes of the projection weight "
+                                       f"(state quantized once by the oracle, outside the timed region)"},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
