@@ -71,10 +71,10 @@ constexpr uint32_t pow2_at_least(uint32_t v) {
 }
 
 // Token tile BT (MMA N), pipeline depth and dequant warpgroups of one
-// instantiation: BT = 256 for the large-M GEMM; BT = 16 serves decode-size M
-// when built with NF4_SMALL_M_TC=1 (one 128-row tile per CTA: 86 CTAs for an
-// 11008-row weight, and a k-step rate bound by the dequant warps' latency,
-// measured slower than the warp-MMA GEMV kernels, so not the default).
+// instantiation: BT = 256 for the large-M GEMM; BT = 16 serves 9 to 16 tokens
+// (one 128-row tile per CTA, a rate bound by the dequantization, the same for
+// any token count up to 16; below 9 tokens the warp-MMA GEMV kernels are
+// faster).
 constexpr uint32_t AccColsFor(int bt) { return bt < 32 ? 32u : (uint32_t)bt; }
 
 template <int BT_, int STAGES_, int WG_, int SUB_>

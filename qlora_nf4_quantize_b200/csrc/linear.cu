@@ -18,8 +18,13 @@ cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const
                            void *y, cudaStream_t stream, int num_sms, unsigned *err_word);
 
 constexpr int kGemvMaxTokens = 16;
-#ifndef NF4_SMALL_M_TC
-#define NF4_SMALL_M_TC 0
+// Token counts from which decode-size calls take the tcgen05 pipeline with a
+// 16-token tile instead of the warp-MMA GEMV kernels: that pipeline takes
+// the same time for any count up to 16 (25.7 us without LoRA on an 11008 x
+// 4096 weight), the warp-MMA kernels grow with it (17.0 us at 1 token, 21.8
+// at 8, 27.5 at 12, 30.3 at 16: above 8 tokens they need two token tiles).
+#ifndef NF4_SMALL_M_TC_FROM
+#define NF4_SMALL_M_TC_FROM 9
 #endif
 
 // Device error word: one per device, cleared by nf4_device_status().
@@ -52,9 +57,9 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
                                             : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream, 0);
         if (e != cudaSuccess) return e;
     }
-    // decode-size M: the warp-MMA GEMV kernels, or (built with
-    // NF4_SMALL_M_TC=1) the tcgen05 pipeline with a 16-token tile
-    if (M <= kGemvMaxTokens && !NF4_SMALL_M_TC)
+    // decode-size M: the warp-MMA GEMV kernels up to NF4_SMALL_M_TC_FROM - 1
+    // tokens, then the tcgen05 pipeline with a 16-token tile
+    if (M < NF4_SMALL_M_TC_FROM && M <= kGemvMaxTokens)
         return launch_gemv(x, (int)M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms);
     return launch_gemm_tc(x, M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms,
                           err_word);
