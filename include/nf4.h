@@ -167,8 +167,10 @@ NF4_API int64_t nf4_lora_linear_workspace_size(int64_t M, int r);
  *   y          device bf16[M, N] (output)
  *   workspace  device scratch, workspace_bytes >=
  *              nf4_lora_linear_workspace_size(M, r); NULL allowed when r == 0
- * M <= 16 runs the streaming GEMV kernel, larger M the tensor-core GEMM
- * kernel; the LoRA pre-step is one extra launch when r > 0. */
+ * M <= 8 runs the streaming warp-MMA GEMV kernel, 9 <= M <= 16 the
+ * tensor-core GEMM pipeline with a 16-token tile, larger M the same
+ * pipeline with 256-token tiles; the LoRA pre-step is one extra launch
+ * when r > 0. */
 NF4_API nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N,
                                const uint8_t *packed, const uint8_t *absmax_q,
                                const float *absmax2, const float *offset,
