@@ -22,8 +22,9 @@ cudaError_t launch_dequantize(const uint8_t *packed, const uint8_t *q8, const fl
 cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
                                const uint8_t *q8, const float *scales, const float *offset, const void *A,
                                const void *B, int r, float scaling, void *y, void *workspace,
-                               cudaStream_t stream, int num_sms, unsigned *err_word);
+                               int64_t workspace_bytes, cudaStream_t stream, int num_sms, unsigned *err_word);
 int64_t lora_workspace_bytes(int64_t M, int r);
+int64_t linear_workspace_bytes(int64_t M, int r);
 unsigned *device_error_word(cudaError_t *status);
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_merge_requantize(const uint8_t *packed, const uint8_t *q8, const float *scales,
@@ -147,8 +148,8 @@ nf4_status nf4_dequantize(const uint8_t *packed, const uint8_t *absmax_q, const 
 }
 
 int64_t nf4_lora_linear_workspace_size(int64_t M, int r) {
-    if (M <= 0 || r <= 0) return 0;
-    return nf4::lora_workspace_bytes(M, r);
+    if (M <= 0 || r < 0) return 0;
+    return nf4::linear_workspace_bytes(M, r);
 }
 
 nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
@@ -172,7 +173,8 @@ nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N, c
     if (st != cudaSuccess) return cuda_status(st);
     return cuda_status(nf4::launch_lora_linear(x, M, K, N, packed, absmax_q, absmax2, offset, lora ? A : nullptr,
                                                lora ? B : nullptr, lora ? r : 0, scaling, y, workspace,
-                                               (cudaStream_t)stream, sms, err));
+                                               workspace == nullptr ? 0 : workspace_bytes, (cudaStream_t)stream,
+                                               sms, err));
 }
 
 int64_t nf4_lora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {

@@ -127,6 +127,7 @@ struct __align__(1024) SmemLayout {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    int last[2];  // stream-K: this CTA adds up tile tile0 + h (h = segment)
 };
 
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -219,32 +220,87 @@ __device__ __forceinline__ void lora_step(const __nv_bfloat16 *__restrict__ Bl, 
     else lora_step_r<64>(Bl, n, valid, e, out);
 }
 
-template <int kMode, class C>
+// Stream-K split (kSK, 16-token tile only).  The CTAs share out the
+// sequence of (weight tile, k-step) pairs, tile after tile, in equal
+// contiguous ranges [c T / G, (c + 1) T / G) of the T = tiles x kt_total
+// steps, so that every SM streams the same share of the weight whatever the
+// number of 128-row tiles.  With at least as many CTAs as tiles a range
+// covers the end of one tile and the start of the next at most; each part
+// (segment) accumulates into its own tensor-memory columns and is written as
+// an fp32 partial tile [16 tokens][128 rows].  The CTA that completes a
+// tile's arrival count adds the tile's partials in CTA order (so the result
+// does not depend on timing) and writes y.  The counts are zeroed by the
+// kernel launched just before (programmatic dependent launch), which is
+// awaited before the first count.
+template <class C, bool kSK>
+struct TmemPlan {
+    static constexpr int kAccs = kSK ? 2 : 1;                   // accumulators (segments)
+    static constexpr uint32_t ACol = kAccs * C::AccCols;        // first A column
+    static constexpr uint32_t Cols = pow2_at_least(ACol + 32 * C::Sub * C::Stages);
+    static_assert(Cols <= 512, "tensor memory: accumulators + 32 columns per A stage");
+    static_assert(!kSK || (C::Sub == 1 && C::BT == 16), "stream-K split: 16-token tile, one k-step per stage");
+    static_assert(!kSK || C::WG >= 2, "stream-K split: one epilogue warpgroup per segment");
+};
+
+// Partial tile of one segment: [16 tokens][128 rows] fp32.
+constexpr int kPartialFloats = 16 * 128;
+// Most CTAs of a split launch (the partials are sized for them) and fewest
+// k-steps per CTA worth a split.
+constexpr int kStreamKMaxCtas = 192;
+constexpr int kStreamKMinSteps = 8;
+
+// CTA of a split launch of `ctas` CTAs whose range holds global step s of
+// `total`: the largest c with c total / ctas <= s.
+__device__ __forceinline__ int64_t streamk_cta_of(int64_t s, int64_t total, int64_t ctas) {
+    return (s * ctas + ctas - 1) / total;
+}
+
+template <int kMode, class C, bool kSK>
 __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_t,
               const __grid_constant__ CUtensorMap tmap_y, int64_t M,
               int64_t K, int64_t N, const uint8_t *__restrict__ packed, const uint8_t *__restrict__ q8,
               const float *__restrict__ scales, const float *__restrict__ offset,
-              const __nv_bfloat16 *__restrict__ Bl, int r, int rp, __nv_bfloat16 *__restrict__ y, unsigned *err) {
+              const __nv_bfloat16 *__restrict__ Bl, int r, int rp, __nv_bfloat16 *__restrict__ y,
+              float *__restrict__ partials, unsigned *__restrict__ counts, unsigned *err) {
     extern __shared__ uint8_t smem_raw[];
     constexpr int kBT = C::BT, kStages = C::Stages, kWG = C::WG, kSub = C::Sub;
-    constexpr uint32_t kTmemCols = C::TmemCols, kAccCol = 0, kACol = C::ACol, kXSubBytes = C::XSubBytes,
-                       kXStageBytes = C::XStageBytes;
+    constexpr uint32_t kTmemCols = TmemPlan<C, kSK>::Cols, kAccCol = 0, kACol = TmemPlan<C, kSK>::ACol,
+                       kXSubBytes = C::XSubBytes, kXStageBytes = C::XStageBytes;
     SmemLayout<C> &S =
         *reinterpret_cast<SmemLayout<C> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     volatile int *abort = &S.abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n0 = (int64_t)blockIdx.x * kBN;
     const int64_t m0 = (int64_t)blockIdx.y * kBT;
     const int kw_steps = (int)(K / kBK);
     const int kt_total = kw_steps + (r > 0 ? rp / kBK : 0);
-    const int kg_total = (kt_total + kSub - 1) / kSub;  // pipeline stages (groups of kSub k-steps)
+    // This CTA's k-steps: i = 0 .. steps-1 run over weight tile tile0 from
+    // k-step kt_first, and from i = i_next over tile tile0 + 1 from k-step 0
+    // (stream-K only; otherwise one whole tile, i_next = steps).
+    int64_t tile0 = blockIdx.x, total = 0;
+    int kt_first = 0, steps = kt_total, i_next = kt_total;
+    if constexpr (kSK) {
+        total = ((N + kBN - 1) / kBN) * kt_total;
+        const int64_t lo = (int64_t)blockIdx.x * total / gridDim.x;
+        const int64_t hi = (int64_t)(blockIdx.x + 1) * total / gridDim.x;
+        tile0 = lo / kt_total;
+        kt_first = (int)(lo - tile0 * kt_total);
+        steps = (int)(hi - lo);
+        i_next = kt_total - kt_first;
+    }
+    const int64_t n0 = tile0 * kBN;
+    // segment (0 or 1) and k-step of step i
+    auto seg_of = [&](int i) { return kSK ? (i >= i_next ? 1 : 0) : 0; };
+    auto kt_of = [&](int i) { return kSK ? (i >= i_next ? i - i_next : kt_first + i) : i; };
+    const int kg_total = (steps + kSub - 1) / kSub;  // pipeline stages (groups of kSub k-steps)
     // Programmatic dependent launch.  With an adapter the grid before this one
     // is the down-projection, which releases it only after its own
     // predecessor completed: x and W may be read at once, t only after the
-    // wait in the extension steps.  Without one, wait before reading anything.
-    if (r <= 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // wait in the extension steps.  The split launch is always preceded by a
+    // kernel of that kind (the down-projection, or the zeroing of its arrival
+    // counts).  Otherwise, without an adapter, wait before reading anything.
+    if (!kSK && r <= 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
@@ -275,19 +331,24 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         // (the whole warp runs the loop; one elected lane issues the copies)
         const bool leader = elect_one();
         int issued = 0;
+        bool t_ready = false;
         for (int g = 0; g < kg_total; ++g) {
             const int s = g % kStages;
             const uint32_t ph = (uint32_t)(g / kStages) & 1u;
-            const int kt0 = g * kSub;
-            const int nsub = kt_total - kt0 < kSub ? kt_total - kt0 : kSub;
+            const int i0 = g * kSub;
+            const int nsub = steps - i0 < kSub ? steps - i0 : kSub;
             // the t workspace is written by the down-projection kernel
-            // launched just before (programmatic dependent launch)
-            if (kt0 <= kw_steps && kw_steps < kt0 + nsub) asm volatile("griddepcontrol.wait;" ::: "memory");
+            // launched just before (programmatic dependent launch): wait
+            // before the first extension step
+            if (!t_ready && kt_of(i0 + nsub - 1) >= kw_steps) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                t_ready = true;
+            }
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.empty[s], ph ^ 1u, abort, err))) break;
             if (leader) {
                 mbar_arrive_expect_tx(&S.full[s], (uint32_t)nsub * kXSubBytes);
                 for (int j = 0; j < nsub; ++j) {
-                    const int kt = kt0 + j;
+                    const int kt = kt_of(i0 + j);
                     uint8_t *dst = S.x[s] + j * kXSubBytes;
                     if (kt < kw_steps) tma_load_2d(dst, &tmap_x, &S.full[s], kt * kBK, (int)m0);
                     else tma_load_2d(dst, &tmap_t, &S.full[s], (kt - kw_steps) * kBK, (int)m0);
@@ -333,14 +394,16 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                 if (leader) {
 #pragma unroll
                     for (int j = 0; j < kSub; ++j) {
-                        const int kt = g * kSub + j;
-                        if (kSub == 1 || kt < kt_total) {
+                        const int i = g * kSub + j;
+                        if (kSub == 1 || i < steps) {
                             const uint64_t bdesc = xdesc0 + (uint64_t)((s * kXStageBytes + j * kXSubBytes) >> 4);
                             const uint32_t acol = tmem + kACol + 32u * (uint32_t)(kSub * s + j);
-                            tc_mma_ts(tmem + kAccCol, acol, bdesc, C::Idesc, kt != 0 ? 1u : 0u);
+                            // the first step of each segment starts its accumulator
+                            const uint32_t dcol = tmem + kAccCol + C::AccCols * (uint32_t)seg_of(i);
+                            tc_mma_ts(dcol, acol, bdesc, C::Idesc, (i != 0 && i != i_next) ? 1u : 0u);
 #pragma unroll
                             for (int kk = 1; kk < kBK / 16; ++kk)
-                                tc_mma_ts(tmem + kAccCol, acol + 8u * kk, bdesc + 2ull * kk, C::Idesc, 1u);
+                                tc_mma_ts(dcol, acol + 8u * kk, bdesc + 2ull * kk, C::Idesc, 1u);
                         }
                     }
                     tc_commit(&S.empty[s]);
@@ -364,8 +427,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         const int q = warp & 3;         // tensor-memory lane quarter
         const int h = (warp - 4) >> 2;  // warpgroup: k-steps with index % kWG == h
         const int row_in_tile = 32 * q + lane;
-        const int64_t n = n0 + row_in_tile;
-        const bool nvalid = n < N;
+        // weight row of step i (the next tile's from i_next on)
+        auto row_of = [&](int i) { return n0 + (int64_t)kBN * seg_of(i) + row_in_tile; };
         const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         bool ok = true;
@@ -379,8 +442,10 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         auto load_group = [&](int g, StepCodes(&set)[kSub]) {
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
-                const int kt = g * kSub + j;
-                if (kt < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, kt, nvalid, set[j]);
+                const int i = g * kSub + j;
+                const int kt = kt_of(i);
+                const int64_t n = row_of(i);
+                if (i < steps && kt < kw_steps) load_step<kMode>(packed, q8, scales, mu, n, K, kt, n < N, set[j]);
             }
         };
 #pragma unroll
@@ -398,14 +463,16 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                 if (g + kPF * kWG < kg_total) load_group(g + kPF * kWG, ring[(i + kPF) % (kPF + 1)]);
 #pragma unroll
                 for (int j = 0; j < kSub; ++j) {
-                    const int kt = g * kSub + j;
-                    if (kt >= kt_total) break;
+                    const int ii = g * kSub + j;
+                    if (ii >= steps) break;
+                    const int kt = kt_of(ii);
                     uint32_t v[32];
                     if (kt < kw_steps) {
                         if ((kLutMask >> h) & 1) dequant_step_smem<kMode>(ring[i][j], mu, S.pairs + (lane & 15), v);
                         else dequant_step<kMode>(ring[i][j], mu, v);
                     } else {
-                        lora_step(Bl, r, n, nvalid, kt - kw_steps, v);
+                        const int64_t n = row_of(ii);
+                        lora_step(Bl, r, n, n < N, kt - kw_steps, v);
                     }
                     if (j == 0) {
                         // warp-uniform outcome: the tcgen05.st below is a warp-wide instruction
@@ -421,7 +488,55 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
             }
         }
         if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err));
-        if (ok) {
+        if constexpr (kSK) {
+            // Epilogue (stream-K): warpgroup h takes segment h.
+            const int nseg = steps > i_next ? 2 : 1;
+            if (h < nseg) {
+                const int64_t tile = tile0 + h;
+                if (ok) {
+                    tc_fence_after();
+                    uint32_t v[32];
+                    tc_load32(lane_base + kAccCol + C::AccCols * (uint32_t)h, v);  // columns 16..31 unused
+                    tc_wait_ld();
+                    float *dst = partials + (int64_t)(2 * blockIdx.x + h) * kPartialFloats + row_in_tile;
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) dst[m * 128] = __uint_as_float(v[m]);
+                }
+                __threadfence();  // the partial is visible before this CTA's arrival
+                asm volatile("bar.sync %0, 128;" ::"r"(2 + h) : "memory");
+                if (row_in_tile == 0) {
+                    // the counts were zeroed by the grid before this one
+                    asm volatile("griddepcontrol.wait;" ::: "memory");
+                    const int64_t c0 = streamk_cta_of(tile * kt_total, total, gridDim.x);
+                    const int64_t c1 = streamk_cta_of(tile * kt_total + kt_total - 1, total, gridDim.x);
+                    const unsigned prev = atomicAdd(counts + tile, 1u);
+                    S.last[h] = prev == (unsigned)(c1 - c0);
+                }
+                asm volatile("bar.sync %0, 128;" ::"r"(2 + h) : "memory");
+                if (S.last[h]) {
+                    // every partial of the tile is in: add them in CTA order
+                    __threadfence();
+                    const int64_t c0 = streamk_cta_of(tile * kt_total, total, gridDim.x);
+                    const int64_t c1 = streamk_cta_of(tile * kt_total + kt_total - 1, total, gridDim.x);
+                    float acc[16];
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) acc[m] = 0.0f;
+                    for (int64_t c = c0; c <= c1; ++c) {
+                        // segment 0 when CTA c's range starts in this tile, else 1
+                        const int seg = (c * total / gridDim.x) / kt_total == tile ? 0 : 1;
+                        const float *src = partials + (2 * c + seg) * kPartialFloats + row_in_tile;
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) acc[m] += __ldcg(src + m * 128);
+                    }
+                    const int64_t n = tile * kBN + row_in_tile;
+                    if (n < N) {
+#pragma unroll
+                        for (int m = 0; m < 16; ++m)
+                            if (m < M) y[m * N + n] = __float2bfloat16_rn(acc[m]);
+                    }
+                }
+            }
+        } else if (ok) {
             // Epilogue: accumulators -> bf16 -> staging tile Y[m][n] (256 x 128,
             // row-major, in the now idle x ring) -> one TMA store, which also
             // clips rows and columns outside y.
@@ -441,7 +556,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         }
         // all dequant/epilogue threads have staged their values (or given up)
         asm volatile("bar.sync 1, %0;" ::"n"(128 * kWG) : "memory");
-        if (threadIdx.x == 128 && !*abort) {
+        if (!kSK && threadIdx.x == 128 && !*abort) {
             asm volatile(
                 "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
                     reinterpret_cast<uint64_t>(&tmap_y)),
@@ -460,15 +575,17 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     }
 }
 
-template <int kMode, class C>
+template <int kMode, class C, bool kSK>
 cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUtensorMap &my, int64_t M, int64_t K, int64_t N,
                         const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
-                        const __nv_bfloat16 *Bl, int r, int rp, __nv_bfloat16 *y, unsigned *err, cudaStream_t stream) {
+                        const __nv_bfloat16 *Bl, int r, int rp, __nv_bfloat16 *y, float *partials, unsigned *counts,
+                        int ctas, unsigned *err, cudaStream_t stream) {
     const size_t smem = sizeof(SmemLayout<C>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<kMode, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_gemm_tc<kMode, C, kSK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + C::BT - 1) / C::BT));
+    cfg.gridDim = kSK ? dim3((unsigned)ctas) : dim3((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + C::BT - 1) / C::BT));
     cfg.blockDim = dim3(C::Threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -477,14 +594,15 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUte
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode, C>, mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, y,
-                              err);
+    return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode, C, kSK>, mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r,
+                              rp, y, partials, counts, err);
 }
 
-template <class C>
+template <class C, bool kSK>
 cudaError_t launch_cfg(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                        const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
-                       void *y, cudaStream_t stream, unsigned *err_word) {
+                       void *y, float *partials, unsigned *counts, int ctas, cudaStream_t stream,
+                       unsigned *err_word) {
     CUtensorMap mx, mt, my;
     cudaError_t e = make_map(&mx, x, M, K, kBK, C::BT, true);
     if (e != cudaSuccess) return e;
@@ -496,10 +614,13 @@ cudaError_t launch_cfg(const void *x, int64_t M, int64_t K, int64_t N, const uin
     auto *Bl = static_cast<const __nv_bfloat16 *>(B);
     auto *yp = static_cast<__nv_bfloat16 *>(y);
     if (q8 == nullptr)
-        return launch_mode<2, C>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+        return launch_mode<2, C, kSK>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, partials, counts,
+                                      ctas, err_word, stream);
     if (offset == nullptr)
-        return launch_mode<1, C>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
-    return launch_mode<0, C>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, err_word, stream);
+        return launch_mode<1, C, kSK>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, partials, counts,
+                                      ctas, err_word, stream);
+    return launch_mode<0, C, kSK>(mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r, rp, yp, partials, counts,
+                                  ctas, err_word, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -744,13 +865,40 @@ cudaError_t launch_down_tc_split(const CUtensorMap &mx, const CUtensorMap &ma, i
 
 }  // namespace
 
+// Scratch of a split launch: the partial tiles (2 per CTA) and one arrival
+// count per weight tile.
+int64_t streamk_partials_bytes() { return (int64_t)kStreamKMaxCtas * 2 * kPartialFloats * (int64_t)sizeof(float); }
+int64_t streamk_counts_bytes() { return (int64_t)kStreamKMaxCtas * (int64_t)sizeof(unsigned); }
+
+// CTAs of a split launch of the 16-token tile (0 = run it unsplit): `sms`
+// SMs for the linear, at most kStreamKMaxCtas, none with fewer than
+// kStreamKMinSteps k-steps, and more CTAs than 128-row tiles.
+int streamk_ctas(int64_t M, int64_t K, int64_t N, int rp, int sms) {
+    if (M > CfgSmall::BT) return 0;
+    const int64_t ntiles = (N + kBN - 1) / kBN;
+    const int64_t total = ntiles * (K / kBK + rp / kBK);
+    int64_t ctas = sms < kStreamKMaxCtas ? sms : kStreamKMaxCtas;
+    if (ctas > total / kStreamKMinSteps) ctas = total / kStreamKMinSteps;
+    return ctas > ntiles ? (int)ctas : 0;
+}
+
+// ctas > 0 (from streamk_ctas): the split launch, with partials and counts
+// from the caller's workspace (counts zeroed by the kernel launched just
+// before); otherwise one CTA per tile.
 cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                            const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
-                           void *y, cudaStream_t stream, int /*num_sms*/, unsigned *err_word) {
+                           void *y, float *partials, unsigned *counts, int ctas, cudaStream_t stream,
+                           unsigned *err_word) {
     if (M > 0x7FFFFFFF || K > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    if (M <= CfgSmall::BT)
-        return launch_cfg<CfgSmall>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream, err_word);
-    return launch_cfg<CfgLarge>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, stream, err_word);
+    if (M <= CfgSmall::BT) {
+        if (ctas > 0)
+            return launch_cfg<CfgSmall, true>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, partials,
+                                              counts, ctas, stream, err_word);
+        return launch_cfg<CfgSmall, false>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, nullptr, nullptr,
+                                           0, stream, err_word);
+    }
+    return launch_cfg<CfgLarge, false>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, nullptr, nullptr, 0,
+                                       stream, err_word);
 }
 
 // Tensor-core LoRA down-projection: see k_lora_down_tc.  split: 0 = the

@@ -36,9 +36,14 @@ namespace {
 #define NF4_GEMV_WARPS 4
 #endif
 constexpr int kGemvWarps = NF4_GEMV_WARPS;
-// resident CTAs per SM the register allocation must allow
+// Resident CTAs per SM the register allocation of the one-token-tile
+// kernel must allow: 5 caps it at 102 registers (it needs 95, no spills), so
+// the 688 tiles of an 11008-row weight run as one wave of 740 slots instead
+// of 1.5 waves of 444 (148 registers): 17.0 -> 16.5 us without LoRA, 18.9
+// -> 18.0 us with r = 16 at one token.  The two-token-tile instantiation
+// spills under that cap and keeps the default.
 #ifndef NF4_GEMV_MINB
-#define NF4_GEMV_MINB 1
+#define NF4_GEMV_MINB 5
 #endif
 // 0 = register lookup table, 1 = shared-memory pair table, 2 = pair table for
 // the first row of each m16 tile and register table for the second
@@ -84,7 +89,7 @@ __device__ __forceinline__ void load_set(const uint8_t *__restrict__ packed, con
 // weights) instead of the per-block register lookup table (lut_lookup4: about
 // three byte permutes per weight, all on the integer pipe).
 template <int kMode, int NT, int MT, int kLutSel>
-__global__ void __launch_bounds__(kGemvWarps * 32, NF4_GEMV_MINB) k_gemv(const __nv_bfloat16 *__restrict__ x, int M, int64_t K,
+__global__ void __launch_bounds__(kGemvWarps * 32, MT == 1 ? NF4_GEMV_MINB : 1) k_gemv(const __nv_bfloat16 *__restrict__ x, int M, int64_t K,
                                                           int64_t N, const uint8_t *__restrict__ packed,
                                                           const uint8_t *__restrict__ q8,
                                                           const float *__restrict__ scales,

@@ -7,7 +7,7 @@ namespace nf4 {
 
 int lora_rp(int r);
 cudaError_t launch_lora_down(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2,
-                             cudaStream_t stream);
+                             unsigned *counts, int ncounts, cudaStream_t stream);
 cudaError_t launch_gemv(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                         const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                         void *y, cudaStream_t stream, int num_sms);
@@ -15,7 +15,11 @@ cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t
                                 unsigned *err, cudaStream_t stream, int split);
 cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                            const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
-                           void *y, cudaStream_t stream, int num_sms, unsigned *err_word);
+                           void *y, float *partials, unsigned *counts, int ctas, cudaStream_t stream,
+                           unsigned *err_word);
+int64_t streamk_partials_bytes();
+int64_t streamk_counts_bytes();
+int streamk_ctas(int64_t M, int64_t K, int64_t N, int rp, int sms);
 
 constexpr int kGemvMaxTokens = 16;
 // Token counts from which decode-size calls take the tcgen05 pipeline with a
@@ -46,22 +50,58 @@ unsigned *device_error_word(cudaError_t *status) {
 // t2 = [t_hi | t_lo | 0 pad] bf16 [M, round_up(2r, 64)], 16-byte aligned rows.
 int64_t lora_workspace_bytes(int64_t M, int r) { return M * (int64_t)lora_rp(r) * 2; }
 
+// Up to 16 tokens the workspace continues (256-byte aligned) with the
+// scratch of the split 16-token pipeline: partial tiles, then arrival
+// counts.  A workspace holding only t (or none, r = 0) runs it unsplit.
+static int64_t partials_offset(int64_t M, int r) {
+    return (lora_workspace_bytes(M, r > 0 ? r : 0) + 255) & ~(int64_t)255;
+}
+int64_t linear_workspace_bytes(int64_t M, int r) {
+    if (M <= kGemvMaxTokens) return partials_offset(M, r) + streamk_partials_bytes() + streamk_counts_bytes();
+    return r > 0 ? lora_workspace_bytes(M, r) : 0;
+}
+
+// The arrival counts of a split launch without an adapter are zeroed by
+// this one-CTA kernel, which keeps the chain of programmatic dependent
+// launches: it waits for the grid before it (the previous call, which may
+// still use the counts), zeroes them and releases the linear.
+__global__ void k_zero_counts(unsigned *counts, int n) {
+    pdl_wait_then_release();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) counts[i] = 0u;
+}
+
 cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
                                const uint8_t *q8, const float *scales, const float *offset, const void *A,
                                const void *B, int r, float scaling, void *y, void *workspace,
-                               cudaStream_t stream, int num_sms, unsigned *err_word) {
+                               int64_t workspace_bytes, cudaStream_t stream, int num_sms, unsigned *err_word) {
     const int rp = r > 0 ? lora_rp(r) : 0;
+    // decode-size M: the warp-MMA GEMV kernels up to NF4_SMALL_M_TC_FROM - 1
+    // tokens, then the tcgen05 pipeline with a 16-token tile, split over the
+    // SMs when the workspace holds its scratch (with an adapter, 8 SMs are
+    // left to the down-projection's cluster, which runs first)
+    const bool gemv = M < NF4_SMALL_M_TC_FROM && M <= kGemvMaxTokens;
+    float *partials = nullptr;
+    unsigned *counts = nullptr;
+    int ctas = 0;
+    if (!gemv && M <= kGemvMaxTokens && workspace != nullptr && workspace_bytes >= linear_workspace_bytes(M, r)) {
+        ctas = streamk_ctas(M, K, N, rp, r > 0 && num_sms > 16 ? num_sms - 8 : num_sms);
+        if (ctas > 0) {
+            partials = reinterpret_cast<float *>(static_cast<char *>(workspace) + partials_offset(M, r));
+            counts = reinterpret_cast<unsigned *>(reinterpret_cast<char *>(partials) + streamk_partials_bytes());
+        }
+    }
+    const int ncounts = ctas > 0 ? (int)((N + 127) / 128) : 0;
+    cudaError_t e = cudaSuccess;
     if (r > 0) {
         // decode-size M: warp-MMA kernel; larger M: tensor-core kernel
-        cudaError_t e = M <= kGemvMaxTokens ? launch_lora_down(x, A, M, K, r, scaling, workspace, stream)
-                                            : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream, 0);
-        if (e != cudaSuccess) return e;
+        e = M <= kGemvMaxTokens ? launch_lora_down(x, A, M, K, r, scaling, workspace, counts, ncounts, stream)
+                                : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream, 0);
+    } else if (ctas > 0) {
+        e = launch_pdl(k_zero_counts, dim3(1), dim3(256), 0, stream, 1, counts, ncounts);
     }
-    // decode-size M: the warp-MMA GEMV kernels up to NF4_SMALL_M_TC_FROM - 1
-    // tokens, then the tcgen05 pipeline with a 16-token tile
-    if (M < NF4_SMALL_M_TC_FROM && M <= kGemvMaxTokens)
-        return launch_gemv(x, (int)M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms);
-    return launch_gemm_tc(x, M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms,
+    if (e != cudaSuccess) return e;
+    if (gemv) return launch_gemv(x, (int)M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms);
+    return launch_gemm_tc(x, M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, partials, counts, ctas, stream,
                           err_word);
 }
 

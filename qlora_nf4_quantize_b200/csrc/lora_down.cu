@@ -37,7 +37,7 @@ template <int kR>
 __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat16 *__restrict__ x,
                                                                const __nv_bfloat16 *__restrict__ A, int64_t M,
                                                                int64_t K, float s, __nv_bfloat16 *__restrict__ t2,
-                                                               int rp) {
+                                                               int rp, unsigned *__restrict__ counts, int ncounts) {
     constexpr int NT = kR / 8;  // n8 tiles
     extern __shared__ float s_dyn[];  // [kDownWarps][NT][4][32] warp partials, then [NT * 128] CTA partial
     auto s_part = reinterpret_cast<float (*)[NT][4][32]>(s_dyn);
@@ -48,6 +48,10 @@ __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat
     pdl_wait_then_release();
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
+    // arrival counts of a split fused linear launched next (its predecessor,
+    // which may still have used them, has completed)
+    if (rank == 0)
+        for (int i = threadIdx.x; i < ncounts; i += kDownWarps * 32) counts[i] = 0u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tq = lane & 3;
     const int64_t ra = g, rb = g + 8;
@@ -118,22 +122,24 @@ __global__ void __launch_bounds__(kDownWarps * 32) k_lora_down(const __nv_bfloat
 
 template <int kR>
 cudaError_t launch_down(cudaStream_t stream, const __nv_bfloat16 *x, const __nv_bfloat16 *A, int64_t M, int64_t K,
-                        float s, __nv_bfloat16 *t2, int rp) {
+                        float s, __nv_bfloat16 *t2, int rp, unsigned *counts, int ncounts) {
     const size_t smem = (size_t)(kDownWarps + 1) * (kR / 8) * 4 * 32 * sizeof(float);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_lora_down<kR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     return launch_pdl(k_lora_down<kR>, dim3(kDownCtas), dim3(kDownWarps * 32), smem, stream, kDownCtas, x, A, M, K,
-                      s, t2, rp);
+                      s, t2, rp, counts, ncounts);
 }
 
 }  // namespace
 
 int lora_rp(int r) { return ((2 * r + 63) / 64) * 64; }
 
+// counts: ncounts arrival counts to zero for a split fused linear launched
+// next (NULL, 0 when there is none).
 cudaError_t launch_lora_down(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2,
-                             cudaStream_t stream) {
+                             unsigned *counts, int ncounts, cudaStream_t stream) {
     if (M > 16) return cudaErrorInvalidValue;  // larger M: launch_lora_down_tc
     const int rp = lora_rp(r);
     auto *xp = static_cast<const __nv_bfloat16 *>(x);
@@ -141,9 +147,9 @@ cudaError_t launch_lora_down(const void *x, const void *A, int64_t M, int64_t K,
     auto *tp = static_cast<__nv_bfloat16 *>(t2);
     cudaError_t e = cudaSuccess;
     switch (r) {
-        case 16: e = launch_down<16>(stream, xp, ap, M, K, s, tp, rp); break;
-        case 32: e = launch_down<32>(stream, xp, ap, M, K, s, tp, rp); break;
-        case 64: e = launch_down<64>(stream, xp, ap, M, K, s, tp, rp); break;
+        case 16: e = launch_down<16>(stream, xp, ap, M, K, s, tp, rp, counts, ncounts); break;
+        case 32: e = launch_down<32>(stream, xp, ap, M, K, s, tp, rp, counts, ncounts); break;
+        case 64: e = launch_down<64>(stream, xp, ap, M, K, s, tp, rp, counts, ncounts); break;
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;

@@ -32,8 +32,9 @@ namespace nf4 {
 cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
                                const uint8_t *q8, const float *scales, const float *offset, const void *A,
                                const void *B, int r, float scaling, void *y, void *workspace,
-                               cudaStream_t stream, int num_sms, unsigned *err_word);
+                               int64_t workspace_bytes, cudaStream_t stream, int num_sms, unsigned *err_word);
 int64_t lora_workspace_bytes(int64_t M, int r);
+int64_t linear_workspace_bytes(int64_t M, int r);
 unsigned *device_error_word(cudaError_t *status);
 nf4_status status_of(cudaError_t e);
 }  // namespace nf4
@@ -97,7 +98,7 @@ extern "C" NF4_API nf4_status nf4_lora_linear_fwd_noalloc(const void *x, int64_t
         if (e == cudaSuccess)
             e = nf4::launch_lora_linear(x, M, K, N, packed, absmax_q, absmax2, offset, lora ? A : nullptr,
                                         lora ? B : nullptr, lora ? r : 0, scaling, y, scratch,
-                                        (cudaStream_t)stream, sms, err);
+                                        (int64_t)NF4_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream, sms, err);
     }
     return nf4::status_of(e);
 }

@@ -85,5 +85,13 @@ def test_workspace_sizes(nf4lib):
     assert nf4lib.nf4_double_quantize_workspace_size(0) == 0
     assert nf4lib.nf4_double_quantize_workspace_size(2048) == 8          # 8 runs -> 1 chunk of 32
     assert nf4lib.nf4_double_quantize_workspace_size(256 * 33) == 16     # 33 runs -> 2 chunks
-    assert nf4lib.nf4_lora_linear_workspace_size(16, 16) == 16 * 64 * 2  # [t_hi | t_lo | pad] rows of 64
+    # up to 16 tokens: [t_hi | t_lo | pad] rows of 64, then (256-byte aligned)
+    # the split pipeline's scratch: 192 CTAs x 2 partial tiles of 16 x 128
+    # fp32, then 192 arrival counts
+    split = 192 * 2 * 16 * 128 * 4 + 192 * 4
+    assert nf4lib.nf4_lora_linear_workspace_size(16, 16) == 16 * 64 * 2 + split
+    assert nf4lib.nf4_lora_linear_workspace_size(3, 16) == 512 + split  # 384 bytes of t, aligned up
+    assert nf4lib.nf4_lora_linear_workspace_size(16, 0) == split
+    assert nf4lib.nf4_lora_linear_workspace_size(17, 0) == 0
+    assert nf4lib.nf4_lora_linear_workspace_size(4096, 0) == 0
     assert nf4lib.nf4_lora_linear_workspace_size(4096, 64) == 4096 * 128 * 2

@@ -164,3 +164,59 @@ def test_gemm_and_gemv_agree_on_shared_rows(nf4lib, cuda_device):
                                      c.scaling)
     nf4lib.nf4_device_status()
     check(y16, y64[:16].float().cpu().numpy())
+
+
+@pytest.mark.parametrize("M,K,N,r,dq", [(9, 1024, 8, 16, True), (12, 512, 2400, 16, False), (16, 512, 2400, 64, True),
+                                        (16, 2048, 640, 32, True), (11, 8192, 1000, 0, True),
+                                        (16, 64, 18936, 32, True), (10, 4096, 11008, 0, True)])
+def test_split_decode_pipeline(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
+    """9 to 16 tokens: the 16-token tensor-core pipeline split over the SMs
+    (full workspace) and unsplit (a workspace holding only t) both match the
+    oracle, and the split result is bitwise the same on every run (each
+    tile's partials are added in CTA order).  Shapes cover one tile split
+    over two CTAs, ranges that start inside the LoRA extension steps, no
+    adapter, and 148 tiles (no split: not more CTAs than tiles)."""
+    c = wl.LinearCase("split", M, K, N, r, 1.25, 57 + M + K + N)
+    W, x, A, B = wl.linear_inputs(c, with_lora=r > 0)
+    st = quantize_on_gpu(nf4lib, W, cuda_device, dq)
+    xd = x.to(cuda_device)
+    dA = None if A is None else A.to(cuda_device)
+    dB = None if B is None else B.to(cuda_device)
+    ref = oracle_linear(oracle_mod, st, x, A, B, r, c.scaling)
+    full = nf4lib.nf4_lora_linear_workspace_size(M, r)
+    t_only = M * ((2 * r + 63) // 64) * 64 * 2
+    assert full > t_only
+    outs = []
+    for ws_bytes in (full, full, t_only, full):
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=cuda_device)
+        outs.append(nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, N, dA, dB,
+                                               c.scaling, workspace=ws))
+    torch.cuda.synchronize()
+    assert nf4lib.nf4_device_status() == 0
+    for y in outs:
+        check(y, ref)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[3])
+
+
+def test_split_decode_pipeline_back_to_back(nf4lib, cuda_device):
+    """Calls of the split pipeline queued back to back on one stream, with
+    and without an adapter, reuse one workspace (its arrival counts are
+    zeroed by the kernel launched before each linear): every output equals
+    the same call run alone."""
+    c = wl.LinearCase("split b2b", 16, 2048, 4096, 16, 2.0, 93)
+    W, x, A, B = wl.linear_inputs(c)
+    st = quantize_on_gpu(nf4lib, W, cuda_device)
+    xd, Ad, Bd = x.to(cuda_device), A.to(cuda_device), B.to(cuda_device)
+    ws = torch.empty(nf4lib.nf4_lora_linear_workspace_size(16, 16), dtype=torch.uint8, device=cuda_device)
+    alone = [nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, a, b, c.scaling,
+                                        workspace=ws) for a, b in ((Ad, Bd), (None, None))]
+    torch.cuda.synchronize()
+    ys = []
+    for i in range(12):
+        a, b = ((Ad, Bd), (None, None))[i % 2]
+        ys.append(nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, a, b, c.scaling,
+                                             workspace=ws))
+    torch.cuda.synchronize()
+    assert nf4lib.nf4_device_status() == 0
+    for i, y in enumerate(ys):
+        assert torch.equal(y, alone[i % 2]), i
