@@ -7,10 +7,14 @@
 // binary32 value to nearest even.
 //
 // HBM-bound streaming kernel.  A warp handles kSeg * 256 consecutive elements
-// per iteration as kSeg segments of 256: in segment j lane l owns the 8
-// elements starting at 256 j + 8 l, i.e. 4 packed bytes (one 32-bit load; the
-// warp's load is 128 contiguous bytes) and 16 output bytes for bf16 (one
-// 128-bit store; the warp's store is 512 contiguous bytes).  All kSeg loads of
+// per iteration as kSeg segments of 256.  bf16 output: in segment j lane l
+// owns the 8 elements starting at 256 j + 8 l, i.e. 4 packed bytes (one
+// 32-bit load; the warp's load is 128 contiguous bytes) and 16 output bytes
+// (one 128-bit store; the warp's store is 512 contiguous bytes).  fp32
+// output: lane l owns elements 256 j + 4 l .. + 3 and 256 j + 128 + 4 l .. + 3
+// (two 16-bit loads), so each of its two 128-bit stores is 512 contiguous
+// bytes per warp; 8 consecutive elements per lane would make every store
+// instruction write every other 16 bytes (4096 x 4096: 19.3 -> 14.7 us).  All kSeg loads of
 // a lane (codes and block constants) are issued before any arithmetic; up to
 // 8 CTAs of 256 threads per SM are resident, and the grid may hold more (see
 // launch_mode for the shape).  Eight segments per iteration (a 4096 x 4096
@@ -56,7 +60,49 @@ __global__ void __launch_bounds__(kDeqThreads, 2048 / kDeqThreads) k_dequantize(
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (kDeqThreads / 32);
     const int64_t nfull = n / kWarpElems;  // warp iterations with no tail
-    for (int64_t c = (int64_t)blockIdx.x * (kDeqThreads / 32) + (threadIdx.x >> 5); c < nfull; c += warps) {
+    for (int64_t c = (int64_t)blockIdx.x * (kDeqThreads / 32) + (threadIdx.x >> 5); c < nfull && !kBf16Out;
+         c += warps) {
+        // fp32 output: in segment j lane l owns elements 4l..4l+3 and
+        // 128+4l..128+4l+3, so each 16-byte store of the warp covers 512
+        // contiguous bytes (with 8 consecutive elements per lane a store
+        // instruction would write every other 16 bytes)
+        const int64_t seg0 = c * kWarpElems;
+        uint32_t ph[kSeg][2];
+        ScaleRaw sr[kSeg][2];
+#pragma unroll
+        for (int j = 0; j < kSeg; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                ph[j][h] = __ldg(reinterpret_cast<const uint16_t *>(packed) + ((seg0 + 256 * j + 128 * h + 4 * lane) >> 2));
+        const float c2 = (kMode == 2) ? 0.0f : __ldg(scales + (seg0 >> 14));
+#pragma unroll
+        for (int j = 0; j < kSeg; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t blk = (seg0 + 256 * j + 128 * h + 4 * lane) >> 6;
+                if constexpr (kMode == 2) {
+                    sr[j][h].v = __ldg(scales + blk);
+                } else {
+                    sr[j][h].q8 = __ldg(q8 + blk);
+                    sr[j][h].v = c2;
+                }
+            }
+#pragma unroll
+        for (int j = 0; j < kSeg; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float scj = block_scale_finish<kMode>(sr[j][h], mu);
+                const uint32_t w = ph[j][h];  // byte 0 = elements 0, 1; byte 1 = elements 2, 3
+                float4 v;
+                v.x = __fmul_rn(s_q[(w >> 4) & 15u], scj);
+                v.y = __fmul_rn(s_q[w & 15u], scj);
+                v.z = __fmul_rn(s_q[(w >> 12) & 15u], scj);
+                v.w = __fmul_rn(s_q[(w >> 8) & 15u], scj);
+                *reinterpret_cast<float4 *>(static_cast<float *>(out) + seg0 + 256 * j + 128 * h + 4 * lane) = v;
+            }
+    }
+    for (int64_t c = (int64_t)blockIdx.x * (kDeqThreads / 32) + (threadIdx.x >> 5); c < nfull && kBf16Out;
+         c += warps) {
         const int64_t base = c * kWarpElems + 8 * lane;
         uint32_t p[kSeg];
         ScaleRaw sr[kSeg];
