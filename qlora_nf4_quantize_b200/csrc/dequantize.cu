@@ -28,20 +28,14 @@ namespace {
 
 constexpr int kDeqThreads = 256;
 
-template <int kMode, bool kBf16Out>
-__device__ __forceinline__ void store8(void *out, int64_t e0, const float v[8]) {
-    if constexpr (kBf16Out) {
-        uint4 o;
-        o.x = pack_bf16x2(v[0], v[1]);
-        o.y = pack_bf16x2(v[2], v[3]);
-        o.z = pack_bf16x2(v[4], v[5]);
-        o.w = pack_bf16x2(v[6], v[7]);
-        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + e0) = o;
-    } else {
-        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + e0);
-        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-    }
+// 8 consecutive bf16 outputs as one 16-byte store.
+__device__ __forceinline__ void store8_bf16(void *out, int64_t e0, const float v[8]) {
+    uint4 o;
+    o.x = pack_bf16x2(v[0], v[1]);
+    o.y = pack_bf16x2(v[2], v[3]);
+    o.z = pack_bf16x2(v[4], v[5]);
+    o.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + e0) = o;
 }
 
 template <int kMode, bool kBf16Out, int kSeg>
@@ -131,7 +125,7 @@ __global__ void __launch_bounds__(kDeqThreads, 2048 / kDeqThreads) k_dequantize(
                 v[2 * b] = __fmul_rn(s_q[byte >> 4], scj);       // element 2b: high nibble
                 v[2 * b + 1] = __fmul_rn(s_q[byte & 15u], scj);  // element 2b+1: low nibble
             }
-            store8<kMode, kBf16Out>(out, base + 256 * j, v);
+            store8_bf16(out, base + 256 * j, v);
         }
     }
     // tail: elements [nfull * kWarpElems, n), one element per thread
