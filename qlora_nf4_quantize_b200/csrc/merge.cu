@@ -32,9 +32,16 @@ constexpr int kMergeCols = 256;
 constexpr int kMergeRows = 64;
 constexpr int kMergeThreads = 256;
 constexpr int kMergeMaxR = 64;
+// sB holds B transposed, [j][row] with rows padded to 68 floats: a warp's 8
+// rows at one j are two 16-byte broadcast loads (one wavefront each, against
+// 8 for 8 scalar loads), and the staging writes, 32 consecutive j of one row,
+// hit 8 banks 4 ways.
+constexpr int kMergeBStride = kMergeRows + 4;
 
 template <int kMode>
-__global__ void __launch_bounds__(kMergeThreads)
+// Two CTAs per SM (128 registers): the epilogue's loads issued before the
+// fma chains need ~150 registers, and one CTA per SM was 35 % slower.
+__global__ void __launch_bounds__(kMergeThreads, 2)
     k_merge_requantize(const uint8_t *packed, const uint8_t *__restrict__ q8, const float *scales,
                        const float *__restrict__ offset, int64_t N, int64_t K,
                        const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ B, int r, float s,
@@ -43,7 +50,7 @@ __global__ void __launch_bounds__(kMergeThreads)
     // sA[j][h][l][c] = A[j, k0 + 8 l + 4 h + c]: lane l's two float4 of row j
     // sit 512 bytes apart, so consecutive lanes read consecutive 16 bytes
     float *sA = s_dyn;                      // [r][2][32][4]
-    float *sB = s_dyn + r * kMergeCols;     // [64][r]
+    float *sB = s_dyn + r * kMergeCols;     // [r][kMergeBStride], row index fastest
     __shared__ float s_t[16];
     __shared__ uint32_t s_cell[kCellTable];
     __shared__ float s_lv[16];
@@ -58,13 +65,34 @@ __global__ void __launch_bounds__(kMergeThreads)
     for (int i = threadIdx.x; i < kMergeRows * r; i += kMergeThreads) {
         const int row = i / r, j = i % r;
         const int64_t n = n0 + row;
-        sB[i] = n < N ? __bfloat162float(B[n * r + j]) : 0.0f;
+        sB[j * kMergeBStride + row] = n < N ? __bfloat162float(B[n * r + j]) : 0.0f;
     }
     if (threadIdx.x < 16) s_lv[threadIdx.x] = c_levels[threadIdx.x];
     build_code_tables(s_t, s_cell);  // (synchronises the CTA: sA, sB, s_lv ready too)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
+
+    // The codes and block-constant operands of this thread's 8 groups are
+    // loaded before the fma chains, so their latency is hidden behind them
+    // (each group's bytes are still read before this thread writes them).
+    const int64_t k = k0 + 8 * lane;
+    const bool kvalid = k < K;  // K % 64 == 0: a group of 8 is all in or all out
+    uint32_t codes_in[8];
+    ScaleRaw sraw[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t n = n0 + 8 * warp + i;
+        const int64_t e = n * K + k;
+        if (kvalid && n < N) {
+            codes_in[i] = __ldg(reinterpret_cast<const uint32_t *>(packed + (e >> 1)));
+            sraw[i] = block_scale_load<kMode>(q8, scales, e >> 6);
+        } else {
+            codes_in[i] = 0x77777777u;
+            sraw[i].q8 = 0u;
+            sraw[i].v = 0.0f;
+        }
+    }
 
     // d[i][c]: row 8 warp + i, column 8 lane + c of the tile
     float d[8][8];
@@ -73,37 +101,30 @@ __global__ void __launch_bounds__(kMergeThreads)
 #pragma unroll
         for (int c = 0; c < 8; ++c) d[i][c] = 0.0f;
     const float4 *a_lane = reinterpret_cast<const float4 *>(sA) + lane;
-    const float *b_rows = sB + (8 * warp) * r;
+    const float4 *b_warp = reinterpret_cast<const float4 *>(sB + 8 * warp);
 #pragma unroll 2
     for (int j = 0; j < r; ++j) {
         const float4 a0 = a_lane[j * 64], a1 = a_lane[j * 64 + 32];
+        const float4 b0 = b_warp[j * (kMergeBStride / 4)], b1 = b_warp[j * (kMergeBStride / 4) + 1];
         const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float b = b_rows[i * r + j];
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) d[i][c] = __fmaf_rn(b, a[c], d[i][c]);
-        }
+            for (int c = 0; c < 8; ++c) d[i][c] = __fmaf_rn(b[i], a[c], d[i][c]);
     }
 
-    const int64_t k = k0 + 8 * lane;
-    const bool kvalid = k < K;  // K % 64 == 0: a group of 8 is all in or all out
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t n = n0 + 8 * warp + i;
         const bool valid = kvalid && n < N;
         const int64_t e = n * K + k;  // first element of this thread's group
-        uint32_t codes_in = 0x77777777u;
-        float c = 0.0f;
-        if (valid) {
-            codes_in = __ldg(reinterpret_cast<const uint32_t *>(packed + (e >> 1)));
-            c = block_scale<kMode>(q8, scales, mu, e >> 6);
-        }
+        const float c = valid ? block_scale_finish<kMode>(sraw[i], mu) : 0.0f;
         float w[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
             // byte t/2 of the group; element 2j in the high nibble
-            const uint32_t code = (codes_in >> (8 * (t >> 1) + ((t & 1) ? 0 : 4))) & 15u;
+            const uint32_t code = (codes_in[i] >> (8 * (t >> 1) + ((t & 1) ? 0 : 4))) & 15u;
             const float wt = __fmul_rn(s_lv[code], c);
             w[t] = __fmaf_rn(s, d[i][t], wt);
         }
@@ -125,7 +146,7 @@ template <int kMode>
 cudaError_t launch_mode(const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
                         int64_t N, int64_t K, const __nv_bfloat16 *A, const __nv_bfloat16 *B, int r, float s,
                         uint8_t *packed_out, float *absmax_out, cudaStream_t stream) {
-    const size_t smem = (size_t)(r * kMergeCols + kMergeRows * r) * sizeof(float);
+    const size_t smem = (size_t)(r * kMergeCols + r * kMergeBStride) * sizeof(float);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_merge_requantize<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
