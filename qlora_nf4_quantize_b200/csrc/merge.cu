@@ -14,8 +14,8 @@
 // accumulation order is not specified, and would not reproduce it.
 //
 // Layout of the work: a CTA owns a tile of 64 rows x 256 columns of W.  A's
-// 256 columns (r x 256, fp32) and B's 64 rows (64 x r, fp32) are staged in
-// shared memory once.  Warp w owns rows 8 w .. 8 w + 7 of the tile and lane l
+// 256 columns (r x 256, fp32) and B's 64 rows (transposed, r x 64, fp32) are
+// staged in shared memory once.  Warp w owns rows 8 w .. 8 w + 7 of the tile and lane l
 // columns 8 l .. 8 l + 7, so every value of A read from shared memory feeds 8
 // rows (64 fma per 2 vector loads and 8 broadcast loads); the 8 lanes
 // 8 m .. 8 m + 7 own one 64-block of each row, whose absmax is a 3-step
@@ -40,7 +40,7 @@ constexpr int kMergeBStride = kMergeRows + 4;
 
 template <int kMode>
 // Two CTAs per SM (128 registers): the epilogue's loads issued before the
-// fma chains need ~150 registers, and one CTA per SM was 35 % slower.
+// fma chains need ~150 registers, and one CTA per SM was about 40 % slower.
 __global__ void __launch_bounds__(kMergeThreads, 2)
     k_merge_requantize(const uint8_t *packed, const uint8_t *__restrict__ q8, const float *scales,
                        const float *__restrict__ offset, int64_t N, int64_t K,
