@@ -24,9 +24,10 @@ int streamk_ctas(int64_t M, int64_t K, int64_t N, int rp, int sms);
 constexpr int kGemvMaxTokens = 16;
 // Token counts from which decode-size calls take the tcgen05 pipeline with a
 // 16-token tile instead of the warp-MMA GEMV kernels: that pipeline takes
-// the same time for any count up to 16 (25.7 us without LoRA on an 11008 x
-// 4096 weight), the warp-MMA kernels grow with it (17.0 us at 1 token, 21.8
-// at 8, 27.5 at 12, 30.3 at 16: above 8 tokens they need two token tiles).
+// the same time for any count up to 16 (split over the SMs, 25.1 us without
+// LoRA on an 11008 x 4096 weight), the warp-MMA kernels grow with it (16.5
+// us at 1 token, 21.7 at 8, 27.5 at 12, 30.3 at 16: above 8 tokens they need
+// two token tiles).
 #ifndef NF4_SMALL_M_TC_FROM
 #define NF4_SMALL_M_TC_FROM 9
 #endif
