@@ -1,5 +1,7 @@
 // gemv.cu -- K4: fused NF4-dequantizing linear for small token counts
-// (M <= 16), y = x W~^T + [t_hi | t_lo] [B | B]^T.
+// (M <= 16; the dispatcher, linear.cu, sends 9 to 16 tokens to the
+// tensor-core pipeline's 16-token tile instead), y = x W~^T + [t_hi | t_lo]
+// [B | B]^T.
 //
 // "QLoRA: Mathematical Foundations ...", section "Forward Pass Computation":
 // the weight is dequantized on the fly into registers and never written to
