@@ -27,6 +27,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import time
@@ -155,17 +156,45 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def code_digest(kernel_file):
+    """First 16 hex digits of a sha256 over the kernel's source file and the
+    local headers it includes (recursively, in include order), each with its
+    comments removed and its white space collapsed: an edit to comments
+    keeps a recorded capture valid, any change to the code voids it."""
+    csrc = os.path.join(ROOT, "qlora_nf4_quantize_b200", "csrc")
+    order, seen = [], set()
+
+    def visit(name):
+        if name in seen:
+            return
+        seen.add(name)
+        order.append(name)
+        with open(os.path.join(csrc, name)) as f:
+            text = f.read()
+        for inc in re.findall(r'#include\s+"([^"/]+)"', text):
+            if os.path.exists(os.path.join(csrc, inc)):
+                visit(inc)
+
+    visit(kernel_file)
+    h = hashlib.sha256()
+    for name in order:
+        with open(os.path.join(csrc, name)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(name.encode() + b"\0" + " ".join(src.split()).encode() + b"\0")
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(kernel_file):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current source of the kernel (else None)."""
+    the current code of the kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
-        with open(os.path.join(ROOT, "qlora_nf4_quantize_b200", "csrc", kernel_file), "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()[:16]
         e = rec.get(kernel_file)
-        if e and e.get("source_sha256_16") == digest:
+        if e and e.get("code_sha256_16") == code_digest(kernel_file):
             return e.get("dram_bytes_per_launch")
     except (OSError, ValueError):
         pass

@@ -10,23 +10,25 @@
 //
 // One CTA computes a 128 (weight rows) x 256 (tokens) tile of y^T:
 //   MMA  D[n, m] += A[n, k] * X[m, k],   M_mma = 128, N_mma = 256, K = 16
-//   A = W~ (bf16) lives in tensor memory: two dequant warpgroups turn the
+//   A = W~ (bf16) lives in tensor memory: three dequant warpgroups turn the
 //       packed nibbles of a 64-wide k-step into bf16 in registers (one scale
 //       and one register lookup table per 64-block per thread, see
 //       mma_util.cuh) and store them with tcgen05.st; no shared memory is
 //       used for the weight.
 //   X = x tile (256 tokens x 64 k, bf16) brought in by TMA with 128-byte
-//       swizzle into a 4-stage shared-memory ring.
+//       swizzle into a 6-stage shared-memory ring.
 //   D = fp32 accumulators in tensor memory (256 columns).
 // After the K/64 weight steps the same pipeline runs RP/64 extension steps in
 // which the warpgroups copy rows of [B | B | 0] into tensor memory and TMA
 // brings tiles of the [t_hi | t_lo | 0] workspace: the LoRA term is summed by
 // the same MMAs into the same accumulators.
 //
-// Warp roles (12 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
-// MMA issuer (one elected thread), warps 4..11 = two dequant warpgroups
-// (warpgroup h produces the k-steps with index = h mod 2) and, at the end,
-// the epilogue (tcgen05.ld, bf16 conversion, stores of y).
+// Warp roles (16 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
+// MMA issuer (one elected lane of the converged warp), warps 4..15 = three
+// dequant warpgroups (warpgroup h produces the k-steps with index = h mod 3)
+// and, at the end, the epilogue (tcgen05.ld, bf16 conversion, one TMA store
+// of y).  The same pipeline with a 16-token tile serves decode calls of 9 to
+// 16 tokens, split over the SMs (stream-K, see TmemPlan below).
 //
 // Every mbarrier wait is bounded (about one second of %globaltimer): on
 // expiry the waiter raises a CTA-wide abort flag and the device error word,
@@ -72,9 +74,9 @@ constexpr uint32_t pow2_at_least(uint32_t v) {
 
 // Token tile BT (MMA N), pipeline depth and dequant warpgroups of one
 // instantiation: BT = 256 for the large-M GEMM; BT = 16 serves 9 to 16 tokens
-// (one 128-row tile per CTA, a rate bound by the dequantization, the same for
-// any token count up to 16; below 9 tokens the warp-MMA GEMV kernels are
-// faster).
+// (a rate bound by the dequantization, the same for any token count up to 16;
+// below 9 tokens the warp-MMA GEMV kernels are faster), normally split over
+// the SMs.
 constexpr uint32_t AccColsFor(int bt) { return bt < 32 ? 32u : (uint32_t)bt; }
 
 template <int BT_, int STAGES_, int WG_, int SUB_>
