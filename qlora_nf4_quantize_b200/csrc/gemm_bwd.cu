@@ -14,7 +14,7 @@
 //   D_h[m, k] += G[m, n] * W~[n, k],  M_mma = 128, N_mma = 256, K = 16
 //   G  = g tile (256 tokens x 64 n) brought by TMA with 128-byte swizzle,
 //        a K-major operand;
-//   W~ = the dequantized weight tile (64 n x 256 k) written by two dequant
+//   W~ = the dequantized weight tile (64 n x 256 k) written by the dequant
 //        warpgroups into shared memory in its own row layout, as an MN-major
 //        operand (instruction descriptor transpose bit): 128-byte swizzle
 //        atoms of 8 rows n x 64 k, the four 64-k atoms of a row group 8 KB
