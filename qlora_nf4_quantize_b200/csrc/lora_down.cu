@@ -20,7 +20,9 @@
 // distributed shared memory, so the result is independent of timing.  The
 // kernel releases the fused linear that follows (programmatic dependent
 // launch) as soon as its own predecessor has completed: the linear starts
-// streaming the weight at once and waits for t only where it reads it.
+// streaming the weight at once and waits for t only where it reads it.  For a
+// linear split over the SMs (9 to 16 tokens) it also zeroes that linear's
+// per-tile arrival counts in the caller's workspace.
 #include <cooperative_groups.h>
 
 #include "mma_util.cuh"
