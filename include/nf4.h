@@ -205,6 +205,10 @@ NF4_API nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int6
  *          scratch (nf4_lora_linear_workspace_size(M, r) <= 4 MiB there).
  *   The first call on a device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
+ *   The address is cached for the life of the process's context on that
+ *   device: after cudaDeviceReset (or anything else that destroys the
+ *   primary context) this entry point must not be called again in the
+ *   same process.
  *   All calls on a device share the array: calls whose kernels may overlap on
  *   the GPU (unordered streams) race and give undefined results.  Nothing has
  *   to be cleared between calls.

@@ -39,6 +39,10 @@ GEMV_CASES = [LinearCase(f"decode GEMV T={T} W 11008x4096 r=16", T, 4096, 11008,
               for T in (1, 4, 16)]
 GEMM_TRAIN = LinearCase("training GEMM x 4096x4096, W 14336x4096, r=64", 4096, 4096, 14336, 64, 0.25, 4)
 GEMM_70B_MLP = LinearCase("70B MLP GEMM x 2048x8192, W 28672x8192, r=16", 2048, 8192, 28672, 16, 2.0, 5)
+# Two more linears of the 8B-shaped decoder layer at the training token count
+# (the layer's longest contraction and its narrowest output)
+GEMM_DOWN_PROJ = LinearCase("down_proj GEMM x 4096x14336, W 4096x14336, r=64", 4096, 14336, 4096, 64, 0.25, 6)
+GEMM_K_PROJ = LinearCase("k_proj GEMM x 4096x4096, W 1024x4096, r=64", 4096, 4096, 1024, 64, 0.25, 7)
 
 # One decoder layer of the 8B-shaped model: (name, out_features N, in_features K)
 LAYER_8B = [("q_proj", 4096, 4096), ("k_proj", 1024, 4096), ("v_proj", 1024, 4096),

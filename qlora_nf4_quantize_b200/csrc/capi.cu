@@ -51,16 +51,21 @@ nf4_status cuda_status(cudaError_t e) {
 
 bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
 
+// SM count of the current device, cached per device (atomic entries: host
+// threads making their first calls at the same time write the same value).
 int sm_count(cudaError_t *status) {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];
     int dev = 0;
     *status = cudaGetDevice(&dev);
     if (*status != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    if (dev >= 0 && dev < 64) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int v = 0;
     *status = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
     if (*status != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64) cached[dev] = v;
+    if (dev >= 0 && dev < 64) cached[dev].store(v, std::memory_order_relaxed);
     return v;
 }
 

@@ -1,6 +1,8 @@
 // linear.cu -- dispatch of the fused frozen-base LoRA linear, its workspace
 // layout, and the device error word written by kernels whose bounded waits
 // expire.
+#include <mutex>
+
 #include "nf4_device.cuh"
 
 namespace nf4 {
@@ -32,20 +34,31 @@ constexpr int kGemvMaxTokens = 16;
 #define NF4_SMALL_M_TC_FROM 9
 #endif
 
-// Device error word: one per device, cleared by nf4_device_status().
+// Device error word: one per device, cleared by nf4_device_status().  Its
+// device address is looked up once per device (with that device current)
+// and cached for the life of the process's context on that device; the
+// cache is guarded so that host threads making their first calls at the
+// same time do not race on it.
 static __device__ unsigned g_error_word;
 
 unsigned *device_error_word(cudaError_t *status) {
+    static std::mutex mutex;
     static unsigned *cached[64] = {nullptr};
     int dev = 0;
     *status = cudaGetDevice(&dev);
     if (*status != cudaSuccess) return nullptr;
-    if (dev >= 0 && dev < 64 && cached[dev] != nullptr) return cached[dev];
-    void *p = nullptr;
-    *status = cudaGetSymbolAddress(&p, g_error_word);
-    if (*status != cudaSuccess) return nullptr;
-    if (dev >= 0 && dev < 64) cached[dev] = static_cast<unsigned *>(p);
-    return static_cast<unsigned *>(p);
+    if (dev < 0 || dev >= 64) {
+        *status = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mutex);
+    if (cached[dev] == nullptr) {
+        void *p = nullptr;
+        *status = cudaGetSymbolAddress(&p, g_error_word);
+        if (*status != cudaSuccess) return nullptr;
+        cached[dev] = static_cast<unsigned *>(p);
+    }
+    return cached[dev];
 }
 
 // t2 = [t_hi | t_lo | 0 pad] bf16 [M, round_up(2r, 64)], 16-byte aligned rows.

@@ -62,15 +62,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
     return ok != 0;
 }
 
-// Bounded wait: true when the phase completed; false after the time limit
-// (abort raised) or when another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err) {
+// Bounded wait: true when the phase completed; false after limit_ns of
+// %globaltimer (abort raised, bit 0 of the error word set) or when another
+// role already aborted.  Every kernel waits with the default limit; the
+// failure-detection self-test passes a short one.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
             *abort = 1;
             atomicOr(err, 1u);
             return false;

@@ -1,8 +1,9 @@
 // selftest.cu -- exercises the bounded-wait expiry path on the GPU without a
-// fault: one thread waits on an mbarrier that nothing arrives on, gives up
-// after the caller's limit, raises the device error word and returns, exactly
-// as the fused kernels do when a wait expires.  The pages have no counterpart;
-// this is the library's failure-detection check.
+// fault: one thread runs the kernels' own bounded wait (mbar_wait) on an
+// mbarrier that nothing arrives on, with the caller's limit instead of the
+// default second; it gives up, raises the device error word and returns, the
+// path every fused kernel takes when one of its waits expires.  The pages
+// have no counterpart; this is the library's failure-detection check.
 #include "mbarrier.cuh"
 
 namespace nf4 {
@@ -13,16 +14,15 @@ namespace {
 
 __global__ void k_selftest_wait(unsigned long long limit_ns, unsigned *err) {
     __shared__ uint64_t bar;
+    __shared__ int abort;
     if (threadIdx.x != 0) return;
+    abort = 0;
     mbar_init(&bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    const unsigned long long t0 = global_ns();
-    while (!mbar_try_wait_sleep(&bar, 0)) {  // phase 0 never completes
-        if (global_ns() - t0 > limit_ns) {
-            atomicOr(err, 1u);
-            return;
-        }
-    }
+    // the kernels' own bounded wait (mbarrier.cuh), on a phase that never
+    // completes: it gives up after limit_ns, raises the abort flag and the
+    // device error word, and returns false
+    mbar_wait(&bar, 0, &abort, err, limit_ns);
 }
 
 }  // namespace

@@ -83,3 +83,46 @@ def rel_error_stats(y, ref):
 
 MATMUL_MAX_REL = 1e-2
 MATMUL_MEAN_REL = 2e-3
+
+
+# ---------------------------------------------------------------- output guards
+# compute-sanitizer is not available where the GPU tests run, so every output
+# buffer of a GPU parity test sits between two poisoned guard regions: a write
+# past either end of the buffer changes a guard byte and fails the test.
+GUARD_BYTES = 4096
+GUARD_FILL = 0xA5
+
+
+def guarded(shape, dtype, device, fill=None):
+    """A tensor of `shape` and `dtype` on `device` placed between two
+    GUARD_BYTES regions filled with GUARD_FILL (16-byte alignment kept).
+    ``fill`` sets the tensor's own contents (default: the poison bytes too,
+    so an output element the call forgets to write also shows up as a
+    mismatch).  check_guards() verifies the guards after the call."""
+    import math
+
+    import torch
+    shape = (shape,) if isinstance(shape, int) else tuple(shape)
+    n = math.prod(shape)
+    nbytes = n * torch.empty(0, dtype=dtype).element_size()
+    raw = torch.full((2 * GUARD_BYTES + nbytes,), GUARD_FILL, dtype=torch.uint8, device=device)
+    t = raw[GUARD_BYTES:GUARD_BYTES + nbytes].view(dtype).view(shape)
+    if fill is not None:
+        t.fill_(fill)
+    t._nf4_guard = (raw, nbytes)
+    return t
+
+
+def check_guards(*tensors):
+    """Assert the guard regions around each guarded() tensor are intact."""
+    import torch
+    for i, t in enumerate(tensors):
+        if t is None:
+            continue
+        raw, nbytes = t._nf4_guard
+        head = raw[:GUARD_BYTES]
+        tail = raw[GUARD_BYTES + nbytes:]
+        bad_head = torch.nonzero(head != GUARD_FILL)
+        bad_tail = torch.nonzero(tail != GUARD_FILL)
+        assert bad_head.numel() == 0, f"buffer {i}: write before its start at byte {int(bad_head[-1]) - GUARD_BYTES}"
+        assert bad_tail.numel() == 0, f"buffer {i}: write past its end at byte +{int(bad_tail[0])}"

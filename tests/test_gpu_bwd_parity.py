@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import nf4_workloads as wl
-from conftest import MATMUL_MAX_REL, MATMUL_MEAN_REL, rel_error_stats
+from conftest import MATMUL_MAX_REL, MATMUL_MEAN_REL, check_guards, guarded, rel_error_stats
 
 pytestmark = pytest.mark.gpu
 
@@ -34,9 +34,15 @@ def inputs(M, K, N, r, seed, dq=True):
 def run(nf4lib, oracle_mod, dev, M, K, N, r, seed, dq=True, rows=None, want=("dx", "dA", "dB")):
     c, W, x, A, B, dy = inputs(M, K, N, r, seed, dq)
     st = nf4lib.quantize_weight(W.to(dev), double_quant=dq)
+    dx = guarded((M, K), torch.bfloat16, dev) if "dx" in want else None
+    dA = guarded((r, K), torch.float32, dev) if "dA" in want else None
+    dB = guarded((N, r), torch.float32, dev) if "dB" in want else None
+    ws = guarded(max(16, nf4lib.nf4_lora_linear_bwd_workspace_size(M, N, K, r)), torch.uint8, dev)
     dx, dA, dB = nf4lib.nf4_lora_linear_bwd(dy.to(dev), x.to(dev), st.packed, st.absmax_q, st.absmax2, st.offset, K,
-                                            A.to(dev), B.to(dev), c.scaling, want=want)
-    torch.cuda.synchronize()
+                                            A.to(dev), B.to(dev), c.scaling, want=want, dx=dx, dA=dA, dB=dB,
+                                            workspace=ws)
+    nf4lib.nf4_device_status()
+    check_guards(dx, dA, dB, ws)
     packed = st.packed.cpu().numpy()
     q8 = None if st.absmax_q is None else st.absmax_q.cpu().numpy()
     sc = st.absmax2.cpu().numpy()
@@ -60,9 +66,11 @@ def test_bwd_dx_only_without_adapter(nf4lib, oracle_mod, cuda_device):
     M, K, N = 130, 384, 200
     c, W, x, A, B, dy = inputs(M, K, N, 16, 5)
     st = nf4lib.quantize_weight(W.to(cuda_device))
+    dx = guarded((M, K), torch.bfloat16, cuda_device)
     dx, dA, dB = nf4lib.nf4_lora_linear_bwd(dy.to(cuda_device), None, st.packed, st.absmax_q, st.absmax2, st.offset,
-                                            K, want=("dx",))
-    torch.cuda.synchronize()
+                                            K, want=("dx",), dx=dx)
+    nf4lib.nf4_device_status()
+    check_guards(dx)
     assert dA is None and dB is None
     wb = nf4lib.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, N * K).view(N, K)
     ref = torch.matmul(dy.to(cuda_device).float(), wb.float())  # library routine on the dequantized weight

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import nf4_workloads as wl
-from conftest import MATMUL_MAX_REL, MATMUL_MEAN_REL, rel_error_stats
+from conftest import MATMUL_MAX_REL, MATMUL_MEAN_REL, check_guards, guarded, rel_error_stats
 
 pytestmark = pytest.mark.gpu
 
@@ -20,6 +20,23 @@ def u16(t: torch.Tensor) -> np.ndarray:
 
 def quantize_on_gpu(q, W: torch.Tensor, dev, dq=True):
     return q.quantize_weight(W.to(dev), double_quant=dq)
+
+
+def linear(q, x, st, N, A=None, B=None, s=1.0, ws_bytes=None):
+    """nf4_lora_linear_fwd with its output and workspace between poisoned
+    guard regions (checked after the call); ws_bytes overrides the
+    workspace size the call is given."""
+    M = x.shape[0]
+    r = 0 if A is None else A.shape[0]
+    dev = x.device
+    y = guarded((M, N), torch.bfloat16, dev)
+    if ws_bytes is None:
+        ws_bytes = q.nf4_lora_linear_workspace_size(M, r)
+    ws = guarded(ws_bytes, torch.uint8, dev) if ws_bytes > 0 else None
+    q.nf4_lora_linear_fwd(x, st.packed, st.absmax_q, st.absmax2, st.offset, N, A, B, s, y=y, workspace=ws)
+    q.nf4_device_status()
+    check_guards(y, ws)
+    return y
 
 
 def oracle_linear(oracle_mod, st, x, A, B, r, s, rows=None):
@@ -43,8 +60,7 @@ def check(y: torch.Tensor, ref: np.ndarray):
 def test_decode_gemv_full_size(nf4lib, oracle_mod, cuda_device, case):
     W, x, A, B = wl.linear_inputs(case)
     st = quantize_on_gpu(nf4lib, W, cuda_device)
-    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, case.N,
-                                   A.to(cuda_device), B.to(cuda_device), case.scaling)
+    y = linear(nf4lib, x.to(cuda_device), st, case.N, A.to(cuda_device), B.to(cuda_device), case.scaling)
     torch.cuda.synchronize()
     check(y, oracle_linear(oracle_mod, st, x, A, B, case.r, case.scaling))
 
@@ -59,8 +75,7 @@ def test_gemv_ragged_shapes(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
     st = quantize_on_gpu(nf4lib, W, cuda_device, dq)
     dA = None if A is None else A.to(cuda_device)
     dB = None if B is None else B.to(cuda_device)
-    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, N, dA, dB,
-                                   c.scaling)
+    y = linear(nf4lib, x.to(cuda_device), st, N, dA, dB, c.scaling)
     torch.cuda.synchronize()
     check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
 
@@ -73,8 +88,7 @@ def test_linear_double_quant_without_centring(nf4lib, oracle_mod, cuda_device, M
     W, x, A, B = wl.linear_inputs(c)
     st = nf4lib.quantize_weight(W.to(cuda_device), centre=False)
     assert st.offset is None
-    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, N,
-                                   A.to(cuda_device), B.to(cuda_device), c.scaling)
+    y = linear(nf4lib, x.to(cuda_device), st, N, A.to(cuda_device), B.to(cuda_device), c.scaling)
     torch.cuda.synchronize()
     check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
 
@@ -84,7 +98,7 @@ def test_gemv_without_lora_equals_matmul_on_dequantized(nf4lib, cuda_device):
     W, x, _, _ = wl.linear_inputs(c, with_lora=False)
     st = quantize_on_gpu(nf4lib, W, cuda_device)
     xd = x.to(cuda_device)
-    y = nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N)
+    y = linear(nf4lib, xd, st, c.N)
     wb = nf4lib.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N * c.K).view(c.N, c.K)
     ref = torch.matmul(xd.float(), wb.float().t())
     torch.cuda.synchronize()
@@ -102,8 +116,7 @@ def test_gemm_small_shapes_full_output(nf4lib, oracle_mod, cuda_device, M, K, N,
     st = quantize_on_gpu(nf4lib, W, cuda_device, dq)
     dA = None if A is None else A.to(cuda_device)
     dB = None if B is None else B.to(cuda_device)
-    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, N, dA, dB,
-                                   c.scaling)
+    y = linear(nf4lib, x.to(cuda_device), st, N, dA, dB, c.scaling)
     nf4lib.nf4_device_status()
     check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
 
@@ -114,13 +127,14 @@ def sampled_rows(M, count, seed):
     return np.unique(np.concatenate([rows, [0, M - 1]])).astype(np.int64)
 
 
-@pytest.mark.parametrize("case,nrows", [(wl.GEMM_TRAIN, 192), (wl.GEMM_70B_MLP, 48)], ids=["train4096", "mlp70b"])
+@pytest.mark.parametrize("case,nrows", [(wl.GEMM_TRAIN, 192), (wl.GEMM_70B_MLP, 48), (wl.GEMM_DOWN_PROJ, 64),
+                                        (wl.GEMM_K_PROJ, 128)],
+                         ids=["train4096", "mlp70b", "down_proj", "k_proj"])
 def test_gemm_full_size_sampled_rows(nf4lib, oracle_mod, cuda_device, case, nrows):
     W, x, A, B = wl.linear_inputs(case)
     st = quantize_on_gpu(nf4lib, W, cuda_device)
     del W
-    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, case.N,
-                                   A.to(cuda_device), B.to(cuda_device), case.scaling)
+    y = linear(nf4lib, x.to(cuda_device), st, case.N, A.to(cuda_device), B.to(cuda_device), case.scaling)
     nf4lib.nf4_device_status()
     rows = sampled_rows(case.M, nrows, case.seed)
     ref = oracle_linear(oracle_mod, st, x, A, B, case.r, case.scaling, rows=rows)
@@ -133,8 +147,7 @@ def test_gemm_partial_last_wave(nf4lib, oracle_mod, cuda_device):
     c = wl.LinearCase("gemm partial wave", 512, 1024, 9600, 16, 0.5, 4242)
     W, x, A, B = wl.linear_inputs(c)
     st = quantize_on_gpu(nf4lib, W, cuda_device)
-    y = nf4lib.nf4_lora_linear_fwd(x.to(cuda_device), st.packed, st.absmax_q, st.absmax2, st.offset, c.N,
-                                   A.to(cuda_device), B.to(cuda_device), c.scaling)
+    y = linear(nf4lib, x.to(cuda_device), st, c.N, A.to(cuda_device), B.to(cuda_device), c.scaling)
     nf4lib.nf4_device_status()
     rows = np.unique(np.concatenate([sampled_rows(c.M, 8, c.seed), np.arange(c.M - 8, c.M)])).astype(np.int64)
     ref = oracle_linear(oracle_mod, st, x, A, B, c.r, c.scaling, rows=rows)
@@ -146,7 +159,7 @@ def test_gemm_without_lora_equals_matmul_on_dequantized(nf4lib, cuda_device):
     W, x, _, _ = wl.linear_inputs(c, with_lora=False)
     st = quantize_on_gpu(nf4lib, W, cuda_device)
     xd = x.to(cuda_device)
-    y = nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N)
+    y = linear(nf4lib, xd, st, c.N)
     wb = nf4lib.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N * c.K).view(c.N, c.K)
     ref = torch.matmul(xd.float(), wb.float().t())
     nf4lib.nf4_device_status()
@@ -159,9 +172,8 @@ def test_gemm_and_gemv_agree_on_shared_rows(nf4lib, cuda_device):
     W, x, A, B = wl.linear_inputs(c)
     st = quantize_on_gpu(nf4lib, W, cuda_device)
     xd, Ad, Bd = x.to(cuda_device), A.to(cuda_device), B.to(cuda_device)
-    y64 = nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, Ad, Bd, c.scaling)
-    y16 = nf4lib.nf4_lora_linear_fwd(xd[:16].contiguous(), st.packed, st.absmax_q, st.absmax2, st.offset, c.N, Ad, Bd,
-                                     c.scaling)
+    y64 = linear(nf4lib, xd, st, c.N, Ad, Bd, c.scaling)
+    y16 = linear(nf4lib, xd[:16].contiguous(), st, c.N, Ad, Bd, c.scaling)
     nf4lib.nf4_device_status()
     check(y16, y64[:16].float().cpu().numpy())
 
@@ -188,9 +200,7 @@ def test_split_decode_pipeline(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
     assert full > t_only
     outs = []
     for ws_bytes in (full, full, t_only, full):
-        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=cuda_device)
-        outs.append(nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, N, dA, dB,
-                                               c.scaling, workspace=ws))
+        outs.append(linear(nf4lib, xd, st, N, dA, dB, c.scaling, ws_bytes=ws_bytes))
     torch.cuda.synchronize()
     assert nf4lib.nf4_device_status() == 0
     for y in outs:
@@ -202,21 +212,23 @@ def test_split_decode_pipeline_back_to_back(nf4lib, cuda_device):
     """Calls of the split pipeline queued back to back on one stream, with
     and without an adapter, reuse one workspace (its arrival counts are
     zeroed by the kernel launched before each linear): every output equals
-    the same call run alone."""
+    the same call run alone, and no call writes outside its output or the
+    shared workspace."""
     c = wl.LinearCase("split b2b", 16, 2048, 4096, 16, 2.0, 93)
     W, x, A, B = wl.linear_inputs(c)
     st = quantize_on_gpu(nf4lib, W, cuda_device)
     xd, Ad, Bd = x.to(cuda_device), A.to(cuda_device), B.to(cuda_device)
-    ws = torch.empty(nf4lib.nf4_lora_linear_workspace_size(16, 16), dtype=torch.uint8, device=cuda_device)
-    alone = [nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, a, b, c.scaling,
-                                        workspace=ws) for a, b in ((Ad, Bd), (None, None))]
-    torch.cuda.synchronize()
+    alone = [linear(nf4lib, xd, st, c.N, a, b, c.scaling) for a, b in ((Ad, Bd), (None, None))]
+    ws = guarded(nf4lib.nf4_lora_linear_workspace_size(16, 16), torch.uint8, cuda_device)
     ys = []
     for i in range(12):
         a, b = ((Ad, Bd), (None, None))[i % 2]
-        ys.append(nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, a, b, c.scaling,
-                                             workspace=ws))
+        y = guarded((c.M, c.N), torch.bfloat16, cuda_device)
+        nf4lib.nf4_lora_linear_fwd(xd, st.packed, st.absmax_q, st.absmax2, st.offset, c.N, a, b, c.scaling, y=y,
+                                   workspace=ws)
+        ys.append(y)
     torch.cuda.synchronize()
     assert nf4lib.nf4_device_status() == 0
+    check_guards(ws, *ys)
     for i, y in enumerate(ys):
         assert torch.equal(y, alone[i % 2]), i

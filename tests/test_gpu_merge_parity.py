@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import nf4_workloads as wl
+from conftest import check_guards, guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -39,8 +40,11 @@ def test_merge_requantize_bit_exact(nf4lib, oracle_mod, cuda_device, N, K, r, mo
     s = 1.75
     Ad = A.to(cuda_device) if r else None
     Bd = B.to(cuda_device) if r else None
-    pk, ab = nf4lib.nf4_merge_requantize(st.packed, st.absmax_q, st.absmax2, st.offset, N, K, Ad, Bd, s)
+    pk, ab = guarded(N * K // 2, torch.uint8, cuda_device), guarded(N * K // 64, torch.float32, cuda_device)
+    nf4lib.nf4_merge_requantize(st.packed, st.absmax_q, st.absmax2, st.offset, N, K, Ad, Bd, s, packed_out=pk,
+                                absmax_out=ab)
     torch.cuda.synchronize()
+    check_guards(pk, ab)
     packed, codes, sc, mu = state_np(st)
     ref_p, ref_a = oracle_mod.merge_requantize(packed, codes, sc, mu, K, bits(A) if r else None,
                                                bits(B) if r else None, r, s)
@@ -57,11 +61,14 @@ def test_merge_requantize_bit_exact(nf4lib, oracle_mod, cuda_device, N, K, r, mo
 def test_merge_in_place(nf4lib, oracle_mod, cuda_device):
     N, K, r = 96, 512, 16
     W, A, B = case(N, K, r, 77)
-    st = nf4lib.quantize_weight(W.to(cuda_device), double_quant=False)
+    pk, ab = guarded(N * K // 2, torch.uint8, cuda_device), guarded(N * K // 64, torch.float32, cuda_device)
+    nf4lib.nf4_quantize(W.to(cuda_device).reshape(-1), packed=pk, absmax=ab)
+    st = nf4lib.QuantState(pk, None, ab, None, (N, K))
     packed, codes, sc, mu = state_np(st)
     nf4lib.nf4_merge_requantize(st.packed, None, st.absmax2, None, N, K, A.to(cuda_device), B.to(cuda_device), 0.5,
                                 packed_out=st.packed, absmax_out=st.absmax2)
     torch.cuda.synchronize()
+    check_guards(pk, ab)
     ref_p, ref_a = oracle_mod.merge_requantize(packed, codes, sc, mu, K, bits(A), bits(B), r, 0.5)
     assert np.array_equal(st.packed.cpu().numpy(), ref_p)
     assert np.array_equal(st.absmax2.cpu().numpy().view(np.uint32), ref_a.view(np.uint32))
@@ -71,9 +78,11 @@ def test_merge_training_weight_sampled_rows(nf4lib, oracle_mod, cuda_device):
     c = wl.GEMM_TRAIN
     W, _, A, B = wl.linear_inputs(c)
     st = nf4lib.quantize_weight(W.to(cuda_device))
-    pk, ab = nf4lib.nf4_merge_requantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N, c.K,
-                                         A.to(cuda_device), B.to(cuda_device), c.scaling)
+    pk, ab = guarded(c.N * c.K // 2, torch.uint8, cuda_device), guarded(c.N * c.K // 64, torch.float32, cuda_device)
+    nf4lib.nf4_merge_requantize(st.packed, st.absmax_q, st.absmax2, st.offset, c.N, c.K, A.to(cuda_device),
+                                B.to(cuda_device), c.scaling, packed_out=pk, absmax_out=ab)
     torch.cuda.synchronize()
+    check_guards(pk, ab)
     packed, codes, sc, mu = state_np(st)
     pk, ab = pk.cpu().numpy(), ab.cpu().numpy()
     K = c.K

@@ -6,6 +6,7 @@ import pytest
 import torch
 
 import nf4_workloads as wl
+from conftest import check_guards, guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -22,16 +23,40 @@ def oracle_input(w_cpu: torch.Tensor) -> np.ndarray:
     return u16(w_cpu).ravel() if w_cpu.dtype == torch.bfloat16 else w_cpu.contiguous().numpy().ravel()
 
 
+def dq_guarded(q, c1: torch.Tensor, centre=True):
+    """nf4_double_quantize into guarded outputs (and workspace); checks the
+    guards and returns (codes, c2, mu or None)."""
+    dev = c1.device
+    nb = c1.numel()
+    nd = -(-nb // 256)
+    q8, c2 = guarded(nb, torch.uint8, dev), guarded(nd, torch.float32, dev)
+    off = guarded(1, torch.float32, dev) if centre else None
+    ws = guarded(q.nf4_double_quantize_workspace_size(nb), torch.uint8, dev)
+    q.nf4_double_quantize(c1, centre=centre, absmax_q=q8, absmax2=c2, offset=off, workspace=ws)
+    torch.cuda.synchronize()
+    check_guards(q8, c2, off, ws)
+    return q8, c2, off
+
+
 def run_round_trip(q, oracle_mod, w_cpu: torch.Tensor, centre=True):
     dev = torch.device("cuda:0")
     w = w_cpu.to(dev)
     n = w.numel()
-    packed, absmax = q.nf4_quantize(w.reshape(-1))
-    q8, c2, off = q.nf4_double_quantize(absmax, centre=centre)
-    f32 = q.nf4_dequantize(packed, q8, c2, off, n, torch.float32)
-    b16 = q.nf4_dequantize(packed, q8, c2, off, n, torch.bfloat16)
-    nodq = q.nf4_dequantize(packed, None, absmax, None, n, torch.float32)
+    nb = -(-n // 64)
+    nd = -(-nb // 256)
+    packed, absmax = guarded(n // 2, torch.uint8, dev), guarded(nb, torch.float32, dev)
+    q.nf4_quantize(w.reshape(-1), packed=packed, absmax=absmax)
+    q8, c2 = guarded(nb, torch.uint8, dev), guarded(nd, torch.float32, dev)
+    off = guarded(1, torch.float32, dev) if centre else None
+    ws = guarded(q.nf4_double_quantize_workspace_size(nb), torch.uint8, dev)
+    q.nf4_double_quantize(absmax, centre=centre, absmax_q=q8, absmax2=c2, offset=off, workspace=ws)
+    f32, b16 = guarded(n, torch.float32, dev), guarded(n, torch.bfloat16, dev)
+    nodq = guarded(n, torch.float32, dev)
+    q.nf4_dequantize(packed, q8, c2, off, n, torch.float32, out=f32)
+    q.nf4_dequantize(packed, q8, c2, off, n, torch.bfloat16, out=b16)
+    q.nf4_dequantize(packed, None, absmax, None, n, torch.float32, out=nodq)
     torch.cuda.synchronize()
+    check_guards(packed, absmax, q8, c2, off, ws, f32, b16, nodq)
 
     op, oa = oracle_mod.quantize(oracle_input(w_cpu))
     assert np.array_equal(packed.cpu().numpy(), op), "packed codes differ"
@@ -120,14 +145,18 @@ def tie_and_edge_tensor(oracle_mod) -> torch.Tensor:
 def test_ties_and_edge_values(nf4lib, oracle_mod, cuda_device):
     w = tie_and_edge_tensor(oracle_mod)
     dev = cuda_device
-    packed, absmax = nf4lib.nf4_quantize(w.to(dev))
+    n = w.numel()
+    packed, absmax = guarded(n // 2, torch.uint8, dev), guarded(n // 64, torch.float32, dev)
+    nf4lib.nf4_quantize(w.to(dev), packed=packed, absmax=absmax)
     op, oa = oracle_mod.quantize(w.numpy())
     assert np.array_equal(packed.cpu().numpy(), op)
     assert np.array_equal(f32bits(absmax.cpu().numpy()), f32bits(oa))
     # dequantize without DQ: exact including signed zeros
-    out = nf4lib.nf4_dequantize(packed, None, absmax, None, w.numel(), torch.float32)
-    ref = oracle_mod.dequantize(op, None, oa, None, w.numel(), "f32")
+    out = guarded(n, torch.float32, dev)
+    nf4lib.nf4_dequantize(packed, None, absmax, None, n, torch.float32, out=out)
+    ref = oracle_mod.dequantize(op, None, oa, None, n, "f32")
     assert np.array_equal(f32bits(out.cpu().numpy()), f32bits(ref))
+    check_guards(packed, absmax, out)
 
 
 def test_dq_sequential_fallback_and_zero_runs(nf4lib, oracle_mod, cuda_device):
@@ -141,7 +170,7 @@ def test_dq_sequential_fallback_and_zero_runs(nf4lib, oracle_mod, cuda_device):
     c1[256 * 9: 256 * 10] = 0.0
     dev = cuda_device
     for centre in (True, False):
-        q8, c2, off = nf4lib.nf4_double_quantize(torch.from_numpy(c1).to(dev), centre=centre)
+        q8, c2, off = dq_guarded(nf4lib, torch.from_numpy(c1).to(dev), centre=centre)
         oq8, oc2, omu = oracle_mod.double_quantize(c1, centre=centre)
         assert np.array_equal(q8.cpu().numpy(), oq8)
         assert np.array_equal(f32bits(c2.cpu().numpy()), f32bits(oc2))
@@ -149,7 +178,7 @@ def test_dq_sequential_fallback_and_zero_runs(nf4lib, oracle_mod, cuda_device):
             assert f32bits(off.cpu().numpy())[0] == f32bits([omu])[0]
     # every constant equal to the mean: c2 = 0 and code 0
     c1 = np.full(1000, 0.0625, np.float32)
-    q8, c2, off = nf4lib.nf4_double_quantize(torch.from_numpy(c1).to(dev))
+    q8, c2, off = dq_guarded(nf4lib, torch.from_numpy(c1).to(dev))
     assert float(off.item()) == 0.0625 and torch.all(c2 == 0) and torch.all(q8 == 0)
 
 
@@ -157,7 +186,7 @@ def test_many_chunks_mean(nf4lib, oracle_mod, cuda_device):
     """More than one chunk of 32 runs, ragged last chunk (tree across chunks)."""
     rng = np.random.default_rng(14)
     c1 = (rng.standard_normal(256 * 1000 + 100) ** 2 * 0.01).astype(np.float32)
-    q8, c2, off = nf4lib.nf4_double_quantize(torch.from_numpy(c1).to(cuda_device))
+    q8, c2, off = dq_guarded(nf4lib, torch.from_numpy(c1).to(cuda_device))
     oq8, oc2, omu = oracle_mod.double_quantize(c1)
     assert f32bits(off.cpu().numpy())[0] == f32bits([omu])[0]
     assert np.array_equal(q8.cpu().numpy(), oq8)
@@ -175,3 +204,61 @@ def test_stream_ordering_on_side_stream(nf4lib, oracle_mod, cuda_device):
     op, oa = oracle_mod.quantize(u16(w).ravel())
     assert np.array_equal(packed.cpu().numpy(), op)
     assert np.array_equal(u16(out), oracle_mod.dequantize(op, None, oa, None, w.numel(), "bf16"))
+
+
+def test_large_weight_dequant_element_by_element(nf4lib, oracle_mod, cuda_device):
+    """The 14336 x 4096 training weight (58.7 M elements, above 2^25, so the
+    dequantizer's large-output launch shape): codes, constants and every
+    element of the bf16 and fp32 dequantization against the oracle."""
+    w = wl.weight((14336, 4096), 0.02, wl.GEMM_TRAIN.seed, "bf16")
+    n = w.numel()
+    dev = cuda_device
+    st = nf4lib.quantize_weight(w.to(dev))
+    op, oa = oracle_mod.quantize(u16(w).ravel())
+    oq8, oc2, omu = oracle_mod.double_quantize(oa)
+    assert np.array_equal(st.packed.cpu().numpy(), op)
+    assert np.array_equal(st.absmax_q.cpu().numpy(), oq8)
+    assert np.array_equal(f32bits(st.absmax2.cpu().numpy()), f32bits(oc2))
+    assert f32bits(st.offset.cpu().numpy())[0] == f32bits([omu])[0]
+    for dt, name in ((torch.bfloat16, "bf16"), (torch.float32, "f32")):
+        out = guarded(n, dt, dev)
+        nf4lib.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, n, dt, out=out)
+        torch.cuda.synchronize()
+        check_guards(out)
+        ref = oracle_mod.dequantize(op, oq8, oc2, omu, n, name)
+        got = u16(out) if name == "bf16" else f32bits(out.cpu().numpy())
+        exp = ref if name == "bf16" else f32bits(ref)
+        bad = np.flatnonzero(got != exp)
+        assert bad.size == 0, f"{name}: {bad.size} elements differ, first at {bad[:5]}"
+        del out
+
+
+def test_70b_mlp_weight_dequant_sampled_runs(nf4lib, oracle_mod, cuda_device):
+    """The 28672 x 8192 MLP weight (234.9 M elements): codes, constants and
+    mean in full; the bf16 dequantization element by element on 48 whole
+    runs of 16,384 elements (one second-level block each) spread over the
+    tensor, first and last run included."""
+    w = wl.weight((28672, 8192), 0.02, wl.GEMM_70B_MLP.seed, "bf16")
+    n = w.numel()
+    run = 64 * 256
+    dev = cuda_device
+    st = nf4lib.quantize_weight(w.to(dev))
+    out = guarded(n, torch.bfloat16, dev)
+    nf4lib.nf4_dequantize(st.packed, st.absmax_q, st.absmax2, st.offset, n, torch.bfloat16, out=out)
+    torch.cuda.synchronize()
+    check_guards(out)
+    bits = u16(w).ravel()
+    del w
+    op, oa = oracle_mod.quantize(bits)
+    oq8, oc2, omu = oracle_mod.double_quantize(oa)
+    assert np.array_equal(st.packed.cpu().numpy(), op)
+    assert np.array_equal(st.absmax_q.cpu().numpy(), oq8)
+    assert np.array_equal(f32bits(st.absmax2.cpu().numpy()), f32bits(oc2))
+    assert f32bits(st.offset.cpu().numpy())[0] == f32bits([omu])[0]
+    runs = n // run
+    rng = np.random.default_rng(70)
+    pick = np.unique(np.concatenate([[0, runs - 1], rng.choice(runs, 46, replace=False)]))
+    for d in pick:
+        e0, e1 = d * run, (d + 1) * run
+        ref = oracle_mod.dequantize(op[e0 // 2:e1 // 2], oq8[e0 // 64:e1 // 64], oc2[d:d + 1], omu, run, "bf16")
+        assert np.array_equal(u16(out[e0:e1]), ref), f"run {d} differs"

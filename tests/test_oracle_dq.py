@@ -109,6 +109,31 @@ def test_double_quantize_without_centring_is_literal_formula(oracle_mod):
         assert np.array_equal(codes[k * 256:(k + 1) * 256], want)
 
 
+def test_centred_codes_bit_for_bit(oracle_mod):
+    """Centred codes are E4M3 (torch.float8_e4m3fn, a library routine) of
+    RN(RN(c1 - mu) / c2), each step one binary32 rounding (numpy float32
+    arithmetic), with c2 the run's max |RN(c1 - mu)|; a run with c2 = 0 stores
+    0.  Constants from the projection weight (outliers included) and a mix of
+    magnitudes on both sides of the mean."""
+    _, proj = oracle_mod.quantize(wl.weight_case(wl.PROJECTION).float().numpy().ravel())
+    rng = np.random.default_rng(17)
+    mixed = (rng.uniform(0.0, 1.0, 256 * 9 + 77) * 2.0 ** rng.integers(-12, 3, 256 * 9 + 77)).astype(np.float32)
+    mixed[256 * 2:256 * 3] = np.float32(0.25)  # a run near the mean of its neighbours
+    for c1 in (proj, mixed):
+        codes, c2, mu = oracle_mod.double_quantize(c1)
+        d = c1 - np.float32(mu)
+        assert d.dtype == np.float32
+        for k in range(c2.size):
+            dk = d[k * 256:(k + 1) * 256]
+            assert c2[k] == np.max(np.abs(dk))
+            if c2[k] == 0:
+                want = np.zeros(dk.size, np.uint8)
+            else:
+                y = dk / np.float32(c2[k])
+                assert y.dtype == np.float32
+                want = torch_e4m3(y)
+            assert np.array_equal(codes[k * 256:(k + 1) * 256], want), k
+
 def test_double_quantize_zero_run(oracle_mod):
     c1 = np.full(300, 0.05, np.float32)  # every constant equal to the mean
     codes, c2, mu = oracle_mod.double_quantize(c1)
