@@ -126,6 +126,45 @@ NF4_API nf4_status nf4_double_quantize(const float *absmax, int64_t nblocks, int
                                uint8_t *absmax_q, float *absmax2, float *offset,
                                void *workspace, int64_t workspace_bytes, void *stream);
 
+/* nf4_dq_run_sums -- the first step of the centring mean of nf4_double_quantize
+ * on its own: run_sums[d] = the binary64 sum of the constants of run d (256
+ * consecutive constants, the last run possibly shorter), summed in index
+ * order ([MF] "Double Quantization (DQ)": the per-tensor "bias/mean
+ * subtraction"; the summation order is the READING stated for
+ * nf4_double_quantize).  For a tensor split over ranks on run boundaries
+ * (every shard but the last a multiple of 16,384 weights) each rank computes
+ * its runs' sums; the caller gathers them in shard order and passes the whole
+ * array to nf4_double_quantize_sharded.
+ *   absmax    device fp32[nblocks]  (this shard's constants, from nf4_quantize)
+ *   run_sums  device fp64[ceil(nblocks / 256)]  (output)
+ * NF4_ERR_UNSUPPORTED if dq_blocksize != 256.  One kernel launch. */
+NF4_API nf4_status nf4_dq_run_sums(const float *absmax, int64_t nblocks, int dq_blocksize, double *run_sums,
+                                   void *stream);
+
+/* Bytes of device workspace nf4_double_quantize_sharded needs for a tensor
+ * of nblocks_total constants. */
+NF4_API int64_t nf4_double_quantize_sharded_workspace_size(int64_t nblocks_total, int dq_blocksize);
+
+/* nf4_double_quantize_sharded -- nf4_double_quantize (with centring) of one
+ * shard of a tensor, with the mean of the whole tensor: mu = RN_f32(S /
+ * nblocks_total), S the fixed pairwise tree over the run sums of ALL runs of
+ * the tensor (run_sums_all, as written by nf4_dq_run_sums on every shard and
+ * concatenated in shard order).  Codes, c2 and mu are bit-identical to
+ * nf4_double_quantize of the whole tensor, for any split on run boundaries.
+ *   absmax        device fp32[nblocks], this shard's constants (0 allowed:
+ *                 only mu is written)
+ *   run_sums_all  device fp64[ceil(nblocks_total / 256)]
+ *   absmax_q      device uint8[nblocks]; absmax2 device fp32[ceil(nblocks/256)]
+ *   offset        device fp32[1] (output mu; required)
+ *   workspace     device scratch, workspace_bytes >=
+ *                 nf4_double_quantize_sharded_workspace_size(nblocks_total)
+ * NF4_ERR_INVALID for nblocks > nblocks_total or missing buffers.  Two kernel
+ * launches (one when nblocks == 0). */
+NF4_API nf4_status nf4_double_quantize_sharded(const float *absmax, int64_t nblocks, int dq_blocksize,
+                                               const double *run_sums_all, int64_t nblocks_total,
+                                               uint8_t *absmax_q, float *absmax2, float *offset,
+                                               void *workspace, int64_t workspace_bytes, void *stream);
+
 /* nf4_dequantize -- w~_j = c1' * q[code_j] in binary32 ([MF] "Block-Wise
  * Quantization Mechanics", dequantization equation), with the block constant
  *   c1' = fma(E4M3(absmax_q[b]), absmax2[b/256], *offset)   (one rounding;

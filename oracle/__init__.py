@@ -70,6 +70,10 @@ def lib() -> ctypes.CDLL:
             L.nf4o_dq_mean.argtypes = [P, i64, ctypes.c_int]
             L.nf4o_dq_mean.restype = ctypes.c_float
             L.nf4o_double_quantize.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P, P]
+            L.nf4o_dq_run_sums.argtypes = [P, i64, ctypes.c_int, P]
+            L.nf4o_dq_mean_from_run_sums.argtypes = [P, i64, i64]
+            L.nf4o_dq_mean_from_run_sums.restype = ctypes.c_float
+            L.nf4o_double_quantize_with_mean.argtypes = [P, i64, ctypes.c_int, ctypes.c_float, P, P]
             L.nf4o_dequantize_f32.argtypes = [P, P, P, P, i64, ctypes.c_int, ctypes.c_int, P]
             L.nf4o_dequantize_bf16.argtypes = [P, P, P, P, i64, ctypes.c_int, ctypes.c_int, P]
             L.nf4o_lora_linear.argtypes = [P, i64, i64, i64, P, P, P, P, ctypes.c_int, ctypes.c_int,
@@ -193,6 +197,31 @@ def double_quantize(absmax: np.ndarray, dq_blocksize: int = DQ_BLOCKSIZE, centre
     lib().nf4o_double_quantize(_ptr(a), nb, dq_blocksize, 1 if centre else 0,
                                _ptr(codes), _ptr(absmax2), _ptr(off))
     return codes, absmax2, np.float32(off[0])
+
+
+def dq_run_sums(absmax: np.ndarray, dq_blocksize: int = DQ_BLOCKSIZE) -> np.ndarray:
+    """Step 1 of the mean: the sequential binary64 sum of each run."""
+    a = np.ascontiguousarray(absmax, np.float32)
+    out = np.zeros(-(-a.size // dq_blocksize), np.float64)
+    lib().nf4o_dq_run_sums(_ptr(a), a.size, dq_blocksize, _ptr(out))
+    return out
+
+
+def dq_mean_from_run_sums(run_sums: np.ndarray, nblocks: int) -> np.float32:
+    """Steps 2 and 3 of the mean (pairwise tree, division, rounding) on the
+    run sums of a whole tensor of nblocks constants."""
+    s = np.ascontiguousarray(run_sums, np.float64)
+    return np.float32(lib().nf4o_dq_mean_from_run_sums(_ptr(s), s.size, int(nblocks)))
+
+
+def double_quantize_with_mean(absmax: np.ndarray, mu, dq_blocksize: int = DQ_BLOCKSIZE):
+    """Double quantization of the runs of ``absmax`` with a given mean mu;
+    returns (codes uint8[nb], absmax2 float32[nd])."""
+    a = np.ascontiguousarray(absmax, np.float32)
+    codes = np.zeros(a.size, np.uint8)
+    absmax2 = np.zeros(-(-a.size // dq_blocksize), np.float32)
+    lib().nf4o_double_quantize_with_mean(_ptr(a), a.size, dq_blocksize, float(mu), _ptr(codes), _ptr(absmax2))
+    return codes, absmax2
 
 
 def dequantize(packed, codes, scales, offset, n, out_dtype="f32",

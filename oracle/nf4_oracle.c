@@ -226,16 +226,25 @@ void nf4o_quantize_bf16(const uint16_t *w, int64_t n, int bs, uint8_t *packed, f
  *   2. the run sums are combined level by level, s[j] = s[2j] + s[2j+1], an
  *      odd last element carried up unchanged, until one value remains;
  *   3. S / nb is rounded to binary64, then to binary32. */
-float nf4o_dq_mean(const float *c1, int64_t nb, int dqbs) {
-    if (nb <= 0) return 0.0f;
+/* Step 1 alone: s[d] = sequential binary64 sum of run d, d < ceil(nb/dqbs).
+ * For a tensor split into shards on run boundaries, the concatenation of the
+ * shards' run sums is the run-sum array of the whole tensor. */
+void nf4o_dq_run_sums(const float *c1, int64_t nb, int dqbs, double *s) {
     int64_t nd = (nb + dqbs - 1) / dqbs;
-    double *s = (double *)malloc((size_t)nd * sizeof(double));
     for (int64_t d = 0; d < nd; ++d) {
         int64_t lo = d * dqbs, hi = lo + dqbs < nb ? lo + dqbs : nb;
         double acc = 0.0;
         for (int64_t k = lo; k < hi; ++k) acc += (double)c1[k];
         s[d] = acc;
     }
+}
+
+/* Steps 2 and 3 on a run-sum array of nd entries (not modified) for a
+ * tensor of nb constants. */
+float nf4o_dq_mean_from_run_sums(const double *run_sums, int64_t nd, int64_t nb) {
+    if (nb <= 0 || nd <= 0) return 0.0f;
+    double *s = (double *)malloc((size_t)nd * sizeof(double));
+    memcpy(s, run_sums, (size_t)nd * sizeof(double));
     int64_t len = nd;
     while (len > 1) {
         int64_t half = len / 2;
@@ -248,6 +257,16 @@ float nf4o_dq_mean(const float *c1, int64_t nb, int dqbs) {
     return (float)mean;
 }
 
+float nf4o_dq_mean(const float *c1, int64_t nb, int dqbs) {
+    if (nb <= 0) return 0.0f;
+    int64_t nd = (nb + dqbs - 1) / dqbs;
+    double *s = (double *)malloc((size_t)nd * sizeof(double));
+    nf4o_dq_run_sums(c1, nb, dqbs, s);
+    float mu = nf4o_dq_mean_from_run_sums(s, nd, nb);
+    free(s);
+    return mu;
+}
+
 /* Double quantization, [MF] section "Double Quantization (DQ)": the fp32
  * constants are grouped in runs of dqbs (the last may be shorter); per run
  * c2 = max |c1 - mu| in fp32, and each constant is stored as the 8-bit float
@@ -256,10 +275,10 @@ float nf4o_dq_mean(const float *c1, int64_t nb, int dqbs) {
  * centre = 1 subtracts the mean above.  A run whose centred values are all
  * zero (c2 = 0) stores code 0x00.  codes[nb], absmax2[ceil(nb/dqbs)],
  * *offset = mu (if offset is not NULL). */
-void nf4o_double_quantize(const float *c1, int64_t nb, int dqbs, int centre,
-                          uint8_t *codes, float *absmax2, float *offset) {
-    float mu = centre ? nf4o_dq_mean(c1, nb, dqbs) : 0.0f;
-    if (offset) *offset = mu;
+/* The runs of the double quantization with a given mean mu (the tensor's
+ * mean; for a shard of a tensor, the whole tensor's). */
+void nf4o_double_quantize_with_mean(const float *c1, int64_t nb, int dqbs, float mu, uint8_t *codes,
+                                    float *absmax2) {
     int64_t nd = (nb + dqbs - 1) / dqbs;
     for (int64_t d = 0; d < nd; ++d) {
         int64_t lo = d * dqbs, hi = lo + dqbs < nb ? lo + dqbs : nb;
@@ -272,6 +291,13 @@ void nf4o_double_quantize(const float *c1, int64_t nb, int dqbs, int centre,
         for (int64_t k = lo; k < hi; ++k)
             codes[k] = (c2 == 0.0f) ? 0x00 : nf4o_e4m3_encode((c1[k] - mu) / c2);
     }
+}
+
+void nf4o_double_quantize(const float *c1, int64_t nb, int dqbs, int centre,
+                          uint8_t *codes, float *absmax2, float *offset) {
+    float mu = centre ? nf4o_dq_mean(c1, nb, dqbs) : 0.0f;
+    if (offset) *offset = mu;
+    nf4o_double_quantize_with_mean(c1, nb, dqbs, mu, codes, absmax2);
 }
 
 /* ------------------------------------------------------------------------ */

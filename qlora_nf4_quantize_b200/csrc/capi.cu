@@ -17,6 +17,10 @@ int64_t dq_chunk_count(int64_t nblocks);
 int64_t dq_max_chunks();
 cudaError_t launch_double_quantize(const float *absmax, int64_t nb, uint8_t *codes, float *absmax2,
                                    float *offset, double *chunk_sums, cudaStream_t stream, int num_sms);
+cudaError_t launch_dq_run_sums(const float *absmax, int64_t nb, double *run_sums, cudaStream_t stream);
+cudaError_t launch_double_quantize_sharded(const float *absmax, int64_t nb, const double *run_sums_all,
+                                           int64_t nd_total, int64_t nb_total, uint8_t *codes, float *absmax2,
+                                           float *offset, double *chunk_sums, cudaStream_t stream, int num_sms);
 cudaError_t launch_dequantize(const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
                               int64_t n, void *out, bool bf16, cudaStream_t stream, int num_sms);
 cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
@@ -134,6 +138,43 @@ nf4_status nf4_double_quantize(const float *absmax, int64_t nblocks, int dq_bloc
     if (st != cudaSuccess) return cuda_status(st);
     return cuda_status(nf4::launch_double_quantize(absmax, nblocks, absmax_q, absmax2, offset,
                                                    static_cast<double *>(workspace), (cudaStream_t)stream, sms));
+}
+
+nf4_status nf4_dq_run_sums(const float *absmax, int64_t nblocks, int dq_blocksize, double *run_sums,
+                           void *stream) {
+    if (dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
+    if (nblocks < 0) return NF4_ERR_INVALID;
+    if (nblocks == 0) return NF4_OK;
+    if (!absmax || !run_sums || !aligned16(absmax) || !aligned16(run_sums)) return NF4_ERR_INVALID;
+    return cuda_status(nf4::launch_dq_run_sums(absmax, nblocks, run_sums, (cudaStream_t)stream));
+}
+
+int64_t nf4_double_quantize_sharded_workspace_size(int64_t nblocks_total, int dq_blocksize) {
+    return nf4_double_quantize_workspace_size(nblocks_total, dq_blocksize);
+}
+
+nf4_status nf4_double_quantize_sharded(const float *absmax, int64_t nblocks, int dq_blocksize,
+                                       const double *run_sums_all, int64_t nblocks_total, uint8_t *absmax_q,
+                                       float *absmax2, float *offset, void *workspace, int64_t workspace_bytes,
+                                       void *stream) {
+    if (dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
+    if (nblocks < 0 || nblocks_total < 1 || nblocks > nblocks_total) return NF4_ERR_INVALID;
+    if (!run_sums_all || !offset || !workspace) return NF4_ERR_INVALID;
+    if (nblocks > 0 && (!absmax || !absmax_q || !absmax2)) return NF4_ERR_INVALID;
+    if (!aligned16(absmax) || !aligned16(absmax_q) || !aligned16(absmax2) || !aligned16(offset) ||
+        !aligned16(workspace) || !aligned16(run_sums_all))
+        return NF4_ERR_INVALID;
+    if (nf4::dq_chunk_count(nblocks_total) > nf4::dq_max_chunks()) return NF4_ERR_UNSUPPORTED;
+    if (workspace_bytes < nf4_double_quantize_sharded_workspace_size(nblocks_total, dq_blocksize))
+        return NF4_ERR_INVALID;
+    cudaError_t st;
+    int sms = sm_count(&st);
+    if (st != cudaSuccess) return cuda_status(st);
+    const int64_t nd_total = (nblocks_total + nf4::kDqBlock - 1) / nf4::kDqBlock;
+    return cuda_status(nf4::launch_double_quantize_sharded(absmax, nblocks, run_sums_all, nd_total, nblocks_total,
+                                                           absmax_q, absmax2, offset,
+                                                           static_cast<double *>(workspace), (cudaStream_t)stream,
+                                                           sms));
 }
 
 nf4_status nf4_dequantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2, const float *offset,

@@ -17,6 +17,12 @@
 //   k_dq_quantize    every CTA rebuilds mu from the chunk sums (the same
 //                    tree, continued); then one warp per run computes c2 and
 //                    the E4M3 codes.
+//   k_dq_run_sums, k_dq_chunks_from_runs
+//                    the same two steps split for a tensor sharded over
+//                    ranks on run boundaries: each rank writes its runs'
+//                    sums, the sums of all runs are gathered (the caller's
+//                    collective), and every rank rebuilds the same chunk
+//                    sums, so mu is bit-identical to a one-rank run.
 // The pairwise tree restricted to an aligned group of 2^L leaves is the
 // perfect tree of that group, and the last partial group follows the same
 // level-by-level rule on its own leaves, so splitting the tree at level 5
@@ -41,6 +47,51 @@ __device__ __forceinline__ int biased_exp(float v) {
     return e == 0 ? 1 : e;
 }
 
+// The fp64 sum of run d (constants lo .. lo + cnt - 1), as if summed
+// sequentially in index order; every lane of the warp gets it.
+__device__ __forceinline__ double run_sum_fp64(const float *__restrict__ c1, int64_t lo, int64_t cnt, int lane) {
+    double sum = 0.0;
+    int emin = 255, emax = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int64_t k = lane + 32 * i;
+        if (k < cnt) {
+            float v = __ldg(c1 + lo + k);
+            sum += (double)v;
+            if (v != 0.0f) {
+                int e = biased_exp(v);
+                emin = min(emin, e);
+                emax = max(emax, e);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        emin = min(emin, __shfl_xor_sync(0xFFFFFFFFu, emin, o));
+        emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
+    }
+    if (emax != 0 && emax - emin > 21) {  // rare: reproduce the sequential order
+        double acc = 0.0;
+        if (lane == 0)
+            for (int64_t k = 0; k < cnt; ++k) acc += (double)c1[lo + k];
+        sum = __shfl_sync(0xFFFFFFFFu, acc, 0);
+    }
+    return sum;
+}
+
+// Level-by-level pairwise combination of s[0..len) by one thread, in place
+// (each level reads s[2j], s[2j+1] before writing s[j], j increasing).
+__device__ __forceinline__ double tree_serial(double *s, int64_t len) {
+    while (len > 1) {
+        int64_t half = len >> 1;
+        for (int64_t j = 0; j < half; ++j) s[j] = s[2 * j] + s[2 * j + 1];
+        if (len & 1) s[half] = s[len - 1];
+        len = half + (len & 1);
+    }
+    return s[0];
+}
+
 __global__ void __launch_bounds__(1024) k_dq_chunk_sums(const float *__restrict__ c1, int64_t nb,
                                                          double *__restrict__ chunk_sums) {
     __shared__ double s_run[kRunsPerChunk];
@@ -51,48 +102,45 @@ __global__ void __launch_bounds__(1024) k_dq_chunk_sums(const float *__restrict_
     if (d < nd) {
         const int64_t lo = d * kDqBlock;
         const int64_t cnt = (nb - lo) < kDqBlock ? (nb - lo) : kDqBlock;
-        double sum = 0.0;
-        int emin = 255, emax = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            int64_t k = lane + 32 * i;
-            if (k < cnt) {
-                float v = __ldg(c1 + lo + k);
-                sum += (double)v;
-                if (v != 0.0f) {
-                    int e = biased_exp(v);
-                    emin = min(emin, e);
-                    emax = max(emax, e);
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-            emin = min(emin, __shfl_xor_sync(0xFFFFFFFFu, emin, o));
-            emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
-        }
-        if (emax != 0 && emax - emin > 21) {  // rare: reproduce the sequential order
-            if (lane == 0) {
-                double acc = 0.0;
-                for (int64_t k = 0; k < cnt; ++k) acc += (double)c1[lo + k];
-                sum = acc;
-            }
-        }
+        const double sum = run_sum_fp64(c1, lo, cnt, lane);
         if (lane == 0) s_run[warp] = sum;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
         int64_t len = nd - (int64_t)blockIdx.x * kRunsPerChunk;
         if (len > kRunsPerChunk) len = kRunsPerChunk;
-        while (len > 1) {
-            int64_t half = len >> 1;
-            for (int64_t j = 0; j < half; ++j) s_run[j] = s_run[2 * j] + s_run[2 * j + 1];
-            if (len & 1) s_run[half] = s_run[len - 1];
-            len = half + (len & 1);
-        }
-        chunk_sums[blockIdx.x] = s_run[0];
+        chunk_sums[blockIdx.x] = tree_serial(s_run, len);
     }
+}
+
+// Per-run fp64 sums only (the first step of a sharded double quantization):
+// one warp per run, run_sums[d] for d < ceil(nb / 256).
+__global__ void __launch_bounds__(256) k_dq_run_sums(const float *__restrict__ c1, int64_t nb,
+                                                      double *__restrict__ run_sums) {
+    pdl_wait_then_release();
+    const int lane = threadIdx.x & 31;
+    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
+    const int64_t d = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (d >= nd) return;  // whole warps leave together
+    const int64_t lo = d * kDqBlock;
+    const int64_t cnt = (nb - lo) < kDqBlock ? (nb - lo) : kDqBlock;
+    const double sum = run_sum_fp64(c1, lo, cnt, lane);
+    if (lane == 0) run_sums[d] = sum;
+}
+
+// Chunk sums (level-5 nodes of the pairwise tree) from the run sums of a
+// whole tensor: one thread per chunk of 32 consecutive runs.
+__global__ void __launch_bounds__(256) k_dq_chunks_from_runs(const double *__restrict__ run_sums, int64_t nd,
+                                                              double *__restrict__ chunk_sums) {
+    pdl_wait_then_release();
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nchunks = (nd + kRunsPerChunk - 1) / kRunsPerChunk;
+    if (c >= nchunks) return;
+    double s[kRunsPerChunk];
+    int64_t len = nd - c * kRunsPerChunk;
+    if (len > kRunsPerChunk) len = kRunsPerChunk;
+    for (int64_t j = 0; j < len; ++j) s[j] = run_sums[c * kRunsPerChunk + j];
+    chunk_sums[c] = tree_serial(s, len);
 }
 
 // Level-by-level pairwise combination of s[0..len) in shared memory (two
@@ -109,10 +157,13 @@ __device__ double tree_reduce(double *a, double *b, int64_t len) {
     return a[0];
 }
 
+// nb constants of c1 are quantized; the mean is S / nb_mean, where S is
+// the tree over nchunks chunk sums (nb_mean = nb unless c1 is one shard of a
+// larger tensor whose chunk sums cover all of it).
 __global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c1, int64_t nb,
                                                       const double *__restrict__ chunk_sums, int64_t nchunks,
-                                                      uint8_t *__restrict__ codes, float *__restrict__ absmax2,
-                                                      float *__restrict__ offset) {
+                                                      int64_t nb_mean, uint8_t *__restrict__ codes,
+                                                      float *__restrict__ absmax2, float *__restrict__ offset) {
     extern __shared__ double s_tree[];  // 2 * nchunks doubles when centring
     __shared__ float s_mu;
     pdl_wait_then_release();
@@ -121,7 +172,7 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c
         __syncthreads();
         double S = tree_reduce(s_tree, s_tree + nchunks, nchunks);
         if (threadIdx.x == 0) {
-            float mu = (float)(S / (double)nb);
+            float mu = (float)(S / (double)nb_mean);
             s_mu = mu;
             if (blockIdx.x == 0) *offset = mu;
         }
@@ -195,7 +246,39 @@ cudaError_t launch_double_quantize(const float *absmax, int64_t nb, uint8_t *cod
     int64_t cap = (int64_t)num_sms * 4;
     int grid = (int)(want < cap ? want : cap);
     return launch_pdl(k_dq_quantize, dim3(grid), dim3(256), smem, stream, 1, absmax, nb,
-                      static_cast<const double *>(chunk_sums), nchunks, codes, absmax2, offset);
+                      static_cast<const double *>(chunk_sums), nchunks, nb, codes, absmax2, offset);
+}
+
+cudaError_t launch_dq_run_sums(const float *absmax, int64_t nb, double *run_sums, cudaStream_t stream) {
+    if (nb == 0) return cudaSuccess;
+    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
+    return launch_pdl(k_dq_run_sums, dim3((unsigned)((nd + 7) / 8)), dim3(256), 0, stream, 1, absmax, nb, run_sums);
+}
+
+// Double quantization of one shard (nb constants, starting on a run
+// boundary of the whole tensor) with the mean of the whole tensor: the chunk
+// sums are rebuilt from all nd_total run sums, then the shard is quantized
+// with mu = RN_f32(S / nb_total).
+cudaError_t launch_double_quantize_sharded(const float *absmax, int64_t nb, const double *run_sums_all,
+                                           int64_t nd_total, int64_t nb_total, uint8_t *codes, float *absmax2,
+                                           float *offset, double *chunk_sums, cudaStream_t stream, int num_sms) {
+    if (nd_total == 0) return cudaSuccess;
+    const int64_t nchunks = (nd_total + kRunsPerChunk - 1) / kRunsPerChunk;
+    cudaError_t e = launch_pdl(k_dq_chunks_from_runs, dim3((unsigned)((nchunks + 255) / 256)), dim3(256), 0, stream,
+                               1, run_sums_all, nd_total, chunk_sums);
+    if (e != cudaSuccess) return e;
+    const size_t smem = (size_t)(2 * nchunks) * sizeof(double);
+    if (smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(k_dq_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
+    int64_t want = (nd + 7) / 8;
+    int64_t cap = (int64_t)num_sms * 4;
+    int grid = (int)(want < cap ? want : cap);
+    if (grid < 1) grid = 1;  // an empty shard still writes mu
+    return launch_pdl(k_dq_quantize, dim3(grid), dim3(256), smem, stream, 1, absmax, nb,
+                      static_cast<const double *>(chunk_sums), nchunks, nb_total, codes, absmax2, offset);
 }
 
 }  // namespace nf4

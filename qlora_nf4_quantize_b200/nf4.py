@@ -55,6 +55,12 @@ def lib() -> ctypes.CDLL:
     L.nf4_double_quantize_workspace_size.argtypes = [i64, i32]
     L.nf4_double_quantize.restype = i32
     L.nf4_double_quantize.argtypes = [P, i64, i32, P, P, P, P, i64, P]
+    L.nf4_dq_run_sums.restype = i32
+    L.nf4_dq_run_sums.argtypes = [P, i64, i32, P, P]
+    L.nf4_double_quantize_sharded_workspace_size.restype = i64
+    L.nf4_double_quantize_sharded_workspace_size.argtypes = [i64, i32]
+    L.nf4_double_quantize_sharded.restype = i32
+    L.nf4_double_quantize_sharded.argtypes = [P, i64, i32, P, i64, P, P, P, P, i64, P]
     L.nf4_dequantize.restype = i32
     L.nf4_dequantize.argtypes = [P, P, P, P, i64, i32, i32, P, i32, P]
     L.nf4_lora_linear_workspace_size.restype = i64
@@ -150,6 +156,43 @@ def nf4_double_quantize(absmax: torch.Tensor, dq_blocksize: int = DQ_BLOCKSIZE, 
                                    _p(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
                                    _stream(stream))
     _check("nf4_double_quantize", st)
+    return absmax_q, absmax2, offset
+
+
+def nf4_dq_run_sums(absmax: torch.Tensor, dq_blocksize: int = DQ_BLOCKSIZE, out=None, stream=None) -> torch.Tensor:
+    """fp64 sum of each run of 256 constants (the first step of the centring
+    mean); returns float64[ceil(nb / 256)]."""
+    _need(absmax, "absmax", torch.float32)
+    nb = absmax.numel()
+    nd = (nb + dq_blocksize - 1) // dq_blocksize
+    out = torch.empty(nd, dtype=torch.float64, device=absmax.device) if out is None else out
+    _need(out, "out", torch.float64, nd)
+    _check("nf4_dq_run_sums", lib().nf4_dq_run_sums(_p(absmax), nb, dq_blocksize, _p(out), _stream(stream)))
+    return out
+
+
+def nf4_double_quantize_sharded(absmax: torch.Tensor, run_sums_all: torch.Tensor, nblocks_total: int,
+                                dq_blocksize: int = DQ_BLOCKSIZE, absmax_q=None, absmax2=None, offset=None,
+                                workspace=None, stream=None):
+    """Double quantization of one shard with the mean of the whole tensor
+    (run_sums_all: every run's fp64 sum, in shard order).  Returns
+    (absmax_q uint8[nb], absmax2 fp32[ceil(nb/256)], offset fp32[1])."""
+    _need(absmax, "absmax", torch.float32)
+    nb = absmax.numel()
+    nd = (nb + dq_blocksize - 1) // dq_blocksize
+    nd_total = (nblocks_total + dq_blocksize - 1) // dq_blocksize
+    _need(run_sums_all, "run_sums_all", torch.float64, nd_total)
+    dev = absmax.device
+    absmax_q = torch.empty(nb, dtype=torch.uint8, device=dev) if absmax_q is None else absmax_q
+    absmax2 = torch.empty(nd, dtype=torch.float32, device=dev) if absmax2 is None else absmax2
+    offset = torch.empty(1, dtype=torch.float32, device=dev) if offset is None else offset
+    ws_bytes = int(lib().nf4_double_quantize_sharded_workspace_size(nblocks_total, dq_blocksize))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    st = lib().nf4_double_quantize_sharded(_p(absmax), nb, dq_blocksize, _p(run_sums_all), nblocks_total,
+                                           _p(absmax_q), _p(absmax2), _p(offset), _p(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("nf4_double_quantize_sharded", st)
     return absmax_q, absmax2, offset
 
 

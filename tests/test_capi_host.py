@@ -95,3 +95,19 @@ def test_workspace_sizes(nf4lib):
     assert nf4lib.nf4_lora_linear_workspace_size(17, 0) == 0
     assert nf4lib.nf4_lora_linear_workspace_size(4096, 0) == 0
     assert nf4lib.nf4_lora_linear_workspace_size(4096, 64) == 4096 * 128 * 2
+
+
+def test_sharded_dq_arguments_checked_on_the_host(nf4lib):
+    L = nf4lib.lib()
+    fake = ctypes.c_void_p(0x1000)
+    assert L.nf4_dq_run_sums(fake, 512, 128, fake, None) == 2            # second-level block must be 256
+    assert L.nf4_dq_run_sums(fake, -1, 256, fake, None) == 1
+    assert L.nf4_dq_run_sums(None, 0, 256, None, None) == 0               # empty: no-op
+    assert L.nf4_dq_run_sums(fake, 512, 256, ctypes.c_void_p(0x1008), None) == 1  # misaligned sums
+    ws = 1 << 20
+    args = lambda nb, tot, off: (fake, nb, 256, fake, tot, fake, fake, off, fake, ws, None)
+    assert L.nf4_double_quantize_sharded(*args(600, 500, fake)) == 1     # shard larger than the tensor
+    assert L.nf4_double_quantize_sharded(*args(100, 500, None)) == 1     # the mean must be written
+    assert L.nf4_double_quantize_sharded(*args(100, 0, fake)) == 1
+    assert L.nf4_double_quantize_sharded(fake, 100, 256, fake, 500, fake, fake, fake, fake, 0, None) == 1
+    assert nf4lib.lib().nf4_double_quantize_sharded_workspace_size(256 * 33, 256) == 16
