@@ -96,6 +96,31 @@ NF4_API nf4_status nf4_codebook(float *out_host);
 NF4_API nf4_status nf4_quantize(const void *w, nf4_dtype w_dtype, int64_t n, int blocksize,
                         uint8_t *packed, float *absmax, void *stream);
 
+/* Bytes of device workspace nf4_quantize_dq needs for n weights (the fp32
+ * block constants, then the fp64 run sums of the centring mean); 0 for
+ * n <= 0 or unsupported block sizes. */
+NF4_API int64_t nf4_quantize_dq_workspace_size(int64_t n, int blocksize, int dq_blocksize);
+
+/* nf4_quantize_dq -- nf4_quantize followed by nf4_double_quantize in one call
+ * ([MF] "Block-Wise Quantization Mechanics" and "Double Quantization (DQ)"):
+ * the stored format straight from the weight.  Every output is bit-identical
+ * to the two calls made in turn; the fp32 constants only pass through the
+ * workspace.
+ *   w          device, n elements of w_dtype; n even, >= 0
+ *   blocksize 64, dq_blocksize 256 (else NF4_ERR_UNSUPPORTED)
+ *   packed     device uint8[n/2]            (output)
+ *   absmax_q   device uint8[ceil(n/64)]     (output)
+ *   absmax2    device fp32[ceil(n/16384)]   (output)
+ *   offset     device fp32[1] (output mu) or NULL (no centring)
+ *   workspace  device scratch, 256-byte aligned, workspace_bytes >=
+ *              nf4_quantize_dq_workspace_size(n, 64, 256); contents on entry
+ *              are ignored.
+ * Three kernel launches with centring (four above 2048 runs, i.e. 33.5 M
+ * weights), two without. */
+NF4_API nf4_status nf4_quantize_dq(const void *w, nf4_dtype w_dtype, int64_t n, int blocksize, int dq_blocksize,
+                                   uint8_t *packed, uint8_t *absmax_q, float *absmax2, float *offset,
+                                   void *workspace, int64_t workspace_bytes, void *stream);
+
 /* Bytes of device workspace nf4_double_quantize needs for nblocks first-level
  * constants with centring (0 when nblocks == 0). */
 NF4_API int64_t nf4_double_quantize_workspace_size(int64_t nblocks, int dq_blocksize);
@@ -121,7 +146,7 @@ NF4_API int64_t nf4_double_quantize_workspace_size(int64_t nblocks, int dq_block
  *              is NULL.  Contents on entry are ignored; the caller keeps
  *              ownership; it must not be used by other work until the
  *              stream passes this call.
- * Two kernel launches with centring, one without. */
+ * Two kernel launches with centring (three above 2048 runs), one without. */
 NF4_API nf4_status nf4_double_quantize(const float *absmax, int64_t nblocks, int dq_blocksize,
                                uint8_t *absmax_q, float *absmax2, float *offset,
                                void *workspace, int64_t workspace_bytes, void *stream);

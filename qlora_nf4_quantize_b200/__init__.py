@@ -10,7 +10,8 @@ from .nf4 import (  # noqa: F401
     BLOCKSIZE, DQ_BLOCKSIZE, Nf4Error, lib, nf4_codebook, nf4_quantize, nf4_double_quantize,
     nf4_double_quantize_workspace_size, nf4_dequantize, nf4_lora_linear_fwd,
     nf4_lora_linear_workspace_size, nf4_lora_linear_fwd_noalloc, nf4_device_status, nf4_selftest_wait_timeout, nf4_merge_requantize, nf4_lora_linear_bwd,
-    nf4_lora_linear_bwd_workspace_size, nf4_dq_run_sums, nf4_double_quantize_sharded, QuantState,
+    nf4_lora_linear_bwd_workspace_size, nf4_dq_run_sums, nf4_double_quantize_sharded, nf4_quantize_dq,
+    nf4_quantize_dq_workspace_size, QuantState,
     quantize_weight, merge_and_requantize,
 )
 from . import sharded  # noqa: F401

@@ -13,14 +13,16 @@
 namespace nf4 {
 cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed, float *absmax,
                             cudaStream_t stream, int num_sms);
+int64_t dq_run_count(int64_t nblocks);
 int64_t dq_chunk_count(int64_t nblocks);
 int64_t dq_max_chunks();
+int64_t dq_workspace_bytes(int64_t nblocks);
 cudaError_t launch_double_quantize(const float *absmax, int64_t nb, uint8_t *codes, float *absmax2,
-                                   float *offset, double *chunk_sums, cudaStream_t stream, int num_sms);
+                                   float *offset, double *workspace, cudaStream_t stream, int num_sms);
 cudaError_t launch_dq_run_sums(const float *absmax, int64_t nb, double *run_sums, cudaStream_t stream);
-cudaError_t launch_double_quantize_sharded(const float *absmax, int64_t nb, const double *run_sums_all,
-                                           int64_t nd_total, int64_t nb_total, uint8_t *codes, float *absmax2,
-                                           float *offset, double *chunk_sums, cudaStream_t stream, int num_sms);
+cudaError_t launch_dq_from_run_sums(const float *absmax, int64_t nb, const double *run_sums, int64_t nb_total,
+                                    uint8_t *codes, float *absmax2, float *offset, double *chunk_sums,
+                                    cudaStream_t stream, int num_sms);
 cudaError_t launch_dequantize(const uint8_t *packed, const uint8_t *q8, const float *scales, const float *offset,
                               int64_t n, void *out, bool bf16, cudaStream_t stream, int num_sms);
 cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed,
@@ -113,9 +115,43 @@ nf4_status nf4_quantize(const void *w, nf4_dtype w_dtype, int64_t n, int blocksi
     return cuda_status(nf4::launch_quantize(w, w_dtype == NF4_BF16, n, packed, absmax, (cudaStream_t)stream, sms));
 }
 
+// Workspace of nf4_quantize_dq: the fp32 first-level constants (256-byte
+// aligned), then the run sums and chunk sums of the centring mean.
+static int64_t qdq_absmax_bytes(int64_t nb) { return (nb * 4 + 255) & ~(int64_t)255; }
+
+int64_t nf4_quantize_dq_workspace_size(int64_t n, int blocksize, int dq_blocksize) {
+    if (n <= 0 || blocksize != nf4::kBlock || dq_blocksize != nf4::kDqBlock) return 0;
+    const int64_t nb = (n + nf4::kBlock - 1) / nf4::kBlock;
+    return qdq_absmax_bytes(nb) + nf4::dq_workspace_bytes(nb);
+}
+
+nf4_status nf4_quantize_dq(const void *w, nf4_dtype w_dtype, int64_t n, int blocksize, int dq_blocksize,
+                           uint8_t *packed, uint8_t *absmax_q, float *absmax2, float *offset, void *workspace,
+                           int64_t workspace_bytes, void *stream) {
+    if (blocksize != nf4::kBlock || dq_blocksize != nf4::kDqBlock) return NF4_ERR_UNSUPPORTED;
+    if (n < 0 || (n & 1) || (w_dtype != NF4_F32 && w_dtype != NF4_BF16)) return NF4_ERR_INVALID;
+    if (n == 0) return NF4_OK;
+    if (!w || !packed || !absmax_q || !absmax2 || !workspace) return NF4_ERR_INVALID;
+    if (!aligned16(w) || !aligned16(packed) || !aligned16(absmax_q) || !aligned16(absmax2) || !aligned16(offset) ||
+        ((uintptr_t)workspace & 255u) != 0)
+        return NF4_ERR_INVALID;
+    if (workspace_bytes < nf4_quantize_dq_workspace_size(n, blocksize, dq_blocksize)) return NF4_ERR_INVALID;
+    const int64_t nb = (n + nf4::kBlock - 1) / nf4::kBlock;
+    if (offset != nullptr && nf4::dq_chunk_count(nb) > nf4::dq_max_chunks()) return NF4_ERR_UNSUPPORTED;
+    cudaError_t st;
+    int sms = sm_count(&st);
+    if (st != cudaSuccess) return cuda_status(st);
+    float *c1 = static_cast<float *>(workspace);
+    double *sums = reinterpret_cast<double *>(static_cast<char *>(workspace) + qdq_absmax_bytes(nb));
+    st = nf4::launch_quantize(w, w_dtype == NF4_BF16, n, packed, c1, (cudaStream_t)stream, sms);
+    if (st != cudaSuccess) return cuda_status(st);
+    return cuda_status(
+        nf4::launch_double_quantize(c1, nb, absmax_q, absmax2, offset, sums, (cudaStream_t)stream, sms));
+}
+
 int64_t nf4_double_quantize_workspace_size(int64_t nblocks, int dq_blocksize) {
     if (nblocks <= 0 || dq_blocksize != nf4::kDqBlock) return 0;
-    return nf4::dq_chunk_count(nblocks) * (int64_t)sizeof(double);
+    return nf4::dq_workspace_bytes(nblocks);
 }
 
 nf4_status nf4_double_quantize(const float *absmax, int64_t nblocks, int dq_blocksize, uint8_t *absmax_q,
@@ -150,7 +186,8 @@ nf4_status nf4_dq_run_sums(const float *absmax, int64_t nblocks, int dq_blocksiz
 }
 
 int64_t nf4_double_quantize_sharded_workspace_size(int64_t nblocks_total, int dq_blocksize) {
-    return nf4_double_quantize_workspace_size(nblocks_total, dq_blocksize);
+    if (nblocks_total <= 0 || dq_blocksize != nf4::kDqBlock) return 0;
+    return nf4::dq_chunk_count(nblocks_total) * (int64_t)sizeof(double);
 }
 
 nf4_status nf4_double_quantize_sharded(const float *absmax, int64_t nblocks, int dq_blocksize,
@@ -170,11 +207,9 @@ nf4_status nf4_double_quantize_sharded(const float *absmax, int64_t nblocks, int
     cudaError_t st;
     int sms = sm_count(&st);
     if (st != cudaSuccess) return cuda_status(st);
-    const int64_t nd_total = (nblocks_total + nf4::kDqBlock - 1) / nf4::kDqBlock;
-    return cuda_status(nf4::launch_double_quantize_sharded(absmax, nblocks, run_sums_all, nd_total, nblocks_total,
-                                                           absmax_q, absmax2, offset,
-                                                           static_cast<double *>(workspace), (cudaStream_t)stream,
-                                                           sms));
+    return cuda_status(nf4::launch_dq_from_run_sums(absmax, nblocks, run_sums_all, nblocks_total, absmax_q, absmax2,
+                                                    offset, static_cast<double *>(workspace), (cudaStream_t)stream,
+                                                    sms));
 }
 
 nf4_status nf4_dequantize(const uint8_t *packed, const uint8_t *absmax_q, const float *absmax2, const float *offset,

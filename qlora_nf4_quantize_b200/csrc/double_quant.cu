@@ -11,74 +11,34 @@
 // up unchanged.
 //
 // Kernels
-//   k_dq_chunk_sums  one warp per run: the run's fp64 sum, then one CTA
-//                    combines 32 consecutive run sums (a level-5 node of the
-//                    pairwise tree) into the workspace.
-//   k_dq_quantize    every CTA rebuilds mu from the chunk sums (the same
-//                    tree, continued); then one warp per run computes c2 and
-//                    the E4M3 codes.
-//   k_dq_run_sums, k_dq_chunks_from_runs
-//                    the same two steps split for a tensor sharded over
-//                    ranks on run boundaries: each rank writes its runs'
-//                    sums, the sums of all runs are gathered (the caller's
-//                    collective), and every rank rebuilds the same chunk
-//                    sums, so mu is bit-identical to a one-rank run.
+//   k_dq_run_sums    one warp per run: the run's fp64 sum (dq_sum.cuh).  The
+//                    quantizer can write the same sums as it goes
+//                    (nf4_quantize_dq), and a tensor sharded over ranks
+//                    gathers its shards' sums (nf4_double_quantize_sharded).
+//   k_dq_chunks_from_runs
+//                    for large tensors only: one thread per chunk of 32
+//                    consecutive run sums combines them (a level-5 node of
+//                    the pairwise tree).
+//   k_dq_quantize    every CTA rebuilds mu from the run sums (folding each
+//                    chunk of 32 itself) or from the chunk sums, by the same
+//                    tree; then one warp per run computes c2 and the E4M3
+//                    codes.
 // The pairwise tree restricted to an aligned group of 2^L leaves is the
 // perfect tree of that group, and the last partial group follows the same
 // level-by-level rule on its own leaves, so splitting the tree at level 5
 // reproduces the single-pass order exactly.
 //
-// Run sums in parallel: the sequential fp64 sum of one run equals its exact
-// sum whenever every partial sum is representable.  The constants are >= 0
-// and multiples of 2^(emin - 150) (emin = smallest biased exponent among the
-// non-zero ones, 1 for subnormals), and the total is below
-// 256 * 2^(emax - 126); if emax - emin <= 21 every subset sum is exact in
-// fp64, so any summation order gives the sequential result.  Otherwise lane 0
-// sums the run sequentially.
-#include "nf4_device.cuh"
+// Run sums: dq_sum.cuh (in parallel when exact, else sequentially).
+#include "dq_sum.cuh"
 
 namespace nf4 {
 namespace {
 
 constexpr int kRunsPerChunk = 32;
-
-__device__ __forceinline__ int biased_exp(float v) {
-    int e = (int)((__float_as_uint(v) >> 23) & 0xFF);
-    return e == 0 ? 1 : e;
-}
-
-// The fp64 sum of run d (constants lo .. lo + cnt - 1), as if summed
-// sequentially in index order; every lane of the warp gets it.
-__device__ __forceinline__ double run_sum_fp64(const float *__restrict__ c1, int64_t lo, int64_t cnt, int lane) {
-    double sum = 0.0;
-    int emin = 255, emax = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        int64_t k = lane + 32 * i;
-        if (k < cnt) {
-            float v = __ldg(c1 + lo + k);
-            sum += (double)v;
-            if (v != 0.0f) {
-                int e = biased_exp(v);
-                emin = min(emin, e);
-                emax = max(emax, e);
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        emin = min(emin, __shfl_xor_sync(0xFFFFFFFFu, emin, o));
-        emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
-    }
-    if (emax != 0 && emax - emin > 21) {  // rare: reproduce the sequential order
-        double acc = 0.0;
-        if (lane == 0)
-            for (int64_t k = 0; k < cnt; ++k) acc += (double)c1[lo + k];
-        sum = __shfl_sync(0xFFFFFFFFu, acc, 0);
-    }
-    return sum;
-}
+// Up to this many chunks every CTA of k_dq_quantize folds the run sums into
+// chunk sums itself (reading nd doubles, 16 KB at most); above, a separate
+// kernel writes the chunk sums once.
+constexpr int64_t kDirectChunks = 64;
 
 // Level-by-level pairwise combination of s[0..len) by one thread, in place
 // (each level reads s[2j], s[2j+1] before writing s[j], j increasing).
@@ -92,29 +52,16 @@ __device__ __forceinline__ double tree_serial(double *s, int64_t len) {
     return s[0];
 }
 
-__global__ void __launch_bounds__(1024) k_dq_chunk_sums(const float *__restrict__ c1, int64_t nb,
-                                                         double *__restrict__ chunk_sums) {
-    __shared__ double s_run[kRunsPerChunk];
-    pdl_wait_then_release();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
-    const int64_t d = (int64_t)blockIdx.x * kRunsPerChunk + warp;
-    if (d < nd) {
-        const int64_t lo = d * kDqBlock;
-        const int64_t cnt = (nb - lo) < kDqBlock ? (nb - lo) : kDqBlock;
-        const double sum = run_sum_fp64(c1, lo, cnt, lane);
-        if (lane == 0) s_run[warp] = sum;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int64_t len = nd - (int64_t)blockIdx.x * kRunsPerChunk;
-        if (len > kRunsPerChunk) len = kRunsPerChunk;
-        chunk_sums[blockIdx.x] = tree_serial(s_run, len);
-    }
+// The chunk sum (level-5 node) of runs 32 c .. min(32 c + 32, nd) - 1.
+__device__ __forceinline__ double chunk_sum(const double *__restrict__ run_sums, int64_t nd, int64_t c) {
+    double s[kRunsPerChunk];
+    int64_t len = nd - c * kRunsPerChunk;
+    if (len > kRunsPerChunk) len = kRunsPerChunk;
+    for (int64_t j = 0; j < len; ++j) s[j] = run_sums[c * kRunsPerChunk + j];
+    return tree_serial(s, len);
 }
 
-// Per-run fp64 sums only (the first step of a sharded double quantization):
-// one warp per run, run_sums[d] for d < ceil(nb / 256).
+// Per-run fp64 sums: one warp per run, run_sums[d] for d < ceil(nb / 256).
 __global__ void __launch_bounds__(256) k_dq_run_sums(const float *__restrict__ c1, int64_t nb,
                                                       double *__restrict__ run_sums) {
     pdl_wait_then_release();
@@ -124,23 +71,17 @@ __global__ void __launch_bounds__(256) k_dq_run_sums(const float *__restrict__ c
     if (d >= nd) return;  // whole warps leave together
     const int64_t lo = d * kDqBlock;
     const int64_t cnt = (nb - lo) < kDqBlock ? (nb - lo) : kDqBlock;
-    const double sum = run_sum_fp64(c1, lo, cnt, lane);
+    const double sum = run_sum_fp64(c1 + lo, cnt, lane);
     if (lane == 0) run_sums[d] = sum;
 }
 
-// Chunk sums (level-5 nodes of the pairwise tree) from the run sums of a
-// whole tensor: one thread per chunk of 32 consecutive runs.
+// Chunk sums of a whole tensor's run sums: one thread per chunk.
 __global__ void __launch_bounds__(256) k_dq_chunks_from_runs(const double *__restrict__ run_sums, int64_t nd,
                                                               double *__restrict__ chunk_sums) {
     pdl_wait_then_release();
     const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t nchunks = (nd + kRunsPerChunk - 1) / kRunsPerChunk;
-    if (c >= nchunks) return;
-    double s[kRunsPerChunk];
-    int64_t len = nd - c * kRunsPerChunk;
-    if (len > kRunsPerChunk) len = kRunsPerChunk;
-    for (int64_t j = 0; j < len; ++j) s[j] = run_sums[c * kRunsPerChunk + j];
-    chunk_sums[c] = tree_serial(s, len);
+    if (c < nchunks) chunk_sums[c] = chunk_sum(run_sums, nd, c);
 }
 
 // Level-by-level pairwise combination of s[0..len) in shared memory (two
@@ -157,18 +98,22 @@ __device__ double tree_reduce(double *a, double *b, int64_t len) {
     return a[0];
 }
 
-// nb constants of c1 are quantized; the mean is S / nb_mean, where S is
-// the tree over nchunks chunk sums (nb_mean = nb unless c1 is one shard of a
-// larger tensor whose chunk sums cover all of it).
+// nb constants of c1 are quantized.  With offset non-NULL the mean is
+// S / nb_mean, S the tree over the sums: run sums of nd_mean runs when
+// sums_are_runs (each CTA folds the chunks itself), else their nchunks chunk
+// sums.  nb_mean = nb unless c1 is one shard of a larger tensor.
 __global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c1, int64_t nb,
-                                                      const double *__restrict__ chunk_sums, int64_t nchunks,
-                                                      int64_t nb_mean, uint8_t *__restrict__ codes,
-                                                      float *__restrict__ absmax2, float *__restrict__ offset) {
+                                                      const double *__restrict__ sums, int64_t nd_mean,
+                                                      int sums_are_runs, int64_t nb_mean,
+                                                      uint8_t *__restrict__ codes, float *__restrict__ absmax2,
+                                                      float *__restrict__ offset) {
     extern __shared__ double s_tree[];  // 2 * nchunks doubles when centring
     __shared__ float s_mu;
     pdl_wait_then_release();
     if (offset != nullptr) {
-        for (int64_t j = threadIdx.x; j < nchunks; j += blockDim.x) s_tree[j] = chunk_sums[j];
+        const int64_t nchunks = (nd_mean + kRunsPerChunk - 1) / kRunsPerChunk;
+        for (int64_t j = threadIdx.x; j < nchunks; j += blockDim.x)
+            s_tree[j] = sums_are_runs ? chunk_sum(sums, nd_mean, j) : sums[j];
         __syncthreads();
         double S = tree_reduce(s_tree, s_tree + nchunks, nchunks);
         if (threadIdx.x == 0) {
@@ -218,67 +163,67 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c
 
 }  // namespace
 
-int64_t dq_chunk_count(int64_t nblocks) {
-    int64_t nd = (nblocks + kDqBlock - 1) / kDqBlock;
-    return (nd + kRunsPerChunk - 1) / kRunsPerChunk;
-}
+int64_t dq_run_count(int64_t nblocks) { return (nblocks + kDqBlock - 1) / kDqBlock; }
+int64_t dq_chunk_count(int64_t nblocks) { return (dq_run_count(nblocks) + kRunsPerChunk - 1) / kRunsPerChunk; }
 
 // Largest chunk count whose tree fits in shared memory (2 buffers of doubles).
 int64_t dq_max_chunks() { return (200 * 1024) / (2 * (int64_t)sizeof(double)); }
 
-cudaError_t launch_double_quantize(const float *absmax, int64_t nb, uint8_t *codes, float *absmax2,
-                                   float *offset, double *chunk_sums, cudaStream_t stream, int num_sms) {
-    if (nb == 0) return cudaSuccess;
-    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
-    const int64_t nchunks = dq_chunk_count(nb);
+// Double quantization of nb constants whose runs' fp64 sums (run_sums, of a
+// tensor of nb_total constants; nb_total > nb for a shard) are already in
+// device memory; chunk_sums: scratch of dq_chunk_count(nb_total) doubles.
+// One launch, two for tensors of more than 64 chunks (2048 runs).
+cudaError_t launch_dq_from_run_sums(const float *absmax, int64_t nb, const double *run_sums, int64_t nb_total,
+                                    uint8_t *codes, float *absmax2, float *offset, double *chunk_sums,
+                                    cudaStream_t stream, int num_sms) {
+    const int64_t nd_total = dq_run_count(nb_total);
+    const int64_t nchunks = dq_chunk_count(nb_total);
     size_t smem = 0;
+    const double *sums = run_sums;
+    int are_runs = 1;
     if (offset != nullptr) {
-        cudaError_t e = launch_pdl(k_dq_chunk_sums, dim3((unsigned)nchunks), dim3(1024), 0, stream, 1, absmax, nb,
-                                   chunk_sums);
-        if (e != cudaSuccess) return e;
+        if (nchunks > kDirectChunks) {
+            cudaError_t e = launch_pdl(k_dq_chunks_from_runs, dim3((unsigned)((nchunks + 255) / 256)), dim3(256), 0,
+                                       stream, 1, run_sums, nd_total, chunk_sums);
+            if (e != cudaSuccess) return e;
+            sums = chunk_sums;
+            are_runs = 0;
+        }
         smem = (size_t)(2 * nchunks) * sizeof(double);
         if (smem > 48 * 1024) {
-            e = cudaFuncSetAttribute(k_dq_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            cudaError_t e = cudaFuncSetAttribute(k_dq_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
         }
     }
-    int64_t want = (nd + 7) / 8;
-    int64_t cap = (int64_t)num_sms * 4;
-    int grid = (int)(want < cap ? want : cap);
-    return launch_pdl(k_dq_quantize, dim3(grid), dim3(256), smem, stream, 1, absmax, nb,
-                      static_cast<const double *>(chunk_sums), nchunks, nb, codes, absmax2, offset);
-}
-
-cudaError_t launch_dq_run_sums(const float *absmax, int64_t nb, double *run_sums, cudaStream_t stream) {
-    if (nb == 0) return cudaSuccess;
-    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
-    return launch_pdl(k_dq_run_sums, dim3((unsigned)((nd + 7) / 8)), dim3(256), 0, stream, 1, absmax, nb, run_sums);
-}
-
-// Double quantization of one shard (nb constants, starting on a run
-// boundary of the whole tensor) with the mean of the whole tensor: the chunk
-// sums are rebuilt from all nd_total run sums, then the shard is quantized
-// with mu = RN_f32(S / nb_total).
-cudaError_t launch_double_quantize_sharded(const float *absmax, int64_t nb, const double *run_sums_all,
-                                           int64_t nd_total, int64_t nb_total, uint8_t *codes, float *absmax2,
-                                           float *offset, double *chunk_sums, cudaStream_t stream, int num_sms) {
-    if (nd_total == 0) return cudaSuccess;
-    const int64_t nchunks = (nd_total + kRunsPerChunk - 1) / kRunsPerChunk;
-    cudaError_t e = launch_pdl(k_dq_chunks_from_runs, dim3((unsigned)((nchunks + 255) / 256)), dim3(256), 0, stream,
-                               1, run_sums_all, nd_total, chunk_sums);
-    if (e != cudaSuccess) return e;
-    const size_t smem = (size_t)(2 * nchunks) * sizeof(double);
-    if (smem > 48 * 1024) {
-        e = cudaFuncSetAttribute(k_dq_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
+    const int64_t nd = dq_run_count(nb);
     int64_t want = (nd + 7) / 8;
     int64_t cap = (int64_t)num_sms * 4;
     int grid = (int)(want < cap ? want : cap);
     if (grid < 1) grid = 1;  // an empty shard still writes mu
-    return launch_pdl(k_dq_quantize, dim3(grid), dim3(256), smem, stream, 1, absmax, nb,
-                      static_cast<const double *>(chunk_sums), nchunks, nb_total, codes, absmax2, offset);
+    return launch_pdl(k_dq_quantize, dim3(grid), dim3(256), smem, stream, 1, absmax, nb, sums, nd_total, are_runs,
+                      nb_total, codes, absmax2, offset);
+}
+
+cudaError_t launch_dq_run_sums(const float *absmax, int64_t nb, double *run_sums, cudaStream_t stream) {
+    if (nb == 0) return cudaSuccess;
+    const int64_t nd = dq_run_count(nb);
+    return launch_pdl(k_dq_run_sums, dim3((unsigned)((nd + 7) / 8)), dim3(256), 0, stream, 1, absmax, nb, run_sums);
+}
+
+// nf4_double_quantize: workspace = run sums (nd doubles) then chunk sums.
+int64_t dq_workspace_bytes(int64_t nblocks) {
+    return (dq_run_count(nblocks) + dq_chunk_count(nblocks)) * (int64_t)sizeof(double);
+}
+
+cudaError_t launch_double_quantize(const float *absmax, int64_t nb, uint8_t *codes, float *absmax2,
+                                   float *offset, double *workspace, cudaStream_t stream, int num_sms) {
+    if (nb == 0) return cudaSuccess;
+    if (offset != nullptr) {
+        cudaError_t e = launch_dq_run_sums(absmax, nb, workspace, stream);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_dq_from_run_sums(absmax, nb, workspace, nb, codes, absmax2, offset, workspace + dq_run_count(nb),
+                                   stream, num_sms);
 }
 
 }  // namespace nf4

@@ -113,7 +113,10 @@ using CfgLarge = TileCfg<NF4_GEMM_BT, NF4_GEMM_STAGES, NF4_GEMM_WG, NF4_GEMM_SUB
 #ifndef NF4_GEMV_TC_STAGES
 #define NF4_GEMV_TC_STAGES 6
 #endif
-using CfgSmall = TileCfg<16, NF4_GEMV_TC_STAGES, NF4_GEMV_TC_WG, 1>;
+#ifndef NF4_GEMV_TC_SUB
+#define NF4_GEMV_TC_SUB 1
+#endif
+using CfgSmall = TileCfg<16, NF4_GEMV_TC_STAGES, NF4_GEMV_TC_WG, NF4_GEMV_TC_SUB>;
 
 template <class C>
 struct __align__(1024) SmemLayout {
@@ -240,7 +243,7 @@ struct TmemPlan {
     static constexpr uint32_t ACol = kAccs * C::AccCols;        // first A column
     static constexpr uint32_t Cols = pow2_at_least(ACol + 32 * C::Sub * C::Stages);
     static_assert(Cols <= 512, "tensor memory: accumulators + 32 columns per A stage");
-    static_assert(!kSK || (C::Sub == 1 && C::BT == 16), "stream-K split: 16-token tile, one k-step per stage");
+    static_assert(!kSK || C::BT == 16, "stream-K split: 16-token tile");
     static_assert(!kSK || C::WG >= 2, "stream-K split: one epilogue warpgroup per segment");
 };
 

@@ -23,6 +23,7 @@
 // packed (every thread reads its 4 code bytes before it writes them), and
 // absmax_out may alias fp32 constants (a block's 8 lanes have read its
 // constant before the shuffles that precede its write).
+#include "mma_util.cuh"
 #include "nf4_encode.cuh"
 
 namespace nf4 {
@@ -94,25 +95,37 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
         }
     }
 
-    // d[i][c]: row 8 warp + i, column 8 lane + c of the tile
-    float d[8][8];
+    // d2[i][h] = (d[i][2h], d[i][2h + 1]): row 8 warp + i, columns 8 lane +
+    // 2h and 8 lane + 2h + 1 of the tile, as packed fp32 pairs.  Each step of
+    // the chain is one fma.rn.f32x2, whose two halves are two independent
+    // binary32 fused multiply-adds (each rounded once, to nearest): exactly the
+    // scalar chain, at half the instructions.
+    uint64_t d2[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) d[i][c] = 0.0f;
+        for (int h = 0; h < 4; ++h) d2[i][h] = 0ull;  // (+0, +0)
     const float4 *a_lane = reinterpret_cast<const float4 *>(sA) + lane;
     const float4 *b_warp = reinterpret_cast<const float4 *>(sB + 8 * warp);
 #pragma unroll 2
     for (int j = 0; j < r; ++j) {
         const float4 a0 = a_lane[j * 64], a1 = a_lane[j * 64 + 32];
         const float4 b0 = b_warp[j * (kMergeBStride / 4)], b1 = b_warp[j * (kMergeBStride / 4) + 1];
-        const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const uint64_t a2[4] = {pack_f32x2(a0.x, a0.y), pack_f32x2(a0.z, a0.w), pack_f32x2(a1.x, a1.y),
+                                pack_f32x2(a1.z, a1.w)};
         const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8; ++i) {
+            const uint64_t bb = pack_f32x2(b[i], b[i]);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) d[i][c] = __fmaf_rn(b[i], a[c], d[i][c]);
+            for (int h = 0; h < 4; ++h) asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d2[i][h]) : "l"(bb), "l"(a2[h]));
+        }
     }
+    float d[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int h = 0; h < 4; ++h) asm("mov.b64 {%0, %1}, %2;" : "=f"(d[i][2 * h]), "=f"(d[i][2 * h + 1]) : "l"(d2[i][h]));
 
 #pragma unroll
     for (int i = 0; i < 8; ++i) {

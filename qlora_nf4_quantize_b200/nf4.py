@@ -55,6 +55,10 @@ def lib() -> ctypes.CDLL:
     L.nf4_double_quantize_workspace_size.argtypes = [i64, i32]
     L.nf4_double_quantize.restype = i32
     L.nf4_double_quantize.argtypes = [P, i64, i32, P, P, P, P, i64, P]
+    L.nf4_quantize_dq_workspace_size.restype = i64
+    L.nf4_quantize_dq_workspace_size.argtypes = [i64, i32, i32]
+    L.nf4_quantize_dq.restype = i32
+    L.nf4_quantize_dq.argtypes = [P, i32, i64, i32, i32, P, P, P, P, P, i64, P]
     L.nf4_dq_run_sums.restype = i32
     L.nf4_dq_run_sums.argtypes = [P, i64, i32, P, P]
     L.nf4_double_quantize_sharded_workspace_size.restype = i64
@@ -157,6 +161,41 @@ def nf4_double_quantize(absmax: torch.Tensor, dq_blocksize: int = DQ_BLOCKSIZE, 
                                    _stream(stream))
     _check("nf4_double_quantize", st)
     return absmax_q, absmax2, offset
+
+
+def nf4_quantize_dq_workspace_size(n: int, blocksize: int = BLOCKSIZE, dq_blocksize: int = DQ_BLOCKSIZE) -> int:
+    return int(lib().nf4_quantize_dq_workspace_size(n, blocksize, dq_blocksize))
+
+
+def nf4_quantize_dq(w: torch.Tensor, centre: bool = True, packed=None, absmax_q=None, absmax2=None, offset=None,
+                    workspace=None, stream=None):
+    """NF4 quantization and double quantization in one call.  Returns
+    (packed uint8[n/2], absmax_q uint8[nb], absmax2 fp32[ceil(nb/256)],
+    offset fp32[1] or None)."""
+    if w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("w must be float32 or bfloat16")
+    _need(w, "w")
+    n = w.numel()
+    nb = (n + BLOCKSIZE - 1) // BLOCKSIZE
+    nd = (nb + DQ_BLOCKSIZE - 1) // DQ_BLOCKSIZE
+    dev = w.device
+    packed = torch.empty(n // 2, dtype=torch.uint8, device=dev) if packed is None else packed
+    absmax_q = torch.empty(nb, dtype=torch.uint8, device=dev) if absmax_q is None else absmax_q
+    absmax2 = torch.empty(nd, dtype=torch.float32, device=dev) if absmax2 is None else absmax2
+    if centre and offset is None:
+        offset = torch.empty(1, dtype=torch.float32, device=dev)
+    if not centre:
+        offset = None
+    _need(packed, "packed", torch.uint8, n // 2)
+    _need(absmax_q, "absmax_q", torch.uint8, nb)
+    _need(absmax2, "absmax2", torch.float32, nd)
+    if workspace is None:
+        workspace = torch.empty(max(16, nf4_quantize_dq_workspace_size(n)), dtype=torch.uint8, device=dev)
+    st = lib().nf4_quantize_dq(_p(w), _BF16 if w.dtype == torch.bfloat16 else _F32, n, BLOCKSIZE, DQ_BLOCKSIZE,
+                               _p(packed), _p(absmax_q), _p(absmax2), _p(offset), _p(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("nf4_quantize_dq", st)
+    return packed, absmax_q, absmax2, offset
 
 
 def nf4_dq_run_sums(absmax: torch.Tensor, dq_blocksize: int = DQ_BLOCKSIZE, out=None, stream=None) -> torch.Tensor:

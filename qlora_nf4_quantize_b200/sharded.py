@@ -45,20 +45,31 @@ def shard_range(n: int, world: int, rank: int) -> Tuple[int, int]:
     return min(r0 * RUN, n), min(r1 * RUN, n)
 
 
-def gather_run_sums(local: torch.Tensor, world: int, group=None) -> torch.Tensor:
+def run_counts(n_total: int, world: int):
+    """Runs (second-level blocks) each rank's shard holds."""
+    out = []
+    for r in range(world):
+        e0, e1 = shard_range(n_total, world, r)
+        out.append(-(-(-(-(e1 - e0) // nf4.BLOCKSIZE)) // nf4.DQ_BLOCKSIZE))
+    return out
+
+
+def gather_run_sums(local: torch.Tensor, world: int, group=None, counts=None) -> torch.Tensor:
     """All-gather the ranks' fp64 run sums, concatenated in rank order.
 
-    Shards hold different run counts, so every rank first learns the counts
-    (one all-gather of an int64), pads its sums to the largest count, takes
-    part in one all-gather and drops the padding."""
+    Shards hold different run counts: each rank pads its sums to the largest
+    count, takes part in one all-gather and drops the padding.  `counts`
+    (each rank's run count, e.g. run_counts()) saves a first all-gather that
+    learns them (and its host synchronisation)."""
     import torch.distributed as dist
     if world == 1:
         return local
     dev = local.device
-    count = torch.tensor([local.numel()], dtype=torch.int64, device=dev)
-    counts = [torch.zeros_like(count) for _ in range(world)]
-    dist.all_gather(counts, count, group=group)
-    counts = [int(c.item()) for c in counts]
+    if counts is None:
+        count = torch.tensor([local.numel()], dtype=torch.int64, device=dev)
+        cl = [torch.zeros_like(count) for _ in range(world)]
+        dist.all_gather(cl, count, group=group)
+        counts = [int(c.item()) for c in cl]
     width = max(max(counts), 1)
     padded = torch.zeros(width, dtype=torch.float64, device=dev)
     padded[:local.numel()] = local
@@ -90,6 +101,7 @@ def quantize_sharded(w_shard: torch.Tensor, n_total: int, world: int, group=None
     gather_run_sums over ``group``).  Returns the shard's QuantState (shape
     (numel,))."""
     packed, absmax, sums = quantize_shard_local(w_shard, stream=stream)
-    all_sums = gather(sums) if gather is not None else gather_run_sums(sums, world, group)
+    all_sums = gather(sums) if gather is not None else gather_run_sums(sums, world, group,
+                                                                        run_counts(n_total, world))
     q8, c2, off = finish_shard(absmax, all_sums, n_total, stream=stream)
     return nf4.QuantState(packed, q8, c2, off, (w_shard.numel(), 1))

@@ -83,8 +83,13 @@ def test_host_validation_before_any_device_work(nf4lib):
 
 def test_workspace_sizes(nf4lib):
     assert nf4lib.nf4_double_quantize_workspace_size(0) == 0
-    assert nf4lib.nf4_double_quantize_workspace_size(2048) == 8          # 8 runs -> 1 chunk of 32
-    assert nf4lib.nf4_double_quantize_workspace_size(256 * 33) == 16     # 33 runs -> 2 chunks
+    # fp64 run sums, then the chunk sums (32 runs each)
+    assert nf4lib.nf4_double_quantize_workspace_size(2048) == (8 + 1) * 8        # 8 runs, 1 chunk
+    assert nf4lib.nf4_double_quantize_workspace_size(256 * 33) == (33 + 2) * 8   # 33 runs, 2 chunks
+    # quantize + DQ in one call: fp32 constants (256-byte aligned), then the same sums
+    assert nf4lib.nf4_quantize_dq_workspace_size(4096 * 4096) == 262144 * 4 + (1024 + 32) * 8
+    assert nf4lib.nf4_quantize_dq_workspace_size(130) == 256 + (1 + 1) * 8
+    assert nf4lib.nf4_quantize_dq_workspace_size(128, 32, 256) == 0
     # up to 16 tokens: [t_hi | t_lo | pad] rows of 64, then (256-byte aligned)
     # the split pipeline's scratch: 192 CTAs x 2 partial tiles of 16 x 128
     # fp32, then 192 arrival counts
@@ -110,4 +115,4 @@ def test_sharded_dq_arguments_checked_on_the_host(nf4lib):
     assert L.nf4_double_quantize_sharded(*args(100, 500, None)) == 1     # the mean must be written
     assert L.nf4_double_quantize_sharded(*args(100, 0, fake)) == 1
     assert L.nf4_double_quantize_sharded(fake, 100, 256, fake, 500, fake, fake, fake, fake, 0, None) == 1
-    assert nf4lib.lib().nf4_double_quantize_sharded_workspace_size(256 * 33, 256) == 16
+    assert nf4lib.lib().nf4_double_quantize_sharded_workspace_size(256 * 33, 256) == 16  # 2 chunk sums

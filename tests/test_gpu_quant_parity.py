@@ -262,3 +262,57 @@ def test_70b_mlp_weight_dequant_sampled_runs(nf4lib, oracle_mod, cuda_device):
         e0, e1 = d * run, (d + 1) * run
         ref = oracle_mod.dequantize(op[e0 // 2:e1 // 2], oq8[e0 // 64:e1 // 64], oc2[d:d + 1], omu, run, "bf16")
         assert np.array_equal(u16(out[e0:e1]), ref), f"run {d} differs"
+
+
+def wide_range_weight(n, seed):
+    """Gaussian weights whose 64-blocks are scaled by 2^U, U uniform in
+    [-40, 8]: the block constants of a run span far more than 2^21, so the
+    fp64 run sums of the centring mean take the sequential order."""
+    g = torch.Generator().manual_seed(seed)
+    w = torch.randn(n, generator=g)
+    nb = -(-n // 64)
+    e = torch.randint(-40, 9, (nb,), generator=g).to(torch.float32)
+    return (w * torch.pow(2.0, e).repeat_interleave(64)[:n]).contiguous()
+
+
+@pytest.mark.parametrize("n,dtype,centre", [(4096 * 4096, "bf16", True), (14336 * 4096, "bf16", True),
+                                            (16384 * 3 + 64 * 5 + 6, "f32", True), (2, "bf16", True),
+                                            (16384 * 2100 + 130, "bf16", True), (256 * 512, "f32", False),
+                                            (16384 * 7 + 4, "wide", True)])
+def test_quantize_dq_one_call(nf4lib, oracle_mod, cuda_device, n, dtype, centre):
+    """nf4_quantize_dq (quantizer writing the run sums, then one double
+    quantization kernel; above 2048 runs a chunk-sum kernel too) against the
+    oracle's quantize + double quantize, bit for bit, outputs and workspace
+    guarded."""
+    if dtype == "wide":
+        w_cpu = wide_range_weight(n, 5)
+    else:
+        w_cpu = wl.weight((n,), 0.02, 40 + n % 1000, "f32", outliers=True)
+        if dtype == "bf16":
+            w_cpu = w_cpu.to(torch.bfloat16)
+    dev = cuda_device
+    nb = -(-n // 64)
+    nd = -(-nb // 256)
+    packed, q8 = guarded(n // 2, torch.uint8, dev), guarded(nb, torch.uint8, dev)
+    c2 = guarded(nd, torch.float32, dev)
+    off = guarded(1, torch.float32, dev) if centre else None
+    ws = guarded(nf4lib.nf4_quantize_dq_workspace_size(n), torch.uint8, dev)
+    nf4lib.nf4_quantize_dq(w_cpu.to(dev), centre=centre, packed=packed, absmax_q=q8, absmax2=c2, offset=off,
+                           workspace=ws)
+    nf4lib.nf4_device_status()
+    check_guards(packed, q8, c2, off, ws)
+    op, oa = oracle_mod.quantize(oracle_input(w_cpu))
+    oq8, oc2, omu = oracle_mod.double_quantize(oa, centre=centre)
+    assert np.array_equal(packed.cpu().numpy(), op)
+    assert np.array_equal(q8.cpu().numpy(), oq8)
+    assert np.array_equal(f32bits(c2.cpu().numpy()), f32bits(oc2))
+    if centre:
+        assert f32bits(off.cpu().numpy())[0] == f32bits([omu])[0]
+    # the fp32 constants passed through the workspace (its first nb words)
+    assert np.array_equal(f32bits(ws[:4 * nb].view(torch.float32).cpu().numpy()), f32bits(oa))
+
+
+def test_quantize_wide_range_constants(nf4lib, oracle_mod, cuda_device):
+    """nf4_quantize and nf4_double_quantize on block constants spanning
+    2^-40 .. 2^8 (sequential fp64 order for the mean)."""
+    run_round_trip(nf4lib, oracle_mod, wide_range_weight(16384 * 5 + 64 * 9 + 2, 6))
