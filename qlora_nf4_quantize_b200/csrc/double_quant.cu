@@ -52,7 +52,26 @@ __device__ __forceinline__ double tree_serial(double *s, int64_t len) {
     return s[0];
 }
 
-// The chunk sum (level-5 node) of runs 32 c .. min(32 c + 32, nd) - 1.
+// The chunk sum (level-5 node) of runs 32 c .. min(32 c + 32, nd) - 1, by
+// one warp (every lane gets it): lane j holds s[j], and each level of the
+// pairwise rule (s[j] = s[2j] + s[2j+1], an odd last element carried up) is
+// two shuffles.
+__device__ __forceinline__ double chunk_sum_warp(const double *__restrict__ run_sums, int64_t nd, int64_t c,
+                                                 int lane) {
+    int len = (int)(nd - c * kRunsPerChunk < kRunsPerChunk ? nd - c * kRunsPerChunk : kRunsPerChunk);
+    double v = lane < len ? run_sums[c * kRunsPerChunk + lane] : 0.0;
+    while (len > 1) {  // len is warp-uniform
+        const int half = len >> 1;
+        const double a = __shfl_sync(0xFFFFFFFFu, v, (2 * lane) & 31);
+        const double b = __shfl_sync(0xFFFFFFFFu, v, (2 * lane + 1) & 31);
+        const double carry = __shfl_sync(0xFFFFFFFFu, v, len - 1);
+        v = lane < half ? a + b : ((len & 1) && lane == half ? carry : 0.0);
+        len = half + (len & 1);
+    }
+    return __shfl_sync(0xFFFFFFFFu, v, 0);
+}
+
+// The chunk sum by one thread (level-by-level rule on a local copy).
 __device__ __forceinline__ double chunk_sum(const double *__restrict__ run_sums, int64_t nd, int64_t c) {
     double s[kRunsPerChunk];
     int64_t len = nd - c * kRunsPerChunk;
@@ -112,8 +131,15 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c
     pdl_wait_then_release();
     if (offset != nullptr) {
         const int64_t nchunks = (nd_mean + kRunsPerChunk - 1) / kRunsPerChunk;
-        for (int64_t j = threadIdx.x; j < nchunks; j += blockDim.x)
-            s_tree[j] = sums_are_runs ? chunk_sum(sums, nd_mean, j) : sums[j];
+        if (sums_are_runs) {  // one warp per chunk
+            const int lane = threadIdx.x & 31;
+            for (int64_t j = threadIdx.x >> 5; j < nchunks; j += blockDim.x >> 5) {
+                const double cs = chunk_sum_warp(sums, nd_mean, j, lane);
+                if (lane == 0) s_tree[j] = cs;
+            }
+        } else {
+            for (int64_t j = threadIdx.x; j < nchunks; j += blockDim.x) s_tree[j] = sums[j];
+        }
         __syncthreads();
         double S = tree_reduce(s_tree, s_tree + nchunks, nchunks);
         if (threadIdx.x == 0) {

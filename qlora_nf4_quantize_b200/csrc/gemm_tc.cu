@@ -79,26 +79,33 @@ constexpr uint32_t pow2_at_least(uint32_t v) {
 // the SMs.
 constexpr uint32_t AccColsFor(int bt) { return bt < 32 ? 32u : (uint32_t)bt; }
 
-template <int BT_, int STAGES_, int WG_, int SUB_>
+template <int BT_, int STAGES_, int WG_, int SUB_, bool PAIR_ = false>
 struct TileCfg {
     static constexpr int BT = BT_, Stages = STAGES_, WG = WG_;
+    // CTA pair (cta_group::2): the two CTAs of a 2-CTA cluster own weight
+    // tiles 2p and 2p + 1 and the same token tile; the even CTA issues MMAs
+    // of M = 256 (its 128 rows and its partner's, each in its own tensor
+    // memory) against the whole token tile, of which each CTA loads half.
+    static constexpr bool Pair = PAIR_;
+    static constexpr int XRows = PAIR_ ? BT_ / 2 : BT_;  // tokens of the x tile this CTA loads
     // k-steps of 64 per pipeline stage: the stage's barriers, its TMA
     // transaction and its MMA issue are shared by SUB k-steps
     static constexpr int Sub = SUB_;
     static constexpr int Threads = 128 + 128 * WG;
     // two CTAs per SM when both fit (registers at 128 per thread, tensor
     // memory at 256 columns each)
-    static constexpr int MinBlocks = (Threads <= 256 && AccColsFor(BT_) + 32 * SUB_ * STAGES_ <= 256) ? 2 : 1;
+    static constexpr int MinBlocks =
+        (!PAIR_ && Threads <= 256 && AccColsFor(BT_) + 32 * SUB_ * STAGES_ <= 256) ? 2 : 1;
     static constexpr uint32_t AccCols = AccColsFor(BT);     // accumulator: columns [0, AccCols)
     // A of k-step j of stage s: columns [ACol + 32 (Sub s + j), +32)
     static constexpr uint32_t ACol = AccCols;
     static constexpr uint32_t TmemCols = pow2_at_least(AccCols + 32 * Sub * Stages);
-    static constexpr uint32_t XSubBytes = BT * kBK * 2;     // one 64-wide k-step of x
+    static constexpr uint32_t XSubBytes = XRows * kBK * 2;  // one 64-wide k-step of (this CTA's part of) x
     static constexpr uint32_t XStageBytes = Sub * XSubBytes;
     // UMMA instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both
-    // K-major, N = BT, M = 128.
+    // K-major, N = BT, M = 128 (256 for a pair).
     static constexpr uint32_t Idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BT >> 3) << 17) |
-                                      ((uint32_t)(kBN >> 4) << 24);
+                                      ((uint32_t)((PAIR_ ? 2 * kBN : kBN) >> 4) << 24);
     static_assert(TmemCols <= 512, "tensor memory: accumulator + 32 columns per A stage");
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M = 128");
 };
@@ -107,6 +114,21 @@ struct TileCfg {
 #define NF4_GEMM_BT 256
 #endif
 using CfgLarge = TileCfg<NF4_GEMM_BT, NF4_GEMM_STAGES, NF4_GEMM_WG, NF4_GEMM_SUB>;
+// Large-M calls on CTA pairs (cta_group::2) instead of single CTAs.  Exact
+// (every linear parity test passes with it) but not the default: on B200 the
+// training shape took 573.5 us against 430.6 us for single CTAs (six
+// stages): the pair halves the MMA instructions and each CTA's share of the
+// token tile, but every stage then waits for the slower of two SMs' dequant
+// warps and for the remote arrivals, while each SM still dequantizes a whole
+// 128-row tile per token tile.
+#ifndef NF4_GEMM_PAIR
+#define NF4_GEMM_PAIR 0
+#endif
+#ifndef NF4_GEMM_PAIR_STAGES
+#define NF4_GEMM_PAIR_STAGES 6
+#endif
+using CfgPair = TileCfg<256, NF4_GEMM_PAIR_STAGES, 3, 1, true>;
+static_assert(CfgPair::Stages * CfgPair::XStageBytes >= 256 * 128 * 2, "the y staging tile fits in the x ring");
 #ifndef NF4_GEMV_TC_WG
 #define NF4_GEMV_TC_WG 3
 #endif
@@ -141,6 +163,19 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The same MMA for a CTA pair (issued by the even CTA): A from both CTAs'
+// tensor memory (same address), B from both CTAs' shared memory (same
+// offset, each holding half of the N rows), D in both CTAs' tensor memory.
+__device__ __forceinline__ void tc_mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -270,6 +305,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
               float *__restrict__ partials, unsigned *__restrict__ counts, unsigned *err) {
     extern __shared__ uint8_t smem_raw[];
     constexpr int kBT = C::BT, kStages = C::Stages, kWG = C::WG, kSub = C::Sub;
+    constexpr bool kPair = C::Pair;
+    static_assert(!(kPair && kSK), "a CTA pair runs whole tiles");
     constexpr uint32_t kTmemCols = TmemPlan<C, kSK>::Cols, kAccCol = 0, kACol = TmemPlan<C, kSK>::ACol,
                        kXSubBytes = C::XSubBytes, kXStageBytes = C::XStageBytes;
     SmemLayout<C> &S =
@@ -308,9 +345,13 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     if (!kSK && r <= 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
+    // CTA pair: rank 0 issues the MMAs and owns the full barriers, which
+    // count its own and its partner's dequant arrivals
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const bool issuer = rank == 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&S.full[s], 1 + 128);
+            mbar_init(&S.full[s], 1 + 128 * (kPair ? 2 : 1));
             mbar_init(&S.empty[s], 1);
         }
         mbar_init(&S.acc_full, 1);
@@ -321,13 +362,24 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     }
     if constexpr (kLutMask != 0) fill_pair_table(S.pairs);
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&S.tmem_base)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (kPair) {  // the same warp of both CTAs: one address, valid in both
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_addr(&S.tmem_base)),
+                         "r"(kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_addr(&S.tmem_base)),
+                         "r"(kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    // a pair: both CTAs' barriers are initialised before either signals the other's
+    if constexpr (kPair) cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
 
@@ -351,19 +403,35 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
             }
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.empty[s], ph ^ 1u, abort, err))) break;
             if (leader) {
-                mbar_arrive_expect_tx(&S.full[s], (uint32_t)nsub * kXSubBytes);
-                for (int j = 0; j < nsub; ++j) {
-                    const int kt = kt_of(i0 + j);
-                    uint8_t *dst = S.x[s] + j * kXSubBytes;
-                    if (kt < kw_steps) tma_load_2d(dst, &tmap_x, &S.full[s], kt * kBK, (int)m0);
-                    else tma_load_2d(dst, &tmap_t, &S.full[s], (kt - kw_steps) * kBK, (int)m0);
+                if constexpr (kPair) {
+                    // each CTA loads its half of the token tile; the bytes of
+                    // both halves are counted on the even CTA's full barrier
+                    if (issuer) mbar_arrive_expect_tx(&S.full[s], 2u * (uint32_t)nsub * kXSubBytes);
+                    const uint32_t bar = cluster_addr(&S.full[s], 0);
+                    const int row = (int)m0 + (int)rank * C::XRows;
+                    for (int j = 0; j < nsub; ++j) {
+                        const int kt = kt_of(i0 + j);
+                        uint8_t *dst = S.x[s] + j * kXSubBytes;
+                        if (kt < kw_steps) tma_load_2d_pair(dst, &tmap_x, bar, kt * kBK, row);
+                        else tma_load_2d_pair(dst, &tmap_t, bar, (kt - kw_steps) * kBK, row);
+                    }
+                } else {
+                    mbar_arrive_expect_tx(&S.full[s], (uint32_t)nsub * kXSubBytes);
+                    for (int j = 0; j < nsub; ++j) {
+                        const int kt = kt_of(i0 + j);
+                        uint8_t *dst = S.x[s] + j * kXSubBytes;
+                        if (kt < kw_steps) tma_load_2d(dst, &tmap_x, &S.full[s], kt * kBK, (int)m0);
+                        else tma_load_2d(dst, &tmap_t, &S.full[s], (kt - kw_steps) * kBK, (int)m0);
+                    }
                 }
             }
             __syncwarp();
             issued = g + 1;
         }
-        // drain: every issued load has landed before the CTA may exit
-        if (leader) {
+        // drain: every issued load has landed before the CTA may exit (a
+        // pair's loads complete on the even CTA's barriers: its MMA issuer
+        // drains them, and the cluster barrier at the end holds both CTAs)
+        if (leader && (!kPair || issuer)) {
             for (int g = issued - kStages < 0 ? 0 : issued - kStages; g < issued; ++g) {
                 const int s = g % kStages;
                 const uint32_t ph = (uint32_t)(g / kStages) & 1u;
@@ -373,7 +441,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == 1 && issuer) {
         // ---------------- MMA issuer ----------------
         // The whole warp runs the loop (its values stay warp-uniform); one
         // elected lane issues the MMAs and the commits.
@@ -391,7 +459,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
             for (int s = 0; s < kStages; ++s) {
                 const int g = g0 + s;
                 if (g >= kg_total) break;
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.full[s], ph, abort, err))) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait<kPair>(&S.full[s], ph, abort, err))) {
                     stop = true;
                     break;
                 }
@@ -405,22 +473,35 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                             const uint32_t acol = tmem + kACol + 32u * (uint32_t)(kSub * s + j);
                             // the first step of each segment starts its accumulator
                             const uint32_t dcol = tmem + kAccCol + C::AccCols * (uint32_t)seg_of(i);
-                            tc_mma_ts(dcol, acol, bdesc, C::Idesc, (i != 0 && i != i_next) ? 1u : 0u);
+                            if constexpr (kPair) {
+                                tc_mma_ts_pair(dcol, acol, bdesc, C::Idesc, i != 0 ? 1u : 0u);
 #pragma unroll
-                            for (int kk = 1; kk < kBK / 16; ++kk)
-                                tc_mma_ts(dcol, acol + 8u * kk, bdesc + 2ull * kk, C::Idesc, 1u);
+                                for (int kk = 1; kk < kBK / 16; ++kk)
+                                    tc_mma_ts_pair(dcol, acol + 8u * kk, bdesc + 2ull * kk, C::Idesc, 1u);
+                            } else {
+                                tc_mma_ts(dcol, acol, bdesc, C::Idesc, (i != 0 && i != i_next) ? 1u : 0u);
+#pragma unroll
+                                for (int kk = 1; kk < kBK / 16; ++kk)
+                                    tc_mma_ts(dcol, acol + 8u * kk, bdesc + 2ull * kk, C::Idesc, 1u);
+                            }
                         }
                     }
-                    tc_commit(&S.empty[s]);
+                    // stage s is free again in both CTAs of a pair
+                    if constexpr (kPair) tc_commit_pair(&S.empty[s], 0x3);
+                    else tc_commit(&S.empty[s]);
                 }
                 __syncwarp();
                 any = true;
             }
         }
         if (leader) {
-            if (any && !stop) tc_commit(&S.acc_full);
+            if (any && !stop) {
+                if constexpr (kPair) tc_commit_pair(&S.acc_full, 0x3);
+                else tc_commit(&S.acc_full);
+            }
             if (any && *abort) {  // drain our own MMAs before tensor memory is released
-                tc_commit(&S.drain);
+                if constexpr (kPair) tc_commit_pair(&S.drain, 0x1);
+                else tc_commit(&S.drain);
                 unsigned long long t0 = global_ns();
                 while (!mbar_try_wait(&S.drain, 0) && global_ns() - t0 < kWaitLimitNs) {
                 }
@@ -489,7 +570,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                 }
                 if (!ok) break;
                 tc_fence_before();
-                mbar_arrive(&S.full[s]);
+                if constexpr (kPair) mbar_arrive_cluster(cluster_addr(&S.full[s], 0));
+                else mbar_arrive(&S.full[s]);
             }
         }
         if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full, 0, abort, err));
@@ -573,10 +655,16 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     }
     tc_fence_before();
     __syncthreads();
+    // a pair: neither CTA releases its tensor memory (read by the pair's
+    // MMAs) or leaves (its shared memory is the pair's B operand) before the other is done
+    if constexpr (kPair) cluster_sync_all();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        if constexpr (kPair)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
@@ -590,15 +678,21 @@ cudaError_t launch_mode(const CUtensorMap &mx, const CUtensorMap &mt, const CUte
         cudaFuncSetAttribute(k_gemm_tc<kMode, C, kSK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = kSK ? dim3((unsigned)ctas) : dim3((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + C::BT - 1) / C::BT));
+    int64_t tiles = (N + kBN - 1) / kBN;
+    if (C::Pair) tiles = (tiles + 1) & ~(int64_t)1;  // whole pairs (a last odd tile's partner has no rows)
+    cfg.gridDim = kSK ? dim3((unsigned)ctas) : dim3((unsigned)tiles, (unsigned)((M + C::BT - 1) / C::BT));
     cfg.blockDim = dim3(C::Threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = C::Pair ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, k_gemm_tc<kMode, C, kSK>, mx, mt, my, M, K, N, packed, q8, scales, offset, Bl, r,
                               rp, y, partials, counts, err);
 }
@@ -609,10 +703,10 @@ cudaError_t launch_cfg(const void *x, int64_t M, int64_t K, int64_t N, const uin
                        void *y, float *partials, unsigned *counts, int ctas, cudaStream_t stream,
                        unsigned *err_word) {
     CUtensorMap mx, mt, my;
-    cudaError_t e = make_map(&mx, x, M, K, kBK, C::BT, true);
+    cudaError_t e = make_map(&mx, x, M, K, kBK, C::XRows, true);
     if (e != cudaSuccess) return e;
-    if (r > 0) e = make_map(&mt, t2, M, rp, kBK, C::BT, true);
-    else e = make_map(&mt, x, M, K, kBK, C::BT, true);  // unused: no extension steps
+    if (r > 0) e = make_map(&mt, t2, M, rp, kBK, C::XRows, true);
+    else e = make_map(&mt, x, M, K, kBK, C::XRows, true);  // unused: no extension steps
     if (e != cudaSuccess) return e;
     e = make_map(&my, y, M, N, kBN, C::BT, false);
     if (e != cudaSuccess) return e;
@@ -668,23 +762,6 @@ struct __align__(1024) DownSmem {
 };
 static_assert(kDownStages * kDownRows * 128 >= 64 * kDownRows * 4, "partial tile fits in the x ring");
 
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// address of the same shared-memory location in cluster CTA `rank`
-__device__ __forceinline__ uint32_t map_rank(const void *p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
-    return r;
-}
-
 __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -708,7 +785,7 @@ __global__ void __launch_bounds__(128, 1)
     pdl_wait_then_release();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_rank();
+    const uint32_t rank = cluster_ctarank();
     const int64_t m0 = (int64_t)blockIdx.y * kDownRows;
     const int kt_all = (int)((K + 63) / 64);  // a partial last step reads zeros beyond K (TMA fill)
     const int kt_begin = (int)((int64_t)rank * kt_all / kSplit);
@@ -810,7 +887,7 @@ __global__ void __launch_bounds__(128, 1)
         const int cb = (t / kRowsPer) * kCw;
         uint32_t base[kSplit];
 #pragma unroll
-        for (int c = 0; c < kSplit; ++c) base[c] = map_rank(part + cb * kDownRows + r_loc, (uint32_t)c);
+        for (int c = 0; c < kSplit; ++c) base[c] = cluster_addr(part + cb * kDownRows + r_loc, (uint32_t)c);
 #pragma unroll 1
         for (int j0 = 0; j0 < kCw; j0 += 4) {
             float v[4];
@@ -902,6 +979,9 @@ cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const
         return launch_cfg<CfgSmall, false>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, nullptr, nullptr,
                                            0, stream, err_word);
     }
+    if (NF4_GEMM_PAIR)
+        return launch_cfg<CfgPair, false>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, nullptr, nullptr,
+                                          0, stream, err_word);
     return launch_cfg<CfgLarge, false>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, nullptr, nullptr, 0,
                                        stream, err_word);
 }

@@ -62,16 +62,33 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
     return ok != 0;
 }
 
+// As mbar_try_wait_sleep, with acquire semantics at cluster scope: the
+// phase may have been completed by arrivals (release, cluster scope) of
+// threads in another CTA of the cluster.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(100000u)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: true when the phase completed; false after limit_ns of
 // %globaltimer (abort raised, bit 0 of the error word set) or when another
 // role already aborted.  Every kernel waits with the default limit; the
-// failure-detection self-test passes a short one.
+// failure-detection self-test passes a short one.  kCluster: acquire at
+// cluster scope (arrivals from the other CTA of a pair).
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err,
                                           unsigned long long limit_ns = kWaitLimitNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
         if (global_ns() - t0 > limit_ns) {
             *abort = 1;
