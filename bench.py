@@ -15,6 +15,9 @@ One step is one pass over every call of the path on per-GPU synthetic inputs
   - 70B MLP GEMM, x[2048, 8192], W 28672x8192, r = 16, s = 2;
   - one 8B-shaped decoder layer's seven weights: quantize + double-quantize +
     dequantize (the whole-model sweep is 32 such layers);
+  - the same layer's seven linears at M = 4096 tokens, r = 64, through the
+    fused NF4 path, and as unquantized bf16 LoRA GEMMs on cuBLAS (the
+    comparison behind `overhead_vs_bf16_lora`; not this library's kernels);
   - backward (dx, dA, dB) and merge + requantize of the training GEMM.
 Each call is captured R times back to back in a CUDA graph, its inputs
 rotating over copies larger than the 126 MB L2 (no call reads a warm input),
@@ -51,8 +54,9 @@ BYTES_PER_PARAM_DQ = 0.5 + 1 / 64 + 4 / 16384
 WORKLOAD = ("every call of the path, each replayed back to back: projection 4096x4096 bf16 (0.1% x10 outliers) "
             "quantize, double-quantize, quantize+DQ, dequantize to bf16 (headline value) / fp32 / bf16 without DQ; "
             "decode GEMV x[T,4096] T=1,4,16, W 11008x4096 r=16; training GEMM x[4096,4096] W 14336x4096 r=64; "
-            "70B MLP GEMM x[2048,8192] W 28672x8192 r=16; one 8B-shaped layer's 7 weights quantize+DQ+dequantize; "
-            "backward and merge+requantize of the training GEMM")
+            "70B MLP GEMM x[2048,8192] W 28672x8192 r=16; one 8B-shaped layer's 7 weights quantize+DQ+dequantize "
+            "and its 7 linears at M=4096 r=64 (vs bf16 LoRA on cuBLAS); backward and merge+requantize of the "
+            "training GEMM")
 
 
 # ------------------------------------------------------------------ algorithmic work per call
@@ -250,6 +254,7 @@ def build_segments(q, wl, dev, rank, world):
     for c, tag in ((wl.GEMM_TRAIN, "gemm_M4096"), (wl.GEMM_70B_MLP, "gemm_70B_M2048")):
         _gemm_segment(q, wl, dev, rank, segs, c, tag)
     _sweep_segment(q, wl, dev, segs)
+    _layer_linear_segments(q, wl, dev, rank, segs)
     _bwd_merge_segments(q, wl, dev, rank, segs)
     torch.cuda.synchronize()
     return segs, wp, state
@@ -381,6 +386,44 @@ def _sweep_segment(q, wl, dev, segs):
                         "the 7 linear weights of one 8B-shaped decoder layer (218.1 M params): nf4_quantize_dq + "
                         "nf4_dequantize (bf16); the sweep is 32 such layers"))
 
+
+
+def _layer_linear_segments(q, wl, dev, rank, segs):
+    """Next row 4: the seven linears of one 8B-shaped decoder layer at M =
+    4096 tokens, r = 64, s = 0.25 through the fused NF4 path, and the same
+    linears as unquantized bf16 LoRA GEMMs on cuBLAS (torch.matmul; timed for
+    the overhead figure only, not counted as this library's launches)."""
+    import torch
+    M, r, sc = 4096, 64, 0.25
+    nf4_fns, bf16_fns, flops = [], [], 0
+    for idx, (name, N, K) in enumerate(wl.LAYER_8B):
+        W = wl.sweep_weight(0, idx).to(dev)
+        g = torch.Generator().manual_seed(rank_seed(wl.sweep_seed(0, idx) + 1, rank))
+        x = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
+        A = (torch.randn(r, K, generator=g) * 0.01).to(torch.bfloat16).to(dev)
+        B = (torch.randn(N, r, generator=g) * 0.01).to(torch.bfloat16).to(dev)
+        st = q.quantize_weight(W)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(q.nf4_lora_linear_workspace_size(M, r), dtype=torch.uint8, device=dev)
+        nf4_fns.append(lambda x=x, st=st, N=N, A=A, B=B, y=y, ws=ws: q.nf4_lora_linear_fwd(
+            x, st.packed, st.absmax_q, st.absmax2, st.offset, N, A, B, sc, y=y, workspace=ws))
+        Wt, At, Bt = W.t(), A.t(), B.t()
+        yb = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        bf16_fns.append(lambda x=x, Wt=Wt, At=At, Bt=Bt, yb=yb: torch.addmm(torch.matmul(x, Wt), torch.matmul(x, At),
+                                                                             Bt, alpha=sc, out=yb))
+        flops += linear_flops(M, K, N, r)
+
+    def f_nf4():
+        for f in nf4_fns:
+            f()
+
+    def f_bf16():
+        for f in bf16_fns:
+            f()
+    cfg = f"the 7 linears of one 8B-shaped decoder layer, M = {M} tokens, r = {r}, s = {sc}"
+    segs.append(Segment("layer_8B_linears", [f_nf4], 1, flops, "TFLOP/s", 2 * len(nf4_fns), cfg + ", fused NF4+LoRA"))
+    segs.append(Segment("layer_8B_linears_bf16_cublas", [f_bf16], 1, flops, "TFLOP/s", 0,
+                        cfg + ", unquantized bf16 LoRA GEMMs on cuBLAS (comparison, not this library)"))
 
 
 def _bwd_merge_segments(q, wl, dev, rank, segs):
@@ -530,6 +573,9 @@ def run_ours(args):
             e["sweep_32_layers_s"] = round(us * wl.N_LAYERS_8B * 1e-6, 5)
         kernels.append(e)
         by[s.name] = e
+    if "layer_8B_linears" in by and "layer_8B_linears_bf16_cublas" in by:
+        by["layer_8B_linears"]["overhead_vs_bf16_lora"] = round(
+            by["layer_8B_linears"]["us"] / by["layer_8B_linears_bf16_cublas"]["us"] - 1, 4)
     launches = sum(s.reps * s.launches for s in segs + eager) * K
 
     if rank != 0:

@@ -36,6 +36,7 @@
 // producer drains its own loads, and tensor memory is released before the
 // CTA exits.  nf4_device_status() reports the expiry as NF4_ERR_TIMEOUT.
 #include "mma_util.cuh"
+#include "streamk.h"
 #include "tc_util.cuh"
 
 namespace nf4 {
@@ -114,6 +115,12 @@ struct TileCfg {
 #define NF4_GEMM_BT 256
 #endif
 using CfgLarge = TileCfg<NF4_GEMM_BT, NF4_GEMM_STAGES, NF4_GEMM_WG, NF4_GEMM_SUB>;
+// How the MMA-issuing thread waits for a stage (mbar_wait kPoll).
+#ifndef NF4_MMA_POLL
+#define NF4_MMA_POLL 0
+#endif
+constexpr int kMmaPoll = NF4_MMA_POLL;
+
 // Large-M calls on CTA pairs (cta_group::2) instead of single CTAs.  Exact
 // (every linear parity test passes with it) but not the default: on B200 the
 // training shape took 573.5 us against 430.6 us for single CTAs (six
@@ -289,11 +296,6 @@ constexpr int kPartialFloats = 16 * 128;
 constexpr int kStreamKMaxCtas = 192;
 constexpr int kStreamKMinSteps = 8;
 
-// CTA of a split launch of `ctas` CTAs whose range holds global step s of
-// `total`: the largest c with c total / ctas <= s.
-__device__ __forceinline__ int64_t streamk_cta_of(int64_t s, int64_t total, int64_t ctas) {
-    return (s * ctas + ctas - 1) / total;
-}
 
 template <int kMode, class C, bool kSK>
 __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
@@ -324,8 +326,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     int kt_first = 0, steps = kt_total, i_next = kt_total;
     if constexpr (kSK) {
         total = ((N + kBN - 1) / kBN) * kt_total;
-        const int64_t lo = (int64_t)blockIdx.x * total / gridDim.x;
-        const int64_t hi = (int64_t)(blockIdx.x + 1) * total / gridDim.x;
+        const int64_t lo = nf4_sk_begin(blockIdx.x, total, gridDim.x);
+        const int64_t hi = nf4_sk_begin(blockIdx.x + 1, total, gridDim.x);
         tile0 = lo / kt_total;
         kt_first = (int)(lo - tile0 * kt_total);
         steps = (int)(hi - lo);
@@ -459,7 +461,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
             for (int s = 0; s < kStages; ++s) {
                 const int g = g0 + s;
                 if (g >= kg_total) break;
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait<kPair>(&S.full[s], ph, abort, err))) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait<kPair, kMmaPoll>(&S.full[s], ph, abort, err))) {
                     stop = true;
                     break;
                 }
@@ -487,8 +489,12 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                         }
                     }
                     // stage s is free again in both CTAs of a pair
-                    if constexpr (kPair) tc_commit_pair(&S.empty[s], 0x3);
-                    else tc_commit(&S.empty[s]);
+                    if constexpr (kPair) {
+                        tc_commit_pair(cluster_addr(&S.empty[s], 0));
+                        tc_commit_pair(cluster_addr(&S.empty[s], 1));
+                    } else {
+                        tc_commit(&S.empty[s]);
+                    }
                 }
                 __syncwarp();
                 any = true;
@@ -496,11 +502,15 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         }
         if (leader) {
             if (any && !stop) {
-                if constexpr (kPair) tc_commit_pair(&S.acc_full, 0x3);
-                else tc_commit(&S.acc_full);
+                if constexpr (kPair) {
+                    tc_commit_pair(cluster_addr(&S.acc_full, 0));
+                    tc_commit_pair(cluster_addr(&S.acc_full, 1));
+                } else {
+                    tc_commit(&S.acc_full);
+                }
             }
             if (any && *abort) {  // drain our own MMAs before tensor memory is released
-                if constexpr (kPair) tc_commit_pair(&S.drain, 0x1);
+                if constexpr (kPair) tc_commit_pair(cluster_addr(&S.drain, 0));
                 else tc_commit(&S.drain);
                 unsigned long long t0 = global_ns();
                 while (!mbar_try_wait(&S.drain, 0) && global_ns() - t0 < kWaitLimitNs) {
@@ -594,8 +604,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                 if (row_in_tile == 0) {
                     // the counts were zeroed by the grid before this one
                     asm volatile("griddepcontrol.wait;" ::: "memory");
-                    const int64_t c0 = streamk_cta_of(tile * kt_total, total, gridDim.x);
-                    const int64_t c1 = streamk_cta_of(tile * kt_total + kt_total - 1, total, gridDim.x);
+                    const int64_t c0 = nf4_sk_owner(tile * kt_total, total, gridDim.x);
+                    const int64_t c1 = nf4_sk_owner(tile * kt_total + kt_total - 1, total, gridDim.x);
                     const unsigned prev = atomicAdd(counts + tile, 1u);
                     S.last[h] = prev == (unsigned)(c1 - c0);
                 }
@@ -603,14 +613,14 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
                 if (S.last[h]) {
                     // every partial of the tile is in: add them in CTA order
                     __threadfence();
-                    const int64_t c0 = streamk_cta_of(tile * kt_total, total, gridDim.x);
-                    const int64_t c1 = streamk_cta_of(tile * kt_total + kt_total - 1, total, gridDim.x);
+                    const int64_t c0 = nf4_sk_owner(tile * kt_total, total, gridDim.x);
+                    const int64_t c1 = nf4_sk_owner(tile * kt_total + kt_total - 1, total, gridDim.x);
                     float acc[16];
 #pragma unroll
                     for (int m = 0; m < 16; ++m) acc[m] = 0.0f;
                     for (int64_t c = c0; c <= c1; ++c) {
                         // segment 0 when CTA c's range starts in this tile, else 1
-                        const int seg = (c * total / gridDim.x) / kt_total == tile ? 0 : 1;
+                        const int seg = nf4_sk_segment(c, tile, kt_total, total, gridDim.x);
                         const float *src = partials + (2 * c + seg) * kPartialFloats + row_in_tile;
 #pragma unroll
                         for (int m = 0; m < 16; ++m) acc[m] += __ldcg(src + m * 128);

@@ -31,7 +31,7 @@ __device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
 
 // TMA 2-D load into this CTA's shared memory whose completion (transaction
 // bytes) is counted on the barrier at shared::cluster address `bar_leader`
-// (the even CTA's).  No multicast: each CTA loads its own half of the operand.
+// (the even CTA's); each CTA loads only its own half of the operand.
 __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint32_t bar_leader, int c0,
                                                  int c1) {
     asm volatile(
@@ -48,13 +48,10 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
 }
 
 // Commit of the pair's MMAs issued so far: one arrival on the barrier at
-// offset `bar` in each CTA of cta_mask (bit r = CTA rank r).
-__device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t cta_mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_addr(bar)),
-        "h"(cta_mask)
-        : "memory");
+// shared::cluster address `bar` (this CTA's or its partner's) once they have
+// completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
