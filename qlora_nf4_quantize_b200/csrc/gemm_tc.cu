@@ -115,12 +115,6 @@ struct TileCfg {
 #define NF4_GEMM_BT 256
 #endif
 using CfgLarge = TileCfg<NF4_GEMM_BT, NF4_GEMM_STAGES, NF4_GEMM_WG, NF4_GEMM_SUB>;
-// How the MMA-issuing thread waits for a stage (mbar_wait kPoll).
-#ifndef NF4_MMA_POLL
-#define NF4_MMA_POLL 0
-#endif
-constexpr int kMmaPoll = NF4_MMA_POLL;
-
 // Large-M calls on CTA pairs (cta_group::2) instead of single CTAs.  Exact
 // (every linear parity test passes with it) but not the default: on B200 the
 // training shape took 573.5 us against 430.6 us for single CTAs (six
@@ -461,7 +455,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
             for (int s = 0; s < kStages; ++s) {
                 const int g = g0 + s;
                 if (g >= kg_total) break;
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait<kPair, kMmaPoll>(&S.full[s], ph, abort, err))) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait<kPair>(&S.full[s], ph, abort, err))) {
                     stop = true;
                     break;
                 }

@@ -62,19 +62,6 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
     return ok != 0;
 }
 
-// Non-blocking test of the phase (no suspension).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // As mbar_try_wait_sleep, with acquire semantics at cluster scope: the
 // phase may have been completed by arrivals (release, cluster scope) of
 // threads in another CTA of the cluster.
@@ -95,21 +82,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 // role already aborted.  Every kernel waits with the default limit; the
 // failure-detection self-test passes a short one.  kCluster: acquire at
 // cluster scope (arrivals from the other CTA of a pair).
-// kPoll: 0 = suspend between polls (try_wait with a 0.1 ms hint; the
-// thread is woken when the phase completes), 1 = try_wait without a hint,
-// 2 = spin on test_wait (no suspension at all).
-template <bool kCluster = false, int kPoll = 0>
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err,
                                           unsigned long long limit_ns = kWaitLimitNs) {
     if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-        bool done;
-        if (kCluster) done = mbar_try_wait_cluster(bar, parity);
-        else if (kPoll == 2) done = mbar_test_wait(bar, parity);
-        else if (kPoll == 1) done = mbar_try_wait(bar, parity);
-        else done = mbar_try_wait_sleep(bar, parity);
-        if (done) return true;
+        if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
         if (global_ns() - t0 > limit_ns) {
             *abort = 1;

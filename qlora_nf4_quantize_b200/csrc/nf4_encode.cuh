@@ -26,6 +26,12 @@ constexpr float kAmbiguity = 0x1p-18f;
 constexpr int kCells = 129;      // cells 0..128 cover q in [-1, 1]
 constexpr int kCellTable = 256;  // indexed by the low byte of RN(64 q) + 64 (+ 1.5 * 2^23)
 
+// 1: the compare q > t is taken from the sign of t - q, the difference the
+// ambiguity test needs anyway
+#ifndef NF4_ENCODE_SIGN
+#define NF4_ENCODE_SIGN 0
+#endif
+
 #ifndef NF4_QUANT_RCP_APPROX
 #define NF4_QUANT_RCP_APPROX 1
 #endif
@@ -98,9 +104,18 @@ __device__ __forceinline__ uint32_t encode8(const float v[8], float c1, const fl
                 // mask keeps any input inside the 256-entry table
                 const uint32_t e = s_cell[__float_as_uint(f[j]) & 0xFFu];
                 const float t = __uint_as_float(e);
+#if NF4_ENCODE_SIGN
+                // d = RN(t - q) is negative exactly when q > t (a nonzero
+                // difference of two finite binary32 values in [-4, 4] never
+                // rounds to zero, and t - t = +0): its sign bit is the compare
+                const float d = t - q[j];
+                word = (word << 4) + (e & 15u) + (__float_as_uint(d) >> 31);
+                dmin = fminf(dmin, fabsf(d));
+#else
                 const uint32_t code = (e & 15u) + ((q[j] > t) ? 1u : 0u);
                 word = (word << 4) | code;
                 dmin = fminf(dmin, fabsf(q[j] - t));
+#endif
             }
         }
         amb = dmin <= kAmbiguity;  // rare: some quotient is within 2^-18 of a threshold
