@@ -29,7 +29,7 @@ constexpr int kCellTable = 256;  // indexed by the low byte of RN(64 q) + 64 (+ 
 // 1: the compare q > t is taken from the sign of t - q, the difference the
 // ambiguity test needs anyway
 #ifndef NF4_ENCODE_SIGN
-#define NF4_ENCODE_SIGN 0
+#define NF4_ENCODE_SIGN 1
 #endif
 
 #ifndef NF4_QUANT_RCP_APPROX
