@@ -10,9 +10,9 @@ namespace nf4 {
 int lora_rp(int r);
 cudaError_t launch_lora_down(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2,
                              unsigned *counts, int ncounts, cudaStream_t stream);
-cudaError_t launch_gemv(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
-                        const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
-                        void *y, cudaStream_t stream, int num_sms);
+cudaError_t launch_decode(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
+                          const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
+                          void *y, unsigned *err, cudaStream_t stream, int num_sms);
 cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
                                 unsigned *err, cudaStream_t stream, int split);
 cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
@@ -25,14 +25,13 @@ int streamk_ctas(int64_t M, int64_t K, int64_t N, int rp, int sms);
 
 constexpr int kGemvMaxTokens = 16;
 // Token counts from which decode-size calls take the tcgen05 pipeline with a
-// 16-token tile instead of the warp-MMA GEMV kernels: that pipeline takes
-// the same time for any count up to 16 (split over the SMs, 25.1 us without
-// LoRA on an 11008 x 4096 weight), the warp-MMA kernels grow with it (16.5
-// us at 1 token, 21.7 at 8, 27.5 at 12, 30.3 at 16: above 8 tokens they need
-// two token tiles).
+// 16-token tile instead of the warp-MMA decode kernel (decode.cu, one n8
+// token tile: up to 8 tokens); the pipeline takes the same time for any
+// count up to 16.
 #ifndef NF4_SMALL_M_TC_FROM
 #define NF4_SMALL_M_TC_FROM 9
 #endif
+static_assert(NF4_SMALL_M_TC_FROM <= 9, "the decode kernel serves at most 8 tokens");
 
 // Device error word: one per device, cleared by nf4_device_status().  Its
 // device address is looked up once per device (with that device current)
@@ -89,7 +88,7 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
                                const void *B, int r, float scaling, void *y, void *workspace,
                                int64_t workspace_bytes, cudaStream_t stream, int num_sms, unsigned *err_word) {
     const int rp = r > 0 ? lora_rp(r) : 0;
-    // decode-size M: the warp-MMA GEMV kernels up to NF4_SMALL_M_TC_FROM - 1
+    // decode-size M: the warp-MMA decode kernel up to NF4_SMALL_M_TC_FROM - 1
     // tokens, then the tcgen05 pipeline with a 16-token tile, split over the
     // SMs when the workspace holds its scratch (with an adapter, 8 SMs are
     // left to the down-projection's cluster, which runs first)
@@ -114,7 +113,11 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
         e = launch_pdl(k_zero_counts, dim3(1), dim3(256), 0, stream, 1, counts, ncounts);
     }
     if (e != cudaSuccess) return e;
-    if (gemv) return launch_gemv(x, (int)M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, stream, num_sms);
+    // with an adapter, the 8 SMs of the down-projection's cluster (launched
+    // just before) are left to it
+    if (gemv)
+        return launch_decode(x, (int)M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, err_word, stream,
+                             r > 0 && num_sms > 16 ? num_sms - 8 : num_sms);
     return launch_gemm_tc(x, M, K, N, packed, q8, scales, offset, B, r, workspace, rp, y, partials, counts, ctas, stream,
                           err_word);
 }

@@ -80,6 +80,25 @@ def test_gemv_ragged_shapes(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
     check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
 
 
+@pytest.mark.parametrize("M,K,N,r,dq", [(3, 5120, 264, 16, True),    # 20 slices of 256 columns: warps take several
+                                        (8, 1024, 4000, 0, True),     # 4 slices: four warp groups split the tiles
+                                        (2, 64, 136, 32, False),      # one slice: sixteen groups
+                                        (6, 1344, 48, 64, True),      # ragged last slice (21 blocks)
+                                        (1, 4096, 33024, 16, True)])  # more tiles per CTA than shared memory holds
+def test_decode_work_splits(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
+    """The decode kernel (up to 8 tokens) splits K into slices of 256
+    columns over the warps of a CTA and keeps per-slice partial tiles in
+    shared memory; these shapes reach each way of splitting."""
+    c = wl.LinearCase("decode split", M, K, N, r, 0.5, 977 + M + K + N)
+    W, x, A, B = wl.linear_inputs(c, with_lora=r > 0)
+    st = quantize_on_gpu(nf4lib, W, cuda_device, dq)
+    dA = None if A is None else A.to(cuda_device)
+    dB = None if B is None else B.to(cuda_device)
+    y = linear(nf4lib, x.to(cuda_device), st, N, dA, dB, c.scaling)
+    torch.cuda.synchronize()
+    check(y, oracle_linear(oracle_mod, st, x, A, B, r, c.scaling))
+
+
 @pytest.mark.parametrize("M,K,N,r", [(1, 512, 2400, 16), (13, 256, 200, 64), (4, 192, 64, 32), (40, 512, 264, 16)])
 def test_linear_double_quant_without_centring(nf4lib, oracle_mod, cuda_device, M, K, N, r):
     """Block constants decoded as E4M3 * c2 (no centring offset), through
