@@ -14,10 +14,12 @@
 // accumulation order is not specified, and would not reproduce it.
 //
 // Layout of the work: a CTA owns a tile of 64 rows x 256 columns of W.  A's
-// 256 columns (r x 256, fp32) and B's 64 rows (transposed, r x 64, fp32) are
-// staged in shared memory once.  Warp w owns rows 8 w .. 8 w + 7 of the tile and lane l
+// 256 columns (r x 256, fp32) and B's 64 rows (transposed, r x 64, each value
+// stored twice as an fp32 pair, the broadcast operand of the packed fma) are
+// staged in shared memory once, from 16-byte loads of A's and B's rows.
+// Warp w owns rows 8 w .. 8 w + 7 of the tile and lane l
 // columns 8 l .. 8 l + 7, so every value of A read from shared memory feeds 8
-// rows (64 fma per 2 vector loads and 8 broadcast loads); the 8 lanes
+// rows (32 packed fma per 2 + 4 vector loads); the 8 lanes
 // 8 m .. 8 m + 7 own one 64-block of each row, whose absmax is a 3-step
 // shuffle, and the codes come from the quantizer's exact selection.  The merged weight never leaves registers.  packed_out may alias
 // packed (every thread reads its 4 code bytes before it writes them), and
@@ -33,11 +35,10 @@ constexpr int kMergeCols = 256;
 constexpr int kMergeRows = 64;
 constexpr int kMergeThreads = 256;
 constexpr int kMergeMaxR = 64;
-// sB holds B transposed, [j][row] with rows padded to 68 floats: a warp's 8
-// rows at one j are two 16-byte broadcast loads (one wavefront each, against
-// 8 for 8 scalar loads), and the staging writes, 32 consecutive j of one row,
-// hit 8 banks 4 ways.
-constexpr int kMergeBStride = kMergeRows + 4;
+// sB holds B transposed and doubled, [j][row] = (B[row, j], B[row, j]) as fp32
+// pairs, rows padded to 136 floats: a warp's 8 rows at one j are four 16-byte
+// broadcast loads that give the packed fma its (b, b) operands directly.
+constexpr int kMergeBStride = 2 * kMergeRows + 8;
 
 template <int kMode>
 // Two CTAs per SM (128 registers): the epilogue's loads issued before the
@@ -57,16 +58,40 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
     __shared__ float s_lv[16];
     const int64_t k0 = (int64_t)blockIdx.x * kMergeCols;
     const int64_t n0 = (int64_t)blockIdx.y * kMergeRows;
-    for (int i = threadIdx.x; i < r * kMergeCols; i += kMergeThreads) {
-        const int j = i / kMergeCols, col = i % kMergeCols;
-        const int l = col >> 3, h = (col >> 2) & 1, c = col & 3;
-        const int64_t k = k0 + col;
-        sA[j * kMergeCols + h * 128 + l * 4 + c] = k < K ? __bfloat162float(A[(int64_t)j * K + k]) : 0.0f;
+    // A: 8 columns (one 16-byte load) per item, written as lane l's two float4
+    for (int i = threadIdx.x; i < r * (kMergeCols / 8); i += kMergeThreads) {
+        const int j = i >> 5, l = i & 31;  // kMergeCols / 8 == 32
+        const int64_t k = k0 + 8 * l;      // K % 64 == 0: 8 columns are all in or all out
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (k < K) u = __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)j * K + k));
+        float4 *dst = reinterpret_cast<float4 *>(sA + j * kMergeCols) + l;
+        dst[0] = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                             __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+        dst[32] = make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u),
+                              __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
     }
-    for (int i = threadIdx.x; i < kMergeRows * r; i += kMergeThreads) {
-        const int row = i / r, j = i % r;
+    // B: 8 consecutive j of one row (one 16-byte load) per item when r % 8 ==
+    // 0 (rows 16-byte aligned), else one value per item; each value written
+    // as the pair (b, b)
+    if ((r & 7) != 0) {
+        for (int i = threadIdx.x; i < kMergeRows * r; i += kMergeThreads) {
+            const int row = i % kMergeRows, j = i / kMergeRows;
+            const int64_t n = n0 + row;
+            const float b = n < N ? __bfloat162float(B[n * r + j]) : 0.0f;
+            *reinterpret_cast<float2 *>(sB + j * kMergeBStride + 2 * row) = make_float2(b, b);
+        }
+    }
+    for (int i = threadIdx.x; (r & 7) == 0 && i < kMergeRows * (r / 8); i += kMergeThreads) {
+        const int row = i % kMergeRows, j0 = (i / kMergeRows) * 8;
         const int64_t n = n0 + row;
-        sB[j * kMergeBStride + row] = n < N ? __bfloat162float(B[n * r + j]) : 0.0f;
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (n < N) u = __ldg(reinterpret_cast<const uint4 *>(B + n * r + j0));
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const float b = __uint_as_float((t & 1) ? (w4[t >> 1] & 0xFFFF0000u) : (w4[t >> 1] << 16));
+            *reinterpret_cast<float2 *>(sB + (j0 + t) * kMergeBStride + 2 * row) = make_float2(b, b);
+        }
     }
     if (threadIdx.x < 16) s_lv[threadIdx.x] = c_levels[threadIdx.x];
     build_code_tables(s_t, s_cell);  // (synchronises the CTA: sA, sB, s_lv ready too)
@@ -105,21 +130,24 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
     for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int h = 0; h < 4; ++h) d2[i][h] = 0ull;  // (+0, +0)
-    const float4 *a_lane = reinterpret_cast<const float4 *>(sA) + lane;
-    const float4 *b_warp = reinterpret_cast<const float4 *>(sB + 8 * warp);
+    const ulonglong2 *a_lane = reinterpret_cast<const ulonglong2 *>(sA) + lane;
+    const ulonglong2 *b_warp = reinterpret_cast<const ulonglong2 *>(sB + 16 * warp);
 #pragma unroll 2
     for (int j = 0; j < r; ++j) {
-        const float4 a0 = a_lane[j * 64], a1 = a_lane[j * 64 + 32];
-        const float4 b0 = b_warp[j * (kMergeBStride / 4)], b1 = b_warp[j * (kMergeBStride / 4) + 1];
-        const uint64_t a2[4] = {pack_f32x2(a0.x, a0.y), pack_f32x2(a0.z, a0.w), pack_f32x2(a1.x, a1.y),
-                                pack_f32x2(a1.z, a1.w)};
-        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        // (A[j, 8l + 2h], A[j, 8l + 2h + 1]) pairs and (B[8w + i, j]) x 2
+        const ulonglong2 a01 = a_lane[j * 64], a23 = a_lane[j * 64 + 32];
+        const uint64_t a2[4] = {a01.x, a01.y, a23.x, a23.y};
+        uint64_t bb[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint64_t bb = pack_f32x2(b[i], b[i]);
-#pragma unroll
-            for (int h = 0; h < 4; ++h) asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d2[i][h]) : "l"(bb), "l"(a2[h]));
+        for (int m = 0; m < 4; ++m) {
+            const ulonglong2 p = b_warp[j * (kMergeBStride / 4) + m];
+            bb[2 * m] = p.x;
+            bb[2 * m + 1] = p.y;
         }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int h = 0; h < 4; ++h) asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d2[i][h]) : "l"(bb[i]), "l"(a2[h]));
     }
     float d[8][8];
 #pragma unroll

@@ -33,7 +33,8 @@ def state_np(st):
 
 
 @pytest.mark.parametrize("N,K,r,mode", [(200, 320, 16, "dq"), (64, 256, 64, "nodq"), (130, 192, 32, "uncentred"),
-                                        (48, 4096, 7, "dq"), (33, 64, 0, "dq"), (70, 640, 64, "dq")])
+                                        (48, 4096, 7, "dq"), (33, 64, 0, "dq"), (70, 640, 64, "dq"),
+                                        (96, 128, 8, "dq"), (80, 512, 24, "nodq")])
 def test_merge_requantize_bit_exact(nf4lib, oracle_mod, cuda_device, N, K, r, mode):
     W, A, B = case(N, K, r, 1000 + N + K + r)
     st = nf4lib.quantize_weight(W.to(cuda_device), double_quant=(mode != "nodq"), centre=(mode == "dq"))
