@@ -19,9 +19,10 @@
 //        operand (instruction descriptor transpose bit): 128-byte swizzle
 //        atoms of 8 rows n x 64 k, the four 64-k atoms of a row group 8 KB
 //        apart (leading byte offset), row groups 1 KB apart (stride byte
-//        offset).  A lane owns two rows and one 64-block, dequantizes it with
-//        one register lookup table (mma_util.cuh) and writes it with eight
-//        16-byte stores, conflict-free across the 8 rows of an atom;
+//        offset).  A lane owns two rows (p and p + 32) of one 64-block,
+//        dequantizes each with one register lookup table (mma_util.cuh) and
+//        writes it with eight 16-byte stores; the 8 lanes of a store phase
+//        write the 8 rows of one atom, so the stores are conflict-free;
 // both operands come from shared memory (SS MMA).  Each dequantized weight
 // feeds 256 tokens, as in the forward.  After the N / 64 weight steps, RP / 64
 // extension steps add the LoRA term the same way: G' = [u_hi | u_lo | 0]
@@ -243,16 +244,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // ---------------- dequant warpgroups (transposed tiles), then epilogue ----------------
         const int q = warp & 3;         // k-block of the tile / tensor-memory lane quarter
         const int h = (warp - 4) >> 2;  // warpgroup: k-steps with index % kGWG == h
-        const int p = lane;             // n-pair: rows 2p, 2p + 1 of the step
+        // rows p and p + 32 of the step: the 8 lanes a 16-byte store serves
+        // together write 8 consecutive rows, whose swizzle phases differ
+        const int p = lane;
         const int64_t kb = (k0 >> 6) + q;  // this lane's k-block of W
         const bool kvalid = kb * 64 < K;
         const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
         bool ok = true;
         BlockCodes ca, cb, na, nb;
         auto load_pair = [&](int kt, BlockCodes &x0, BlockCodes &x1) {
-            const int64_t n = (int64_t)kt * kGK + 2 * p;
+            const int64_t n = (int64_t)kt * kGK + p;
             load_block<kMode>(packed, q8, scales, n, K, kb, kvalid && n < N, x0);
-            load_block<kMode>(packed, q8, scales, n + 1, K, kb, kvalid && n + 1 < N, x1);
+            load_block<kMode>(packed, q8, scales, n + 32, K, kb, kvalid && n + 32 < N, x1);
         };
         if (h < kn_steps) load_pair(h, ca, cb);
         for (int kt = h; kt < kt_total; kt += kGWG) {
@@ -262,8 +265,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
             if (kt < kn_steps) {
                 if (kt + kGWG < kn_steps) load_pair(kt + kGWG, na, nb);
                 // word j of a row holds k = 2j (low half) and 2j + 1 (high half):
-                // chunk c = words 4c .. 4c + 3; row 2p is dequantized before the
-                // wait for the stage and stored after it, then row 2p + 1
+                // chunk c = words 4c .. 4c + 3; row p is dequantized before the
+                // wait for the stage and stored after it, then row p + 32
                 uint32_t v[32];
                 {
                     const Lut la = make_lut(block_scale_finish<kMode>(ca.sr, mu));
@@ -274,7 +277,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 if (!ok) break;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
-                    sts128(tile + w_offset(2 * p, q, c), make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
+                    sts128(tile + w_offset(p, q, c), make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
                 {
                     const Lut lb = make_lut(block_scale_finish<kMode>(cb.sr, mu));
 #pragma unroll
@@ -282,25 +285,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
-                    sts128(tile + w_offset(2 * p + 1, q, c),
+                    sts128(tile + w_offset(p + 32, q, c),
                            make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
                 ca = na;
                 cb = nb;
             } else {
                 // rows j of [A ; A ; 0] (row j -> A[j mod r] for j < 2r), columns
-                // k0 + 64 q .. + 63: rows 2p and 2p + 1 of the step
+                // k0 + 64 q .. + 63: rows p and p + 32 of the step
                 const int e = kt - kn_steps;
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&S.empty[s], ph ^ 1u, abort, err));
                 if (!ok) break;
                 const int64_t k = k0 + 64 * q;
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    const int j = 64 * e + 2 * p + i;
+                    const int j = 64 * e + p + 32 * i;
                     const bool v = j < 2 * r && k < K;
                     const uint4 *src = reinterpret_cast<const uint4 *>(Al + (int64_t)(v ? j % r : 0) * K + (v ? k : 0));
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
-                        sts128(tile + w_offset(2 * p + i, q, c), v ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u));
+                        sts128(tile + w_offset(p + 32 * i, q, c), v ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u));
                 }
             }
             // the tile is read by the tensor cores (async proxy)
