@@ -817,24 +817,28 @@ __global__ void __launch_bounds__(128, 1)
 
     bool ok = true;
     if (threadIdx.x == 0 && kt_total > 0) {
-        // producer and MMA issuer in one thread: loads run kDownStages - 1 ahead
-        auto issue = [&](int kt) -> bool {
-            const int st = kt % kDownStages;
-            const uint32_t ph = (uint32_t)(kt / kDownStages) & 1u;
-            if (!mbar_wait(&S.empty[st], ph ^ 1u, abort, err)) return false;
-            mbar_arrive_expect_tx(&S.full[st], kStageBytes);
-            tma_load_2d(S.x[st], &tmap_x, &S.full[st], (kt_begin + kt) * 64, (int)m0);
-            tma_load_2d(S.a[st], &tmap_a, &S.full[st], (kt_begin + kt) * 64, 0);
-            return true;
-        };
+        // producer: the x and A boxes of every k-step, kDownStages ahead of the MMAs
         int issued = 0;
-        for (; issued < kDownStages - 1 && issued < kt_total && ok; ++issued) ok = issue(issued);
-        for (int kt = 0; kt < kt_total && ok; ++kt) {
-            if (issued < kt_total) {
-                ok = issue(issued);
-                ++issued;
-                if (!ok) break;
+        for (; issued < kt_total; ++issued) {
+            const int st = issued % kDownStages;
+            const uint32_t ph = (uint32_t)(issued / kDownStages) & 1u;
+            if (!mbar_wait(&S.empty[st], ph ^ 1u, abort, err)) break;
+            mbar_arrive_expect_tx(&S.full[st], kStageBytes);
+            tma_load_2d(S.x[st], &tmap_x, &S.full[st], (kt_begin + issued) * 64, (int)m0);
+            tma_load_2d(S.a[st], &tmap_a, &S.full[st], (kt_begin + issued) * 64, 0);
+        }
+        if (*abort) {  // every issued load lands before the CTA may exit
+            for (int kt = issued - kDownStages < 0 ? 0 : issued - kDownStages; kt < issued; ++kt) {
+                unsigned long long t0 = global_ns();
+                while (!mbar_try_wait(&S.full[kt % kDownStages], (uint32_t)(kt / kDownStages) & 1u) &&
+                       global_ns() - t0 < kWaitLimitNs) {
+                }
             }
+        }
+    } else if (threadIdx.x == 32 && kt_total > 0) {
+        // MMA issuer (its own thread, so that the loads and the MMAs of
+        // consecutive k-steps overlap): D[128 rows, r] += x A^T per k-step
+        for (int kt = 0; kt < kt_total; ++kt) {
             const int st = kt % kDownStages;
             if (!mbar_wait(&S.full[st], (uint32_t)(kt / kDownStages) & 1u, abort, err)) {
                 ok = false;
@@ -848,13 +852,6 @@ __global__ void __launch_bounds__(128, 1)
             tc_commit(&S.empty[st]);
         }
         tc_commit(&S.acc_full);
-        // every issued load has landed before the CTA may exit
-        for (int kt = issued - kDownStages < 0 ? 0 : issued - kDownStages; kt < issued; ++kt) {
-            unsigned long long t0 = global_ns();
-            while (!mbar_try_wait(&S.full[kt % kDownStages], (uint32_t)(kt / kDownStages) & 1u) &&
-                   global_ns() - t0 < kWaitLimitNs) {
-            }
-        }
     }
     __syncwarp();
     // this CTA's partial tile -> shared memory, column-major [kR][128] fp32
