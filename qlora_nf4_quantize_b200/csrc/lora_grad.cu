@@ -150,11 +150,11 @@ namespace {
 // MN-major operands (instruction descriptor transpose bits): each 8-row x
 // 128-byte swizzle atom holds 64 consecutive columns of 8 tokens; atoms along
 // the columns are a box apart (leading byte offset 8 KB), atoms along the
-// tokens 1 KB apart (stride byte offset).  One thread issues TMA and MMA
-// (ring of kGStagesTc); a cluster of kSplit CTAs splits the token rows and
+// tokens 1 KB apart (stride byte offset).  One thread issues the TMA copies,
+// another the MMAs (ring of kGStagesTc); a cluster of kSplit CTAs splits the token rows and
 // adds its fp32 partials in rank order through distributed shared memory; the
 // epilogue folds the hi and lo columns (c and c + r) and writes fp32.
-constexpr int kGStagesTc = 4;
+constexpr int kGStagesTc = 5;
 constexpr int kGBox = 64;                       // columns and token rows of one TMA box
 constexpr uint32_t kGBoxBytes = kGBox * kGBox * 2;  // 8 KB
 
@@ -230,32 +230,32 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t tmem = S.tmem_base;
 
     if (threadIdx.x == 0 && kt_total > 0) {
-        bool ok = true;
-        auto issue = [&](int kt) -> bool {
-            const int st = kt % kGStagesTc;
-            const uint32_t ph = (uint32_t)(kt / kGStagesTc) & 1u;
-            if (!mbar_wait(&S.empty[st], ph ^ 1u, abort, err)) return false;
+        // producer: the X and T2 boxes of every 64-token step, kGStagesTc ahead
+        int issued = 0;
+        for (; issued < kt_total; ++issued) {
+            const int st = issued % kGStagesTc;
+            const uint32_t ph = (uint32_t)(issued / kGStagesTc) & 1u;
+            if (!mbar_wait(&S.empty[st], ph ^ 1u, abort, err)) break;
             mbar_arrive_expect_tx(&S.full[st], kStageBytes);
-            const int m = (kt_begin + kt) * kGBox;
+            const int m = (kt_begin + issued) * kGBox;
             tma_load_2d(S.a[st][0], &tmap_x, &S.full[st], (int)p0, m);
             tma_load_2d(S.a[st][1], &tmap_x, &S.full[st], (int)p0 + kGBox, m);
 #pragma unroll
             for (int i = 0; i < kC / kGBox; ++i) tma_load_2d(S.b[st][i], &tmap_t, &S.full[st], kGBox * i, m);
-            return true;
-        };
-        int issued = 0;
-        for (; issued < kGStagesTc - 1 && issued < kt_total && ok; ++issued) ok = issue(issued);
-        for (int kt = 0; kt < kt_total && ok; ++kt) {
-            if (issued < kt_total) {
-                ok = issue(issued);
-                ++issued;
-                if (!ok) break;
+        }
+        if (*abort) {  // every issued load lands before the CTA may exit
+            for (int kt = issued - kGStagesTc < 0 ? 0 : issued - kGStagesTc; kt < issued; ++kt) {
+                unsigned long long t0 = global_ns();
+                while (!mbar_try_wait(&S.full[kt % kGStagesTc], (uint32_t)(kt / kGStagesTc) & 1u) &&
+                       global_ns() - t0 < kWaitLimitNs) {
+                }
             }
+        }
+    } else if (threadIdx.x == 32 && kt_total > 0) {
+        // MMA issuer, its own thread so that copies and MMAs overlap
+        for (int kt = 0; kt < kt_total; ++kt) {
             const int st = kt % kGStagesTc;
-            if (!mbar_wait(&S.full[st], (uint32_t)(kt / kGStagesTc) & 1u, abort, err)) {
-                ok = false;
-                break;
-            }
+            if (!mbar_wait(&S.full[st], (uint32_t)(kt / kGStagesTc) & 1u, abort, err)) break;
             tc_fence_after();
             const uint64_t ad = smem_desc_mn_sw128(S.a[st][0], kGBoxBytes);
             const uint64_t bd = smem_desc_mn_sw128(S.b[st][0], kGBoxBytes);
@@ -266,12 +266,6 @@ __global__ void __launch_bounds__(128, 1)
             tc_commit(&S.empty[st]);
         }
         tc_commit(&S.acc_full);
-        for (int kt = issued - kGStagesTc < 0 ? 0 : issued - kGStagesTc; kt < issued; ++kt) {
-            unsigned long long t0 = global_ns();
-            while (!mbar_try_wait(&S.full[kt % kGStagesTc], (uint32_t)(kt / kGStagesTc) & 1u) &&
-                   global_ns() - t0 < kWaitLimitNs) {
-            }
-        }
     }
     __syncwarp();
     // fold hi + lo into this CTA's partial tile, column-major [r][128] fp32, in
