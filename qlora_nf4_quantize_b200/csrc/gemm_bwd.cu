@@ -390,7 +390,7 @@ cudaError_t launch_bwd_mode(const CUtensorMap &mg, const CUtensorMap &mu, int64_
 }  // namespace
 
 cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
-                                unsigned *err, cudaStream_t stream, int split);
+                                unsigned *err, cudaStream_t stream, int split, int max_ctas);
 int lora_rp(int r);
 int64_t grad_chunks(int64_t M, int64_t P);
 cudaError_t launch_lora_grad_product(const __nv_bfloat16 *X, int64_t P, const __nv_bfloat16 *T, int64_t ldt,
@@ -471,11 +471,11 @@ cudaError_t launch_lora_linear_bwd(const void *g, const void *x, int64_t M, int6
             if (e != cudaSuccess) return e;
         }
         if (need_u) {  // u2 = s g (B^T)^T = s g B
-            e = launch_lora_down_tc(g, Bt, M, N, r, s, u2, rp, err, stream, split_for(N));
+            e = launch_lora_down_tc(g, Bt, M, N, r, s, u2, rp, err, stream, split_for(N), 0);
             if (e != cudaSuccess) return e;
         }
         if (dB) {  // t2 = s x A^T
-            e = launch_lora_down_tc(x, A, M, K, r, s, t2, rp, err, stream, split_for(K));
+            e = launch_lora_down_tc(x, A, M, K, r, s, t2, rp, err, stream, split_for(K), 0);
             if (e != cudaSuccess) return e;
         }
     }

@@ -926,6 +926,187 @@ __global__ void __launch_bounds__(128, 1)
     }
 }
 
+// Persistent form without a K split (the default alongside the fused GEMM):
+// CTA c takes the 128-row tiles c, c + gridDim.x, ..., so the launch can be
+// held to the SMs the GEMM leaves idle.  Warp 4 (one lane) streams the x and
+// A boxes of every tile through the ring, warp 5 (one lane) issues the MMAs
+// into one of two tensor-memory accumulators (tile parity), and warps 0-3
+// (tensor-memory lane quarters) turn each finished accumulator into rows of
+// t while the next tile's MMAs run.
+constexpr int kDownPThreads = 192;
+
+template <int kR>
+struct __align__(1024) DownPSmem {
+    uint8_t x[kDownStages][kDownRows * 128];
+    uint8_t a[kDownStages][kR * 128];
+    uint64_t full[kDownStages];
+    uint64_t empty[kDownStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int kR>
+__global__ void __launch_bounds__(kDownPThreads, 1)
+    k_lora_down_tc_p(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_a,
+                     int64_t M, int64_t K, float scaling, __nv_bfloat16 *__restrict__ t2, int rp, unsigned *err) {
+    constexpr uint32_t kCols = kR < 32 ? 32 : kR;  // one accumulator; two are allocated
+    constexpr uint32_t kIdescDown = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kR >> 3) << 17) |
+                                    ((uint32_t)(kDownRows >> 4) << 24);
+    constexpr uint32_t kStageBytes = kDownRows * 128 + kR * 128;
+    extern __shared__ uint8_t smem_raw[];
+    DownPSmem<kR> &S =
+        *reinterpret_cast<DownPSmem<kR> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    volatile int *abort = &S.abort;
+    // the fused linear launched next may start once every CTA is past this
+    // point; it reads x and W at once and waits for t itself
+    pdl_wait_then_release();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntiles = (int)((M + kDownRows - 1) / kDownRows);
+    const int kt_total = (int)((K + 63) / 64);  // a partial last step reads zeros beyond K (TMA fill)
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kDownStages; ++st) {
+            mbar_init(&S.full[st], 1);
+            mbar_init(&S.empty[st], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.acc_full[b], 1);
+            mbar_init(&S.acc_empty[b], 4);
+        }
+        S.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&S.tmem_base)),
+                     "r"(2 * kCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            // producer: every k-step of every tile, kDownStages ahead of the MMAs
+            int64_t g = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                for (int kt = 0; kt < kt_total; ++kt, ++g) {
+                    const int st = (int)(g % kDownStages);
+                    const uint32_t ph = (uint32_t)(g / kDownStages) & 1u;
+                    if (!mbar_wait(&S.empty[st], ph ^ 1u, abort, err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&S.full[st], kStageBytes);
+                    tma_load_2d(S.x[st], &tmap_x, &S.full[st], kt * 64, tile * kDownRows);
+                    tma_load_2d(S.a[st], &tmap_a, &S.full[st], kt * 64, 0);
+                }
+            }
+            if (*abort) {  // every issued load lands before the CTA may exit
+                for (int64_t k2 = g - kDownStages < 0 ? 0 : g - kDownStages; k2 < g; ++k2) {
+                    const unsigned long long t0 = global_ns();
+                    while (!mbar_try_wait(&S.full[k2 % kDownStages], (uint32_t)(k2 / kDownStages) & 1u) &&
+                           global_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            // MMA issuer: D_b[128 rows, r] = x A^T of one tile, b = tile parity
+            int64_t g = 0;
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+                const int b = it & 1;
+                // the accumulator's previous tile has been read out
+                if (it >= 2 && !mbar_wait(&S.acc_empty[b], (uint32_t)((it >> 1) - 1) & 1u, abort, err)) break;
+                tc_fence_after();
+                const uint32_t acc = tmem + (uint32_t)b * kCols;
+                for (int kt = 0; kt < kt_total; ++kt, ++g) {
+                    const int st = (int)(g % kDownStages);
+                    if (!mbar_wait(&S.full[st], (uint32_t)(g / kDownStages) & 1u, abort, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc_sw128(S.x[st]), bd = smem_desc_sw128(S.a[st]);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_ss(acc, ad + 2ull * kk, bd + 2ull * kk, kIdescDown, (kt | kk) != 0 ? 1u : 0u);
+                    tc_commit(&S.empty[st]);
+                }
+                tc_commit(&S.acc_full[b]);
+            }
+        }
+    } else {
+        // epilogue: thread = tile row 32 warp + lane = tensor-memory lane
+        int it = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int b = it & 1;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.acc_full[b], (uint32_t)(it >> 1) & 1u, abort, err))) break;
+            tc_fence_after();
+            const int64_t m = (int64_t)tile * kDownRows + 32 * warp + lane;
+            const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)b * kCols;
+#pragma unroll
+            for (int c0 = 0; c0 < kR; c0 += 32) {
+                uint32_t v[32];
+                tc_load32(taddr + (uint32_t)c0, v);
+                tc_wait_ld();
+                if (m < M) {
+                    const int kW = kR - c0 < 32 ? kR - c0 : 32;  // valid columns of this chunk
+#pragma unroll
+                    for (int j0 = 0; j0 < kW; j0 += 8) {
+                        uint32_t hi[4], lo[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float v0 = __uint_as_float(v[j0 + 2 * j]) * scaling;
+                            const float v1 = __uint_as_float(v[j0 + 2 * j + 1]) * scaling;
+                            const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+                            hi[j] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+                            lo[j] = pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+                        }
+                        *reinterpret_cast<uint4 *>(t2 + m * rp + c0 + j0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4 *>(t2 + m * rp + kR + c0 + j0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    }
+                }
+            }
+            if (m < M)
+                for (int j = 2 * kR; j < rp; j += 8)
+                    *reinterpret_cast<uint4 *>(t2 + m * rp + j) = make_uint4(0u, 0u, 0u, 0u);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acc_empty[b]);  // the accumulator may be reused
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kCols) : "memory");
+    }
+}
+
+template <int kR>
+cudaError_t launch_down_tc_p(const CUtensorMap &mx, const CUtensorMap &ma, int64_t M, int64_t K, float s, void *t2,
+                             int rp, unsigned *err, cudaStream_t stream, int max_ctas) {
+    const size_t smem = sizeof(DownPSmem<kR>) + 1024;
+    cudaError_t e =
+        cudaFuncSetAttribute(k_lora_down_tc_p<kR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (M + kDownRows - 1) / kDownRows;
+    const int64_t grid = max_ctas > 0 && max_ctas < tiles ? max_ctas : tiles;
+    return launch_pdl(k_lora_down_tc_p<kR>, dim3((unsigned)grid), dim3(kDownPThreads), smem, stream, 1u, mx, ma, M,
+                      K, s, static_cast<__nv_bfloat16 *>(t2), rp, err);
+}
+
 template <int kR, int kSplit>
 cudaError_t launch_down_tc(const CUtensorMap &mx, const CUtensorMap &ma, int64_t M, int64_t K, float s, void *t2,
                            int rp, unsigned *err, cudaStream_t stream) {
@@ -941,9 +1122,10 @@ cudaError_t launch_down_tc(const CUtensorMap &mx, const CUtensorMap &ma, int64_t
 
 template <int kR>
 cudaError_t launch_down_tc_split(const CUtensorMap &mx, const CUtensorMap &ma, int64_t M, int64_t K, float s,
-                                 void *t2, int rp, unsigned *err, cudaStream_t stream, int split) {
+                                 void *t2, int rp, unsigned *err, cudaStream_t stream, int split, int max_ctas) {
     if (split == 4) return launch_down_tc<kR, 4>(mx, ma, M, K, s, t2, rp, err, stream);
-    return launch_down_tc<kR, kDownSplit>(mx, ma, M, K, s, t2, rp, err, stream);
+    if (kDownSplit != 1) return launch_down_tc<kR, kDownSplit>(mx, ma, M, K, s, t2, rp, err, stream);
+    return launch_down_tc_p<kR>(mx, ma, M, K, s, t2, rp, err, stream, max_ctas);
 }
 
 }  // namespace
@@ -988,11 +1170,12 @@ cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const
 }
 
 // Tensor-core LoRA down-projection: see k_lora_down_tc.  split: 0 = the
-// default (one CTA per 128 rows, the least SM time while a fused GEMM runs
-// alongside); 4 = K split over a 4-CTA cluster (a long contraction with
-// nothing running alongside).
+// default (persistent CTAs over the 128-row tiles, the least SM time while a
+// fused GEMM runs alongside; max_ctas > 0 caps the grid, e.g. to the SMs the
+// GEMM leaves idle); 4 = K split over a 4-CTA cluster (a long contraction
+// with nothing running alongside).
 cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
-                                unsigned *err, cudaStream_t stream, int split) {
+                                unsigned *err, cudaStream_t stream, int split, int max_ctas) {
     if (M > 0x7FFFFFFF || K > 0x7FFFFFFF) return cudaErrorInvalidValue;
     CUtensorMap mx, ma;
     cudaError_t e = make_map(&mx, x, M, K, 64, kDownRows, true);
@@ -1000,9 +1183,9 @@ cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t
     e = make_map(&ma, A, r, K, 64, r, true);
     if (e != cudaSuccess) return e;
     switch (r) {
-        case 16: return launch_down_tc_split<16>(mx, ma, M, K, s, t2, rp, err, stream, split);
-        case 32: return launch_down_tc_split<32>(mx, ma, M, K, s, t2, rp, err, stream, split);
-        case 64: return launch_down_tc_split<64>(mx, ma, M, K, s, t2, rp, err, stream, split);
+        case 16: return launch_down_tc_split<16>(mx, ma, M, K, s, t2, rp, err, stream, split, max_ctas);
+        case 32: return launch_down_tc_split<32>(mx, ma, M, K, s, t2, rp, err, stream, split, max_ctas);
+        case 64: return launch_down_tc_split<64>(mx, ma, M, K, s, t2, rp, err, stream, split, max_ctas);
         default: return cudaErrorInvalidValue;
     }
 }

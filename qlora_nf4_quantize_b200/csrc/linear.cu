@@ -14,7 +14,7 @@ cudaError_t launch_decode(const void *x, int M, int64_t K, int64_t N, const uint
                           const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                           void *y, unsigned *err, cudaStream_t stream, int num_sms);
 cudaError_t launch_lora_down_tc(const void *x, const void *A, int64_t M, int64_t K, int r, float s, void *t2, int rp,
-                                unsigned *err, cudaStream_t stream, int split);
+                                unsigned *err, cudaStream_t stream, int split, int max_ctas);
 cudaError_t launch_gemm_tc(const void *x, int64_t M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                            const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                            void *y, float *partials, unsigned *counts, int ctas, cudaStream_t stream,
@@ -107,8 +107,14 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
     cudaError_t e = cudaSuccess;
     if (r > 0) {
         // decode-size M: warp-MMA kernel; larger M: tensor-core kernel
-        e = M <= kGemvMaxTokens ? launch_lora_down(x, A, M, K, r, scaling, workspace, counts, ncounts, stream)
-                                : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream, 0);
+        // with fewer GEMM tiles than SMs (a small N), the down-projection is
+        // held to the SMs the GEMM leaves idle, so that no GEMM tile waits
+        // for an SM it holds (one CTA per 128-row tile otherwise)
+        const int64_t gemm_ctas = ((N + 127) / 128) * ((M + 255) / 256);
+        const int idle = gemm_ctas < num_sms ? num_sms - (int)gemm_ctas : 0;
+        e = M <= kGemvMaxTokens
+                ? launch_lora_down(x, A, M, K, r, scaling, workspace, counts, ncounts, stream)
+                : launch_lora_down_tc(x, A, M, K, r, scaling, workspace, rp, err_word, stream, 0, idle >= 8 ? idle : 0);
     } else if (ctas > 0) {
         e = launch_pdl(k_zero_counts, dim3(1), dim3(256), 0, stream, 1, counts, ncounts);
     }
