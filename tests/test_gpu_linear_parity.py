@@ -84,7 +84,8 @@ def test_gemv_ragged_shapes(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
                                         (8, 1024, 4000, 0, True),     # 4 slices: four warp groups split the tiles
                                         (2, 64, 136, 32, False),      # one slice: sixteen groups
                                         (6, 1344, 48, 64, True),      # ragged last slice (21 blocks)
-                                        (1, 4096, 33024, 16, True)])  # more tiles per CTA than shared memory holds
+                                        (1, 4096, 33024, 16, True),   # more tiles per CTA than shared memory holds
+                                        (5, 128, 8, 16, True)])       # one partial tile
 def test_decode_work_splits(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
     """The decode kernel (up to 8 tokens) splits K into slices of 256
     columns over the warps of a CTA and keeps per-slice partial tiles in
