@@ -211,10 +211,11 @@ NF4_API nf4_status nf4_dequantize(const uint8_t *packed, const uint8_t *absmax_q
                           void *out, nf4_dtype out_dtype, void *stream);
 
 /* Bytes of device workspace nf4_lora_linear_fwd needs for M rows of x and
- * rank r: the low-rank intermediate t (M * round_up(2r, 64) * 2 bytes), and
- * for M <= 16 also the scratch of the split 16-token pipeline (partial tiles
- * and arrival counts, about 3 MiB, after t at a 256-byte boundary).  0 for
- * M > 16 and r == 0. */
+ * rank r: the low-rank intermediate t (M * round_up(2r, 64) * 2 bytes); 0 for
+ * r == 0.  (A library built with NF4_SMALL_M_TC_FROM=9, which sends 9 to 16
+ * tokens to the split 16-token tensor-core pipeline, adds that pipeline's
+ * scratch for those M: partial tiles and arrival counts, about 3 MiB, after
+ * t at a 256-byte boundary.) */
 NF4_API int64_t nf4_lora_linear_workspace_size(int64_t M, int r);
 
 /* nf4_lora_linear_fwd -- the frozen-base LoRA linear of [MF] "Forward Pass
@@ -234,16 +235,14 @@ NF4_API int64_t nf4_lora_linear_workspace_size(int64_t M, int r);
  *   y          device bf16[M, N] (output)
  *   workspace  device scratch, workspace_bytes >=
  *              nf4_lora_linear_workspace_size(M, r); NULL allowed when r == 0.
- *              With r > 0 at least the t part is required; for 9 <= M <= 16
- *              a workspace of less than the full size (or none) runs the
- *              16-token pipeline unsplit (slower, same tolerance).  Nothing
- *              has to be cleared between calls; calls that share a workspace
- *              must be ordered (one stream).
- * M <= 8 runs the streaming warp-MMA GEMV kernel, 9 <= M <= 16 the
- * tensor-core GEMM pipeline with a 16-token tile split over the SMs, larger
- * M the same pipeline with 256-token tiles; the LoRA pre-step is one extra
- * launch when r > 0 (without it, a split call adds a one-CTA launch that
- * zeroes the arrival counts). */
+ *              With r > 0 at least the t part is required (in a library
+ *              built with NF4_SMALL_M_TC_FROM=9, a workspace of less than
+ *              the full size for 9 <= M <= 16 runs that pipeline unsplit).
+ *              Nothing has to be cleared between calls; calls that share a
+ *              workspace must be ordered (one stream).
+ * M <= 16 runs the streaming warp-MMA decode kernel (one 8-token MMA tile up
+ * to M = 8, two above), larger M the tensor-core GEMM pipeline with
+ * 256-token tiles; the LoRA pre-step is one extra launch when r > 0. */
 NF4_API nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int64_t N,
                                const uint8_t *packed, const uint8_t *absmax_q,
                                const float *absmax2, const float *offset,
@@ -265,8 +264,9 @@ NF4_API nf4_status nf4_lora_linear_fwd(const void *x, int64_t M, int64_t K, int6
  *   Limit: the intermediate t, M * round_up(2r, 64) * 2 bytes, must not
  *          exceed NF4_NOALLOC_SCRATCH_BYTES (M <= 16384 for r = 64, M <= 32768
  *          for r <= 32); larger sizes return NF4_ERR_UNSUPPORTED before any
- *          work.  Up to 16 tokens the array also holds the split pipeline's
- *          scratch (nf4_lora_linear_workspace_size(M, r) <= 4 MiB there).
+ *          work.  (In a library built with NF4_SMALL_M_TC_FROM=9 the array
+ *          also holds, for 9 to 16 tokens, the split pipeline's
+ *          scratch: nf4_lora_linear_workspace_size(M, r) <= 4 MiB there.)
  *   The first call on a device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
  *   The address is cached for the life of the process's context on that

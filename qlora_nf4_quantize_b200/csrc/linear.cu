@@ -25,13 +25,15 @@ int streamk_ctas(int64_t M, int64_t K, int64_t N, int rp, int sms);
 
 constexpr int kGemvMaxTokens = 16;
 // Token counts from which decode-size calls take the tcgen05 pipeline with a
-// 16-token tile instead of the warp-MMA decode kernel (decode.cu, one n8
-// token tile: up to 8 tokens); the pipeline takes the same time for any
-// count up to 16.
+// 16-token tile, split over the SMs, instead of the warp-MMA decode kernel
+// (decode.cu: up to 16 tokens).  The default (17) sends every decode-size
+// call to the decode kernel, which is faster at every count (at 16 tokens,
+// W 11008 x 4096, r = 16: 22.6 against 26.0 us); a build with 9 keeps the
+// split pipeline for 9..16 tokens.
 #ifndef NF4_SMALL_M_TC_FROM
-#define NF4_SMALL_M_TC_FROM 9
+#define NF4_SMALL_M_TC_FROM 17
 #endif
-static_assert(NF4_SMALL_M_TC_FROM <= 9, "the decode kernel serves at most 8 tokens");
+static_assert(NF4_SMALL_M_TC_FROM >= 9 && NF4_SMALL_M_TC_FROM <= 17, "the decode kernel serves 1..8 tokens at least, 16 at most");
 
 // Device error word: one per device, cleared by nf4_device_status().  Its
 // device address is looked up once per device (with that device current)
@@ -63,14 +65,16 @@ unsigned *device_error_word(cudaError_t *status) {
 // t2 = [t_hi | t_lo | 0 pad] bf16 [M, round_up(2r, 64)], 16-byte aligned rows.
 int64_t lora_workspace_bytes(int64_t M, int r) { return M * (int64_t)lora_rp(r) * 2; }
 
-// Up to 16 tokens the workspace continues (256-byte aligned) with the
-// scratch of the split 16-token pipeline: partial tiles, then arrival
-// counts.  A workspace holding only t (or none, r = 0) runs it unsplit.
+// Token counts served by the split 16-token pipeline (none in the default
+// build): for them the workspace continues (256-byte aligned) with its
+// scratch, partial tiles then arrival counts.  A workspace holding only t (or
+// none, r = 0) runs it unsplit.
+static bool split_tokens(int64_t M) { return M >= NF4_SMALL_M_TC_FROM && M <= kGemvMaxTokens; }
 static int64_t partials_offset(int64_t M, int r) {
     return (lora_workspace_bytes(M, r > 0 ? r : 0) + 255) & ~(int64_t)255;
 }
 int64_t linear_workspace_bytes(int64_t M, int r) {
-    if (M <= kGemvMaxTokens) return partials_offset(M, r) + streamk_partials_bytes() + streamk_counts_bytes();
+    if (split_tokens(M)) return partials_offset(M, r) + streamk_partials_bytes() + streamk_counts_bytes();
     return r > 0 ? lora_workspace_bytes(M, r) : 0;
 }
 
@@ -92,11 +96,11 @@ cudaError_t launch_lora_linear(const void *x, int64_t M, int64_t K, int64_t N, c
     // tokens, then the tcgen05 pipeline with a 16-token tile, split over the
     // SMs when the workspace holds its scratch (with an adapter, 8 SMs are
     // left to the down-projection's cluster, which runs first)
-    const bool gemv = M < NF4_SMALL_M_TC_FROM && M <= kGemvMaxTokens;
+    const bool gemv = M < NF4_SMALL_M_TC_FROM;
     float *partials = nullptr;
     unsigned *counts = nullptr;
     int ctas = 0;
-    if (!gemv && M <= kGemvMaxTokens && workspace != nullptr && workspace_bytes >= linear_workspace_bytes(M, r)) {
+    if (split_tokens(M) && workspace != nullptr && workspace_bytes >= linear_workspace_bytes(M, r)) {
         ctas = streamk_ctas(M, K, N, rp, r > 0 && num_sms > 16 ? num_sms - 8 : num_sms);
         if (ctas > 0) {
             partials = reinterpret_cast<float *>(static_cast<char *>(workspace) + partials_offset(M, r));

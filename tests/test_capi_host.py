@@ -90,13 +90,13 @@ def test_workspace_sizes(nf4lib):
     assert nf4lib.nf4_quantize_dq_workspace_size(4096 * 4096) == 262144 * 4 + (1024 + 32) * 8
     assert nf4lib.nf4_quantize_dq_workspace_size(130) == 256 + (1 + 1) * 8
     assert nf4lib.nf4_quantize_dq_workspace_size(128, 32, 256) == 0
-    # up to 16 tokens: [t_hi | t_lo | pad] rows of 64, then (256-byte aligned)
-    # the split pipeline's scratch: 192 CTAs x 2 partial tiles of 16 x 128
-    # fp32, then 192 arrival counts
-    split = 192 * 2 * 16 * 128 * 4 + 192 * 4
-    assert nf4lib.nf4_lora_linear_workspace_size(16, 16) == 16 * 64 * 2 + split
-    assert nf4lib.nf4_lora_linear_workspace_size(3, 16) == 512 + split  # 384 bytes of t, aligned up
-    assert nf4lib.nf4_lora_linear_workspace_size(16, 0) == split
+    # [t_hi | t_lo | pad] rows of round_up(2r, 64) bf16; nothing without an
+    # adapter (decode-size calls need no scratch of their own)
+    assert nf4lib.nf4_lora_linear_workspace_size(16, 16) == 16 * 64 * 2
+    assert nf4lib.nf4_lora_linear_workspace_size(3, 16) == 3 * 64 * 2
+    assert nf4lib.nf4_lora_linear_workspace_size(9, 64) == 9 * 128 * 2
+    assert nf4lib.nf4_lora_linear_workspace_size(16, 0) == 0
+    assert nf4lib.nf4_lora_linear_workspace_size(1, 0) == 0
     assert nf4lib.nf4_lora_linear_workspace_size(17, 0) == 0
     assert nf4lib.nf4_lora_linear_workspace_size(4096, 0) == 0
     assert nf4lib.nf4_lora_linear_workspace_size(4096, 64) == 4096 * 128 * 2

@@ -2,7 +2,7 @@
 launches (programmatic dependent launch between them).  These tests check
 that such replays compute exactly what the same calls compute when launched
 one by one: quantize + double quantize, dequantize, and the fused linear on
-its three paths (one-token GEMV, split 16-token pipeline, 256-token GEMM),
+its three paths (decode kernel with one and two token tiles, 256-token GEMM),
 each replayed with inputs rotating over several copies, outputs compared bit
 for bit with the eager calls (and the eager calls are the ones the parity
 tests check against the oracle)."""

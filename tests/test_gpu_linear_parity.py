@@ -85,11 +85,21 @@ def test_gemv_ragged_shapes(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
                                         (2, 64, 136, 32, False),      # one slice: sixteen groups
                                         (6, 1344, 48, 64, True),      # ragged last slice (21 blocks)
                                         (1, 4096, 33024, 16, True),   # more tiles per CTA than shared memory holds
-                                        (5, 128, 8, 16, True)])       # one partial tile
+                                        (5, 128, 8, 16, True),        # one partial tile
+                                        # two token tiles (9..16 tokens), slices of 128 columns
+                                        (11, 5120, 264, 16, True),    # 40 slices: warps take two or three
+                                        (13, 11008, 520, 16, True),   # 86 slices, several tiles per CTA
+                                        (16, 1024, 4000, 0, True),    # 8 slices: two warp groups
+                                        (9, 64, 136, 32, False),      # one slice, its second block outside K
+                                        (12, 192, 40, 16, True),      # odd block count: half of the last slice
+                                        (14, 1344, 48, 64, True),     # ragged last slice (21 blocks)
+                                        (16, 4096, 33024, 16, True),  # chunks that use both partial regions
+                                        (10, 128, 8, 16, True)])      # one partial tile
 def test_decode_work_splits(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
-    """The decode kernel (up to 8 tokens) splits K into slices of 256
-    columns over the warps of a CTA and keeps per-slice partial tiles in
-    shared memory; these shapes reach each way of splitting."""
+    """The decode kernel (up to 16 tokens, in one or two tiles of 8) splits K
+    into slices of 256 or 128 columns over the warps of a CTA and keeps
+    per-slice partial tiles in shared memory; these shapes reach each way of
+    splitting."""
     c = wl.LinearCase("decode split", M, K, N, r, 0.5, 977 + M + K + N)
     W, x, A, B = wl.linear_inputs(c, with_lora=r > 0)
     st = quantize_on_gpu(nf4lib, W, cuda_device, dq)
@@ -201,40 +211,37 @@ def test_gemm_and_gemv_agree_on_shared_rows(nf4lib, cuda_device):
 @pytest.mark.parametrize("M,K,N,r,dq", [(9, 1024, 8, 16, True), (12, 512, 2400, 16, False), (16, 512, 2400, 64, True),
                                         (16, 2048, 640, 32, True), (11, 8192, 1000, 0, True),
                                         (16, 64, 18936, 32, True), (10, 4096, 11008, 0, True)])
-def test_split_decode_pipeline(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
-    """9 to 16 tokens: the 16-token tensor-core pipeline split over the SMs
-    (full workspace) and unsplit (a workspace holding only t) both match the
-    oracle, and the split result is bitwise the same on every run (each
-    tile's partials are added in CTA order).  Shapes cover one tile split
-    over two CTAs, ranges that start inside the LoRA extension steps, no
-    adapter, and 148 tiles (no split: not more CTAs than tiles)."""
-    c = wl.LinearCase("split", M, K, N, r, 1.25, 57 + M + K + N)
+def test_two_token_tiles_repeatable(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
+    """9 to 16 tokens (the decode kernel's two 8-token tiles): the result
+    matches the oracle and is bitwise the same on every run and with a
+    workspace larger than required (partial tiles are added in slot order,
+    never in arrival order).  Shapes cover one partial row tile, no adapter,
+    more row tiles than SMs, and K of one block."""
+    c = wl.LinearCase("two tiles", M, K, N, r, 1.25, 57 + M + K + N)
     W, x, A, B = wl.linear_inputs(c, with_lora=r > 0)
     st = quantize_on_gpu(nf4lib, W, cuda_device, dq)
     xd = x.to(cuda_device)
     dA = None if A is None else A.to(cuda_device)
     dB = None if B is None else B.to(cuda_device)
     ref = oracle_linear(oracle_mod, st, x, A, B, r, c.scaling)
-    full = nf4lib.nf4_lora_linear_workspace_size(M, r)
-    t_only = M * ((2 * r + 63) // 64) * 64 * 2
-    assert full > t_only
+    need = nf4lib.nf4_lora_linear_workspace_size(M, r)
+    assert need == (M * ((2 * r + 63) // 64) * 64 * 2 if r > 0 else 0)
     outs = []
-    for ws_bytes in (full, full, t_only, full):
+    for ws_bytes in (need, need, need + 4096, need):
         outs.append(linear(nf4lib, xd, st, N, dA, dB, c.scaling, ws_bytes=ws_bytes))
     torch.cuda.synchronize()
     assert nf4lib.nf4_device_status() == 0
     for y in outs:
         check(y, ref)
-    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[3])
+    assert all(torch.equal(outs[0], y) for y in outs[1:])
 
 
-def test_split_decode_pipeline_back_to_back(nf4lib, cuda_device):
-    """Calls of the split pipeline queued back to back on one stream, with
-    and without an adapter, reuse one workspace (its arrival counts are
-    zeroed by the kernel launched before each linear): every output equals
-    the same call run alone, and no call writes outside its output or the
-    shared workspace."""
-    c = wl.LinearCase("split b2b", 16, 2048, 4096, 16, 2.0, 93)
+def test_two_token_tiles_back_to_back(nf4lib, cuda_device):
+    """16-token decode calls queued back to back on one stream (programmatic
+    dependent launch between them), with and without an adapter, reuse one
+    workspace: every output equals the same call run alone, and no call
+    writes outside its output or the shared workspace."""
+    c = wl.LinearCase("decode b2b", 16, 2048, 4096, 16, 2.0, 93)
     W, x, A, B = wl.linear_inputs(c)
     st = quantize_on_gpu(nf4lib, W, cuda_device)
     xd, Ad, Bd = x.to(cuda_device), A.to(cuda_device), B.to(cuda_device)

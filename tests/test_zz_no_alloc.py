@@ -4,8 +4,7 @@ loops that must not call cudaMalloc mid-step, frameworks whose memory is
 reserved by their own pool).  Its output must match nf4_lora_linear_fwd (the
 entry point with a caller workspace) and the CPU oracle within the matmul
 tolerance, on two calls in a row (the shared scratch keeps the previous
-call's contents; up to 16 tokens it also holds the split pipeline's partial
-tiles and arrival counts), and write nothing outside its output.
+call's contents), and write nothing outside its output.
 
 Collected last on purpose, so a run that stops at the first failure has
 already run every other test; it also passes alone in a fresh process."""
