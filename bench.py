@@ -300,8 +300,9 @@ def _projection_segments(q, wl, dev, rank, segs):
 
     def f_qdq(k):  # the stored format in one call (its fp32 constants stay in the workspace)
         q.nf4_quantize_dq(W2[k], packed=pk[k], absmax_q=q8x[k], absmax2=c2x[k], offset=mux[k], workspace=qdq_ws)
+    # launches: quantize, run sums, double quantization (1024 runs: no chunk sums)
     segs.append(Segment("quantize+dq", [lambda k=k: f_qdq(k) for k in range(C)], 16, quantize_dq_bytes(n), "GB/s",
-                        2, proj + " (nf4_quantize_dq)"))
+                        3, proj + " (nf4_quantize_dq)"))
     segs.append(Segment("dequantize", [lambda k=k: q.nf4_dequantize(pk[k], q8[k], c2[k], mu[k], n, torch.bfloat16,
                                                                      out=deq[k]) for k in range(C)],
                         32, dequant_bytes(n), "GB/s", 1, proj + " -> bf16"))
@@ -380,8 +381,9 @@ def _sweep_segment(q, wl, dev, segs):
             q.nf4_quantize_dq(w, packed=p_, absmax_q=q_, absmax2=c_, offset=o_, workspace=wsd)
             q.nf4_dequantize(p_, q_, c_, o_, m, torch.bfloat16, out=out)
     layer_b = sum(quantize_dq_bytes(w.numel()) + dequant_bytes(w.numel()) for w in Wl)
-    # launches: 2 per quantize + DQ (3 above 2048 runs: gate and up), 1 per dequantize
-    layer_launches = sum(3 + (1 if -(-w.numel() // (BLOCK * DQ_BLOCK)) > 2048 else 0) for w in Wl)
+    # launches: 3 per quantize + DQ (quantize, run sums, double quantization; 4
+    # above 2048 runs: gate, up and down), 1 per dequantize
+    layer_launches = sum(4 + (1 if -(-w.numel() // (BLOCK * DQ_BLOCK)) > 2048 else 0) for w in Wl)
     segs.append(Segment("sweep_8B_layer", [f_layer], 1, layer_b, "GB/s", layer_launches,
                         "the 7 linear weights of one 8B-shaped decoder layer (218.1 M params): nf4_quantize_dq + "
                         "nf4_dequantize (bf16); the sweep is 32 such layers"))

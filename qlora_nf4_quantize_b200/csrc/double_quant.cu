@@ -11,10 +11,9 @@
 // up unchanged.
 //
 // Kernels
-//   k_dq_run_sums    one warp per run: the run's fp64 sum (dq_sum.cuh).  The
-//                    quantizer can write the same sums as it goes
-//                    (nf4_quantize_dq), and a tensor sharded over ranks
-//                    gathers its shards' sums (nf4_double_quantize_sharded).
+//   k_dq_run_sums    one warp per run: the run's fp64 sum (dq_sum.cuh).  A
+//                    tensor sharded over ranks gathers its shards' sums
+//                    (nf4_double_quantize_sharded).
 //   k_dq_chunks_from_runs
 //                    for large tensors only: one thread per chunk of 32
 //                    consecutive run sums combines them (a level-5 node of

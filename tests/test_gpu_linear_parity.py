@@ -113,7 +113,7 @@ def test_decode_work_splits(nf4lib, oracle_mod, cuda_device, M, K, N, r, dq):
 @pytest.mark.parametrize("M,K,N,r", [(1, 512, 2400, 16), (13, 256, 200, 64), (4, 192, 64, 32), (40, 512, 264, 16)])
 def test_linear_double_quant_without_centring(nf4lib, oracle_mod, cuda_device, M, K, N, r):
     """Block constants decoded as E4M3 * c2 (no centring offset), through
-    the persistent GEMV, the per-tile GEMV and the tensor-core GEMM."""
+    the decode kernel (one and two token tiles) and the tensor-core GEMM."""
     c = wl.LinearCase("no centring", M, K, N, r, 1.25, 211 + M + K + N)
     W, x, A, B = wl.linear_inputs(c)
     st = nf4lib.quantize_weight(W.to(cuda_device), centre=False)
