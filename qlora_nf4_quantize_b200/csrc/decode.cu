@@ -31,8 +31,8 @@
 //     of the slice (rows g and g + 8): 64-block t for kNT = 1, half of
 //     64-block t / 2 for kNT = 2.  x uses the same permutation (one 8-byte
 //     fragment per step and token tile).  A lane's columns therefore lie in
-//     one 64-block: one constant per row and unit.  Even and odd steps
-//     accumulate into separate chains.
+//     one 64-block: one constant per row and unit.  With one token tile
+//     even and odd steps accumulate into separate chains.
 //   - dequantization through a shared-memory table of unscaled level pairs
 //     (q[b >> 4], q[b & 15]) for every code byte b, in 16 copies so that the
 //     16 lanes a 64-bit shared load serves together never share a bank; the
@@ -71,6 +71,9 @@ struct DGeom {
     static constexpr int kBlocksPerUnit = 4 / kNT;  // 64-blocks of a row in a unit
     static constexpr int kXFrags = 16 / kNT;        // 8-byte x fragments per token tile
     static constexpr int kTileFloats = 128 * kNT;   // partial tile: 16 rows x 8 kNT tokens
+    // MMA accumulator chains per token tile: even and odd steps apart with
+    // one tile; with two, the tiles' chains already alternate
+    static constexpr int kChains = kNT == 1 ? 2 : 1;
 };
 
 // Work of one CTA: tiles [t0, t0 + my_tiles) in chunks of `chunk` tiles, S
@@ -168,7 +171,9 @@ __device__ __forceinline__ void pair_word(uint32_t base_lane, uint32_t w, uint64
 // the two rows (row g: constant c0, row g + 8: c1).
 template <int kNT>
 __device__ __forceinline__ void mma_unit(const uint32_t (&w)[2][8 / kNT], float c0, float c1, uint32_t base_lane,
-                                         const uint2 (&xr)[kNT][16 / kNT], float (&acc)[kNT][2][4]) {
+                                         const uint2 (&xr)[kNT][16 / kNT],
+                                         float (&acc)[kNT][DGeom<kNT>::kChains][4]) {
+    constexpr int kOdd = DGeom<kNT>::kChains - 1;  // chain of the odd steps
     const uint64_t cc0 = pack_f32x2(c0, c0), cc1 = pack_f32x2(c1, c1);
 #pragma unroll
     for (int q = 0; q < 8 / kNT; ++q) {  // packed word q = MMA steps 2q, 2q+1
@@ -180,7 +185,7 @@ __device__ __forceinline__ void mma_unit(const uint32_t (&w)[2][8 / kNT], float 
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) {
             mma_bf16_16816(acc[nt][0], a0, xr[nt][2 * q].x, xr[nt][2 * q].y);
-            mma_bf16_16816(acc[nt][1], a1, xr[nt][2 * q + 1].x, xr[nt][2 * q + 1].y);
+            mma_bf16_16816(acc[nt][kOdd], a1, xr[nt][2 * q + 1].x, xr[nt][2 * q + 1].y);
         }
     }
 }
@@ -384,11 +389,13 @@ __global__ void __launch_bounds__(kDThreads, 1)
 
             const float sc0 = block_scale_finish<kMode>(sr_cur[0], mu);
             const float sc1 = block_scale_finish<kMode>(sr_cur[1], mu);
-            float acc[kNT][2][4];
+            float acc[kNT][G::kChains][4];
 #pragma unroll
             for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[nt][0][i] = acc[nt][1][i] = 0.0f;
+                for (int ch = 0; ch < G::kChains; ++ch)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[nt][ch][i] = 0.0f;
             mma_unit<kNT>(w, sc0, sc1, base_lane, xr, acc);
             const int sl = wk.S <= kDWarps ? s : warp;
             float *pp = tile_part(j - c0) + sl * G::kTileFloats + lane;
@@ -396,12 +403,14 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
                 for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) pp[128 * nt + 32 * i] = acc[nt][0][i] + acc[nt][1][i];
+                    for (int i = 0; i < 4; ++i)
+                        pp[128 * nt + 32 * i] = G::kChains == 1 ? acc[nt][0][i] : acc[nt][0][i] + acc[nt][G::kChains - 1][i];
             } else {
 #pragma unroll
                 for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) pp[128 * nt + 32 * i] += acc[nt][0][i] + acc[nt][1][i];
+                    for (int i = 0; i < 4; ++i)
+                        pp[128 * nt + 32 * i] += G::kChains == 1 ? acc[nt][0][i] : acc[nt][0][i] + acc[nt][G::kChains - 1][i];
             }
             c_read.step(wk, warp);
 #pragma unroll
