@@ -51,15 +51,13 @@
 //     B operand = [t_hi | t_lo]) by MMA and stores.
 // The kernel has no spin-waits: copies are tracked per thread (cp.async
 // groups) and the warps meet only at CTA barriers.
+#include "decode_split.h"
 #include "mma_util.cuh"
 
 namespace nf4 {
 namespace {
 
-constexpr int kDWarps = 16;
 constexpr int kDThreads = kDWarps * 32;
-constexpr int kDRing = 3;           // unit slots per warp
-constexpr int kDSmem = 227 * 1024;  // all of it: the layout below needs 224 KB
 
 // Unit geometry for kNT token tiles of 8.
 template <int kNT>
@@ -74,58 +72,8 @@ struct DGeom {
     // MMA accumulator chains per token tile: even and odd steps apart with
     // one tile; with two, the tiles' chains already alternate
     static constexpr int kChains = kNT == 1 ? 2 : 1;
-};
-
-// Work of one CTA: tiles [t0, t0 + my_tiles) in chunks of `chunk` tiles, S
-// slices per row.
-struct DWork {
-    int64_t t0;
-    int my_tiles, S, tps, nslot, chunk;
-    int tw, s_w;  // S <= 16: first tile and slice of this warp
-    bool active;  // S <= 16: the warp has a slice
-
-    // n_tiles * gridDim.x < 2^32 (checked by the host): 32-bit divisions
-    __device__ __forceinline__ void init(uint32_t n_tiles, int64_t kblocks, int blocks_per_unit, int warp,
-                                         int chunk_tiles) {
-        const uint32_t b0 = blockIdx.x * n_tiles / gridDim.x, b1 = (blockIdx.x + 1) * n_tiles / gridDim.x;
-        t0 = b0;
-        my_tiles = (int)(b1 - b0);
-        S = (int)((kblocks + blocks_per_unit - 1) / blocks_per_unit);
-        chunk = chunk_tiles;
-        tps = S <= kDWarps ? kDWarps / S : 1;  // tiles a 16-warp round covers
-        nslot = S < kDWarps ? S : kDWarps;
-        tw = S <= kDWarps ? warp / S : 0;
-        s_w = S <= kDWarps ? warp % S : warp;
-        active = S > kDWarps || warp < tps * S;
-    }
-};
-
-// Position in this warp's unit sequence: tile j (in the CTA), slice s; cb =
-// first tile of the current chunk.  S <= 16: tiles tw, tw + tps, ... at slice
-// s_w.  S > 16: within each chunk, slice-major (all tiles of the chunk at
-// slice warp, then at warp + 16, ...).
-struct DCursor {
-    int j, s, cb;
-    __device__ __forceinline__ void start(const DWork &wk) {
-        j = wk.active ? wk.tw : wk.my_tiles;
-        s = wk.s_w;
-        cb = 0;
-    }
-    __device__ __forceinline__ void step(const DWork &wk, int warp) {
-        if (wk.S <= kDWarps) {
-            j += wk.tps;
-            return;
-        }
-        const int ce = min(cb + wk.chunk, wk.my_tiles);
-        if (++j < ce) return;
-        if ((s += kDWarps) < wk.S) {
-            j = cb;
-            return;
-        }
-        s = warp;  // the next chunk, which starts at j == ce
-        cb = ce;
-    }
-    __device__ __forceinline__ bool valid(const DWork &wk) const { return j < wk.my_tiles; }
+    static_assert(kRingBytes == decode_ring_bytes(kNT) && kBlocksPerUnit == decode_blocks_per_unit(kNT),
+                  "unit geometry of decode_split.h");
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
@@ -190,15 +138,13 @@ __device__ __forceinline__ void mma_unit(const uint32_t (&w)[2][8 / kNT], float 
     }
 }
 
-// Shared-memory layout (offsets in the shared window): the pair table at
-// 64 KB (so that byte b of a code word, permuted into bits 8..15, addresses
-// its entry), the warps' rings at 128 KB, the partials from the start of the
-// dynamic shared memory up to the table (the first low_tiles tiles of a
-// chunk) and after the rings (the rest).  The dynamic shared memory starts
-// below 1 KB of the window: the host sizes the low partials for 63 KB and
-// the high ones for what the rings leave of kDSmem.
-constexpr uint32_t kDTableAt = 0x10000, kDRingAt = 0x20000;
-constexpr uint32_t kDPartRoom = kDTableAt - 1024;
+// Shared-memory layout (offsets in the shared window, decode_split.h): the
+// pair table at 64 KB (so that byte b of a code word, permuted into bits
+// 8..15, addresses its entry), the warps' rings at 128 KB, the partials from
+// the start of the dynamic shared memory up to the table (the first
+// low_tiles tiles of a chunk) and after the rings (the rest).  The dynamic
+// shared memory starts below 1 KB of the window: the host sizes the low
+// partials for 63 KB and the high ones for what the rings leave of kDSmem.
 static_assert(kDRingAt + DGeom<1>::kRingBytes <= (uint32_t)kDSmem && DGeom<2>::kRingBytes <= DGeom<1>::kRingBytes,
               "shared-memory layout");
 
@@ -219,7 +165,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
     const int g = lane >> 2, tq = lane & 3;
     const int64_t kblocks = K >> 6, row_bytes = K >> 1;
     DWork wk;
-    wk.init((uint32_t)((N + 15) >> 4), kblocks, G::kBlocksPerUnit, warp, chunk_tiles);
+    wk.init((uint32_t)((N + 15) >> 4), K, kNT, warp, chunk_tiles, blockIdx.x, gridDim.x);
     const uint32_t s_base = (uint32_t)__cvta_generic_to_shared(s_dyn);
     const uint32_t tile_bytes = (uint32_t)wk.nslot * G::kTileFloats * 4u;
     const uint32_t hi_at = kDRingAt + G::kRingBytes;
@@ -397,7 +343,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) acc[nt][ch][i] = 0.0f;
             mma_unit<kNT>(w, sc0, sc1, base_lane, xr, acc);
-            const int sl = wk.S <= kDWarps ? s : warp;
+            const int sl = c_read.slot(wk, warp);
             float *pp = tile_part(j - c0) + sl * G::kTileFloats + lane;
             if (s < kDWarps) {
 #pragma unroll
@@ -502,32 +448,16 @@ template <int kNT>
 cudaError_t launch_decode_nt(const void *x, int M, int64_t K, int64_t N, const uint8_t *packed, const uint8_t *q8,
                              const float *scales, const float *offset, const void *B, int r, const void *t2, int rp,
                              void *y, unsigned *err, cudaStream_t stream, int num_sms) {
-    using G = DGeom<kNT>;
-    const int64_t n_tiles = (N + 15) / 16;
-    const int grid = (int)(n_tiles < num_sms ? n_tiles : num_sms);
-    if (n_tiles * (grid + 1) >= ((int64_t)1 << 32)) return cudaErrorInvalidValue;  // 32-bit work split
-    // tiles of a chunk: those whose partials fit below the table, then those
-    // that fit after the rings; a multiple of the tiles a round of the 16
-    // warps covers unless all of a CTA's tiles fit
-    const int64_t S = (K / 64 + G::kBlocksPerUnit - 1) / G::kBlocksPerUnit;
-    const int64_t nslot = S < kDWarps ? S : kDWarps, tps = S <= kDWarps ? kDWarps / S : 1;
-    const int64_t max_tiles = (n_tiles + grid - 1) / grid;
-    const int64_t tile_bytes = nslot * G::kTileFloats * 4;
-    const int64_t low = kDPartRoom / tile_bytes;
-    const int64_t high = ((int64_t)kDSmem - (int64_t)(kDRingAt + G::kRingBytes)) / tile_bytes;
-    int64_t chunk = low + high;
-    if (chunk >= max_tiles) chunk = max_tiles;
-    else chunk -= chunk % tps;
-    if (chunk < 1) return cudaErrorInvalidValue;
-    const int low_tiles = (int)(low < chunk ? low : chunk);
+    DChunk ch;
+    if (!decode_chunk(N, K, kNT, num_sms, &ch)) return cudaErrorInvalidValue;
     if (q8 == nullptr)
-        return launch_decode_mode<2, kNT>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, err, stream, grid,
-                                          (int)chunk, low_tiles);
+        return launch_decode_mode<2, kNT>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, err, stream,
+                                          ch.grid, ch.chunk, ch.low_tiles);
     if (offset == nullptr)
-        return launch_decode_mode<1, kNT>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, err, stream, grid,
-                                          (int)chunk, low_tiles);
-    return launch_decode_mode<0, kNT>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, err, stream, grid,
-                                      (int)chunk, low_tiles);
+        return launch_decode_mode<1, kNT>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, err, stream,
+                                          ch.grid, ch.chunk, ch.low_tiles);
+    return launch_decode_mode<0, kNT>(x, M, K, N, packed, q8, scales, offset, B, r, t2, rp, y, err, stream, ch.grid,
+                                      ch.chunk, ch.low_tiles);
 }
 
 }  // namespace
