@@ -27,8 +27,10 @@
 // MMA issuer (one elected lane of the converged warp), warps 4..15 = three
 // dequant warpgroups (warpgroup h produces the k-steps with index = h mod 3)
 // and, at the end, the epilogue (tcgen05.ld, bf16 conversion, one TMA store
-// of y).  The same pipeline with a 16-token tile serves decode calls of 9 to
-// 16 tokens, split over the SMs (stream-K, see TmemPlan below).
+// of y).  The same pipeline with a 16-token tile can serve decode calls of 9
+// to 16 tokens, split over the SMs (stream-K, see TmemPlan below): in a
+// library built with NF4_SMALL_M_TC_FROM=9 (linear.cu); by default the
+// decode kernel (decode.cu) takes every call of up to 16 tokens.
 //
 // Every mbarrier wait is bounded (about one second of %globaltimer): on
 // expiry the waiter raises a CTA-wide abort flag and the device error word,

@@ -1,5 +1,6 @@
 /* streamk.h -- the work partition of the split 16-token decode pipeline
- * (gemm_tc.cu, stream-K), in plain C so that the kernel and a CPU test
+ * (gemm_tc.cu, stream-K; taken for 9 to 16 tokens in a library built with
+ * NF4_SMALL_M_TC_FROM=9), in plain C so that the kernel and a CPU test
  * harness compile the same functions.
  *
  * The T = tiles x kt_total (weight tile, k-step) pairs are taken tile after

@@ -1,5 +1,6 @@
 """Host-side check of the work partition that the split 16-token pipeline
-(decode calls of 9 to 16 tokens) relies on: the partition functions are
+(decode calls of 9 to 16 tokens in a library built with
+NF4_SMALL_M_TC_FROM=9) relies on: the partition functions are
 compiled from the kernel's own header (csrc/streamk.h) with gcc and checked
 by exhaustion over many shapes:
 
