@@ -258,9 +258,6 @@ __global__ void __launch_bounds__(kDThreads, 1)
         c_sc.step(wk, warp);
         if (c_read.valid(wk)) load_x(c_read.s);
     };
-    // with an adapter nothing before this kernel writes what it reads: the
-    // stream starts at once and overlaps the table fill
-    if (r > 0) start_stream();
     {
         // 16 copies of (q[b >> 4], q[b & 15]) in the first 128 bytes of
         // entry b (a 64-bit read by 16 lanes is served at once, so lanes l
@@ -285,11 +282,15 @@ __global__ void __launch_bounds__(kDThreads, 1)
             t4[b * 16 + (i & 7)] = make_float4(hi, lo, hi, lo);
         }
     }
-    if (r <= 0) {
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        start_stream();
-    }
+    // with an adapter nothing before this kernel writes what it reads (the
+    // down-projection before it releases it only after its own wait), so
+    // only its epilogue waits; without one x and W wait for the grid before
+    if (r <= 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();  // the pair table is complete
+    // each warp starts its stream after the barrier, so that no warp waits
+    // for the others to have issued their first copies (the copy queue is
+    // full for ~1.4 us as every SM asks for 3 units per warp at once)
+    start_stream();
 
     const float mu = (kMode == 0) ? __ldg(offset) : 0.0f;
     const uint32_t base_lane = kDTableAt | (uint32_t)((lane & 15) * 8);
