@@ -97,8 +97,8 @@ NF4_API nf4_status nf4_quantize(const void *w, nf4_dtype w_dtype, int64_t n, int
                         uint8_t *packed, float *absmax, void *stream);
 
 /* Bytes of device workspace nf4_quantize_dq needs for n weights (the fp32
- * block constants, then the fp64 run sums of the centring mean, then one
- * 8-byte grid-barrier word); 0 for n <= 0 or unsupported block sizes. */
+ * block constants, then the fp64 run sums of the centring mean); 0 for
+ * n <= 0 or unsupported block sizes. */
 NF4_API int64_t nf4_quantize_dq_workspace_size(int64_t n, int blocksize, int dq_blocksize);
 
 /* nf4_quantize_dq -- nf4_quantize followed by nf4_double_quantize in one call
@@ -114,15 +114,9 @@ NF4_API int64_t nf4_quantize_dq_workspace_size(int64_t n, int blocksize, int dq_
  *   offset     device fp32[1] (output mu) or NULL (no centring)
  *   workspace  device scratch, 256-byte aligned, workspace_bytes >=
  *              nf4_quantize_dq_workspace_size(n, 64, 256); contents on entry
- *              are ignored.  Calls that share a workspace must be ordered
- *              (one stream).
- * Two kernel launches: the quantizer, then (with centring, up to 2048 runs,
- * i.e. 33.5 M weights) one kernel that sums the runs, meets at a grid-wide
- * barrier (a word of the workspace that the quantizer zeroes; a bounded wait
- * of about one second, after which nf4_device_status reports
- * NF4_ERR_TIMEOUT) and double-quantizes, or (without centring) the double
- * quantization alone.  Above 2048 runs with centring: four launches, the run
- * sums, chunk sums and double quantization of nf4_double_quantize. */
+ *              are ignored.
+ * Three kernel launches with centring (four above 2048 runs, i.e. 33.5 M
+ * weights), two without. */
 NF4_API nf4_status nf4_quantize_dq(const void *w, nf4_dtype w_dtype, int64_t n, int blocksize, int dq_blocksize,
                                    uint8_t *packed, uint8_t *absmax_q, float *absmax2, float *offset,
                                    void *workspace, int64_t workspace_bytes, void *stream);

@@ -12,10 +12,7 @@
 
 namespace nf4 {
 cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed, float *absmax,
-                            cudaStream_t stream, int num_sms, unsigned *zero_word);
-bool dq_fused_supported(int64_t nb, bool centred);
-cudaError_t launch_dq_fused(const float *absmax, int64_t nb, uint8_t *codes, float *absmax2, float *offset,
-                            double *run_sums, unsigned *count, unsigned *err, cudaStream_t stream, int num_sms);
+                            cudaStream_t stream, int num_sms);
 int64_t dq_run_count(int64_t nblocks);
 int64_t dq_chunk_count(int64_t nblocks);
 int64_t dq_max_chunks();
@@ -115,19 +112,17 @@ nf4_status nf4_quantize(const void *w, nf4_dtype w_dtype, int64_t n, int blocksi
     cudaError_t st;
     int sms = sm_count(&st);
     if (st != cudaSuccess) return cuda_status(st);
-    return cuda_status(
-        nf4::launch_quantize(w, w_dtype == NF4_BF16, n, packed, absmax, (cudaStream_t)stream, sms, nullptr));
+    return cuda_status(nf4::launch_quantize(w, w_dtype == NF4_BF16, n, packed, absmax, (cudaStream_t)stream, sms));
 }
 
 // Workspace of nf4_quantize_dq: the fp32 first-level constants (256-byte
-// aligned), then the run sums and chunk sums of the centring mean, then one
-// 8-byte word for the grid barrier of the fused double quantization.
+// aligned), then the run sums and chunk sums of the centring mean.
 static int64_t qdq_absmax_bytes(int64_t nb) { return (nb * 4 + 255) & ~(int64_t)255; }
 
 int64_t nf4_quantize_dq_workspace_size(int64_t n, int blocksize, int dq_blocksize) {
     if (n <= 0 || blocksize != nf4::kBlock || dq_blocksize != nf4::kDqBlock) return 0;
     const int64_t nb = (n + nf4::kBlock - 1) / nf4::kBlock;
-    return qdq_absmax_bytes(nb) + nf4::dq_workspace_bytes(nb) + 8;
+    return qdq_absmax_bytes(nb) + nf4::dq_workspace_bytes(nb);
 }
 
 nf4_status nf4_quantize_dq(const void *w, nf4_dtype w_dtype, int64_t n, int blocksize, int dq_blocksize,
@@ -148,23 +143,8 @@ nf4_status nf4_quantize_dq(const void *w, nf4_dtype w_dtype, int64_t n, int bloc
     if (st != cudaSuccess) return cuda_status(st);
     float *c1 = static_cast<float *>(workspace);
     double *sums = reinterpret_cast<double *>(static_cast<char *>(workspace) + qdq_absmax_bytes(nb));
-    unsigned *count = reinterpret_cast<unsigned *>(reinterpret_cast<char *>(sums) + nf4::dq_workspace_bytes(nb));
-    // centred tensors of up to 2048 runs: the quantizer zeroes the barrier
-    // word and one fused launch does the run sums and the double
-    // quantization; otherwise the run-sum launches of nf4_double_quantize
-    const bool fused = nf4::dq_fused_supported(nb, offset != nullptr);
-    unsigned *err = nullptr;
-    if (fused) {
-        err = nf4::device_error_word(&st);
-        if (st != cudaSuccess) return cuda_status(st);
-    }
-    st = nf4::launch_quantize(w, w_dtype == NF4_BF16, n, packed, c1, (cudaStream_t)stream, sms,
-                              fused ? count : nullptr);
+    st = nf4::launch_quantize(w, w_dtype == NF4_BF16, n, packed, c1, (cudaStream_t)stream, sms);
     if (st != cudaSuccess) return cuda_status(st);
-    if (fused) {
-        st = nf4::launch_dq_fused(c1, nb, absmax_q, absmax2, offset, sums, count, err, (cudaStream_t)stream, sms);
-        if (st != cudaErrorNotSupported) return cuda_status(st);
-    }
     return cuda_status(
         nf4::launch_double_quantize(c1, nb, absmax_q, absmax2, offset, sums, (cudaStream_t)stream, sms));
 }

@@ -27,15 +27,8 @@
 // level-by-level rule on its own leaves, so splitting the tree at level 5
 // reproduces the single-pass order exactly.
 //
-//   k_dq_fused       run sums, a grid barrier, then k_dq_quantize's work in
-//                    one launch (nf4_quantize_dq, centred, up to 2048 runs):
-//                    the grid is capped at one resident wave, the barrier
-//                    word is zeroed by the quantizer launched before it, and
-//                    the wait is bounded (about one second, then bit 0 of
-//                    the device error word).
 // Run sums: dq_sum.cuh (in parallel when exact, else sequentially).
 #include "dq_sum.cuh"
-#include "mbarrier.cuh"
 
 namespace nf4 {
 namespace {
@@ -61,14 +54,11 @@ __device__ __forceinline__ double tree_serial(double *s, int64_t len) {
 // The chunk sum (level-5 node) of runs 32 c .. min(32 c + 32, nd) - 1, by
 // one warp (every lane gets it): lane j holds s[j], and each level of the
 // pairwise rule (s[j] = s[2j] + s[2j+1], an odd last element carried up) is
-// two shuffles.  kL2: read the sums through L2 (written by other CTAs of the
-// same grid).
-template <bool kL2>
+// two shuffles.
 __device__ __forceinline__ double chunk_sum_warp(const double *__restrict__ run_sums, int64_t nd, int64_t c,
                                                  int lane) {
     int len = (int)(nd - c * kRunsPerChunk < kRunsPerChunk ? nd - c * kRunsPerChunk : kRunsPerChunk);
-    const double *p = run_sums + c * kRunsPerChunk + lane;
-    double v = lane < len ? (kL2 ? __ldcg(p) : *p) : 0.0;
+    double v = lane < len ? run_sums[c * kRunsPerChunk + lane] : 0.0;
     while (len > 1) {  // len is warp-uniform
         const int half = len >> 1;
         const double a = __shfl_sync(0xFFFFFFFFu, v, (2 * lane) & 31);
@@ -126,34 +116,42 @@ __device__ double tree_reduce(double *a, double *b, int64_t len) {
     return a[0];
 }
 
-// The mean from the sums (every thread of the CTA gets it): S / nb_mean, S
-// the tree over the run sums of nd_mean runs when sums_are_runs (the CTA folds
-// the chunks itself), else over their chunk sums.  s_tree: 2 * nchunks doubles.
-template <bool kL2>
-__device__ float dq_mean(const double *__restrict__ sums, int64_t nd_mean, int sums_are_runs, int64_t nb_mean,
-                         double *s_tree) {
+// nb constants of c1 are quantized.  With offset non-NULL the mean is
+// S / nb_mean, S the tree over the sums: run sums of nd_mean runs when
+// sums_are_runs (each CTA folds the chunks itself), else their nchunks chunk
+// sums.  nb_mean = nb unless c1 is one shard of a larger tensor.
+__global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c1, int64_t nb,
+                                                      const double *__restrict__ sums, int64_t nd_mean,
+                                                      int sums_are_runs, int64_t nb_mean,
+                                                      uint8_t *__restrict__ codes, float *__restrict__ absmax2,
+                                                      float *__restrict__ offset) {
+    extern __shared__ double s_tree[];  // 2 * nchunks doubles when centring
     __shared__ float s_mu;
-    const int64_t nchunks = (nd_mean + kRunsPerChunk - 1) / kRunsPerChunk;
-    if (sums_are_runs) {  // one warp per chunk
-        const int lane = threadIdx.x & 31;
-        for (int64_t j = threadIdx.x >> 5; j < nchunks; j += blockDim.x >> 5) {
-            const double cs = chunk_sum_warp<kL2>(sums, nd_mean, j, lane);
-            if (lane == 0) s_tree[j] = cs;
+    pdl_wait_then_release();
+    if (offset != nullptr) {
+        const int64_t nchunks = (nd_mean + kRunsPerChunk - 1) / kRunsPerChunk;
+        if (sums_are_runs) {  // one warp per chunk
+            const int lane = threadIdx.x & 31;
+            for (int64_t j = threadIdx.x >> 5; j < nchunks; j += blockDim.x >> 5) {
+                const double cs = chunk_sum_warp(sums, nd_mean, j, lane);
+                if (lane == 0) s_tree[j] = cs;
+            }
+        } else {
+            for (int64_t j = threadIdx.x; j < nchunks; j += blockDim.x) s_tree[j] = sums[j];
         }
-    } else {
-        for (int64_t j = threadIdx.x; j < nchunks; j += blockDim.x) s_tree[j] = sums[j];
+        __syncthreads();
+        double S = tree_reduce(s_tree, s_tree + nchunks, nchunks);
+        if (threadIdx.x == 0) {
+            float mu = (float)(S / (double)nb_mean);
+            s_mu = mu;
+            if (blockIdx.x == 0) *offset = mu;
+        }
+    } else if (threadIdx.x == 0) {
+        s_mu = 0.0f;
     }
     __syncthreads();
-    const double S = tree_reduce(s_tree, s_tree + nchunks, nchunks);
-    if (threadIdx.x == 0) s_mu = (float)(S / (double)nb_mean);
-    __syncthreads();
-    return s_mu;
-}
+    const float mu = s_mu;
 
-// Runs of 256 constants of c1 (one warp per run, grid-stride): c2 = max
-// |RN(c1 - mu)|, codes E4M3(RN(RN(c1 - mu) / c2)).
-__device__ void dq_quantize_runs(const float *__restrict__ c1, int64_t nb, float mu, uint8_t *__restrict__ codes,
-                                 float *__restrict__ absmax2) {
     const int lane = threadIdx.x & 31;
     const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
     const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -186,79 +184,6 @@ __device__ void dq_quantize_runs(const float *__restrict__ c1, int64_t nb, float
         }
         if (lane == 0) absmax2[d] = c2;
     }
-}
-
-// nb constants of c1 are quantized.  With offset non-NULL the mean is
-// S / nb_mean, S the tree over the sums: run sums of nd_mean runs when
-// sums_are_runs (each CTA folds the chunks itself), else their nchunks chunk
-// sums.  nb_mean = nb unless c1 is one shard of a larger tensor.
-__global__ void __launch_bounds__(256) k_dq_quantize(const float *__restrict__ c1, int64_t nb,
-                                                      const double *__restrict__ sums, int64_t nd_mean,
-                                                      int sums_are_runs, int64_t nb_mean,
-                                                      uint8_t *__restrict__ codes, float *__restrict__ absmax2,
-                                                      float *__restrict__ offset) {
-    extern __shared__ double s_tree[];  // 2 * nchunks doubles when centring
-    pdl_wait_then_release();
-    float mu = 0.0f;
-    if (offset != nullptr) {
-        mu = dq_mean<false>(sums, nd_mean, sums_are_runs, nb_mean, s_tree);
-        if (blockIdx.x == 0 && threadIdx.x == 0) *offset = mu;
-    }
-    dq_quantize_runs(c1, nb, mu, codes, absmax2);
-}
-
-// Barrier of a grid whose CTAs are all resident (the host caps the grid at
-// one wave): each CTA adds 1 to *count (zero when the grid before completed)
-// once its writes are done, then waits until all gridDim.x have arrived, for
-// at most kWaitLimitNs.  False on expiry (bit 0 of the error word raised).
-__device__ bool grid_barrier(unsigned *count, unsigned *err) {
-    __shared__ int s_ok;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(count, 1u);
-        const unsigned long long t0 = global_ns();
-        int ok = 1;
-        for (;;) {
-            unsigned v;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
-            if (v >= gridDim.x) break;
-            if (global_ns() - t0 > kWaitLimitNs) {
-                ok = 0;
-                atomicOr(err, 1u);
-                break;
-            }
-            __nanosleep(128);
-        }
-        __threadfence();
-        s_ok = ok;
-    }
-    __syncthreads();
-    return s_ok != 0;
-}
-
-// Centred double quantization in one launch: the run sums (one warp per run,
-// grid-stride), the grid barrier, then the mean and the runs' codes as
-// k_dq_quantize (every CTA folds all nd run sums itself).
-__global__ void __launch_bounds__(256) k_dq_fused(const float *__restrict__ c1, int64_t nb,
-                                                   double *__restrict__ run_sums, unsigned *count, unsigned *err,
-                                                   uint8_t *__restrict__ codes, float *__restrict__ absmax2,
-                                                   float *__restrict__ offset) {
-    extern __shared__ double s_tree[];  // 2 * nchunks doubles
-    pdl_wait_then_release();
-    const int lane = threadIdx.x & 31;
-    const int64_t nd = (nb + kDqBlock - 1) / kDqBlock;
-    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t d = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); d < nd; d += warps_total) {
-        const int64_t lo = d * kDqBlock;
-        const int64_t cnt = (nb - lo) < kDqBlock ? (nb - lo) : kDqBlock;
-        const double sum = run_sum_fp64(c1 + lo, cnt, lane);
-        if (lane == 0) __stcg(run_sums + d, sum);
-    }
-    if (!grid_barrier(count, err)) return;
-    const float mu = dq_mean<true>(run_sums, nd, 1, nb, s_tree);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *offset = mu;
-    dq_quantize_runs(c1, nb, mu, codes, absmax2);
 }
 
 }  // namespace
@@ -302,34 +227,6 @@ cudaError_t launch_dq_from_run_sums(const float *absmax, int64_t nb, const doubl
     if (grid < 1) grid = 1;  // an empty shard still writes mu
     return launch_pdl(k_dq_quantize, dim3(grid), dim3(256), smem, stream, 1, absmax, nb, sums, nd_total, are_runs,
                       nb_total, codes, absmax2, offset);
-}
-
-// Whether nf4_quantize_dq takes the fused launch: centred, at most
-// kDirectChunks chunks of runs (each CTA folds them itself).
-bool dq_fused_supported(int64_t nb, bool centred) {
-    return centred && nb > 0 && dq_chunk_count(nb) <= kDirectChunks;
-}
-
-// k_dq_fused over the nb constants of absmax; count must be zero when the
-// grid before it completes (k_quantize zeroes it).  cudaErrorNotSupported
-// when the fused form does not apply (dq_fused_supported, or the grid would
-// not fit one wave): the caller then takes the run-sum launch path, which
-// needs no zeroed word.
-cudaError_t launch_dq_fused(const float *absmax, int64_t nb, uint8_t *codes, float *absmax2, float *offset,
-                            double *run_sums, unsigned *count, unsigned *err, cudaStream_t stream, int num_sms) {
-    if (!dq_fused_supported(nb, offset != nullptr) || count == nullptr || err == nullptr)
-        return cudaErrorNotSupported;
-    const int64_t nd = dq_run_count(nb);
-    const size_t smem = (size_t)(2 * dq_chunk_count(nb)) * sizeof(double);
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_dq_fused, 256, smem);
-    if (e != cudaSuccess) return e;
-    const int64_t want = (nd + 7) / 8;
-    const int64_t cap = (int64_t)num_sms * (per_sm < 4 ? per_sm : 4);  // resident at once
-    if (cap < 1) return cudaErrorNotSupported;
-    const int grid = (int)(want < cap ? want : cap);
-    return launch_pdl(k_dq_fused, dim3(grid), dim3(256), smem, stream, 1, absmax, nb, run_sums, count, err, codes,
-                      absmax2, offset);
 }
 
 cudaError_t launch_dq_run_sums(const float *absmax, int64_t nb, double *run_sums, cudaStream_t stream) {

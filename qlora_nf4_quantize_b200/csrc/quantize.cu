@@ -85,16 +85,13 @@ __device__ __forceinline__ void quantize_group(float v[8], int64_t g, int64_t e0
     }
 }
 
-// zero_word (optional): set to 0 once the grid before has completed, for the
-// grid barrier of the fused double quantization launched next (double_quant.cu).
 template <bool kBf16>
 __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restrict__ w, int64_t n,
                                                              uint8_t *__restrict__ packed,
-                                                             float *__restrict__ absmax, unsigned *zero_word) {
+                                                             float *__restrict__ absmax) {
     __shared__ float s_t[16];
     __shared__ uint32_t s_cell[kCellTable];
     pdl_wait_then_release();
-    if (zero_word != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0u;
     build_code_tables(s_t, s_cell);
 
     const int lane = threadIdx.x & 31;
@@ -112,7 +109,7 @@ __global__ void __launch_bounds__(kQuantThreads) k_quantize(const void *__restri
 }  // namespace
 
 cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed, float *absmax,
-                            cudaStream_t stream, int num_sms, unsigned *zero_word) {
+                            cudaStream_t stream, int num_sms) {
     if (n == 0) return cudaSuccess;
     int64_t ngroups = (n + 7) / 8;
     int64_t span = (int64_t)kQuantThreads;
@@ -128,11 +125,8 @@ cudaError_t launch_quantize(const void *w, bool bf16, int64_t n, uint8_t *packed
     }
     int64_t cap = (int64_t)num_sms * per_sm;
     int grid = (int)(want < cap ? want : cap);
-    if (bf16)
-        return launch_pdl(k_quantize<true>, dim3(grid), dim3(kQuantThreads), 0, stream, 1, w, n, packed, absmax,
-                          zero_word);
-    return launch_pdl(k_quantize<false>, dim3(grid), dim3(kQuantThreads), 0, stream, 1, w, n, packed, absmax,
-                      zero_word);
+    if (bf16) return launch_pdl(k_quantize<true>, dim3(grid), dim3(kQuantThreads), 0, stream, 1, w, n, packed, absmax);
+    return launch_pdl(k_quantize<false>, dim3(grid), dim3(kQuantThreads), 0, stream, 1, w, n, packed, absmax);
 }
 
 }  // namespace nf4

@@ -86,10 +86,9 @@ def test_workspace_sizes(nf4lib):
     # fp64 run sums, then the chunk sums (32 runs each)
     assert nf4lib.nf4_double_quantize_workspace_size(2048) == (8 + 1) * 8        # 8 runs, 1 chunk
     assert nf4lib.nf4_double_quantize_workspace_size(256 * 33) == (33 + 2) * 8   # 33 runs, 2 chunks
-    # quantize + DQ in one call: fp32 constants (256-byte aligned), then the
-    # same sums, then the 8-byte grid-barrier word of the fused DQ launch
-    assert nf4lib.nf4_quantize_dq_workspace_size(4096 * 4096) == 262144 * 4 + (1024 + 32) * 8 + 8
-    assert nf4lib.nf4_quantize_dq_workspace_size(130) == 256 + (1 + 1) * 8 + 8
+    # quantize + DQ in one call: fp32 constants (256-byte aligned), then the same sums
+    assert nf4lib.nf4_quantize_dq_workspace_size(4096 * 4096) == 262144 * 4 + (1024 + 32) * 8
+    assert nf4lib.nf4_quantize_dq_workspace_size(130) == 256 + (1 + 1) * 8
     assert nf4lib.nf4_quantize_dq_workspace_size(128, 32, 256) == 0
     # [t_hi | t_lo | pad] rows of round_up(2r, 64) bf16; nothing without an
     # adapter (decode-size calls need no scratch of their own)

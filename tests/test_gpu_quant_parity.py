@@ -280,12 +280,10 @@ def wide_range_weight(n, seed):
                                             (16384 * 2100 + 130, "bf16", True), (256 * 512, "f32", False),
                                             (16384 * 7 + 4, "wide", True)])
 def test_quantize_dq_one_call(nf4lib, oracle_mod, cuda_device, n, dtype, centre):
-    """nf4_quantize_dq against the oracle's quantize + double quantize, bit
-    for bit, outputs and workspace guarded: centred tensors of up to 2048
-    runs take the fused launch (run sums, a grid barrier, the double
-    quantization; one run gives a one-CTA grid), larger ones and the
-    uncentred one the separate run-sum and chunk-sum launches.  A barrier
-    that timed out raises in nf4_device_status."""
+    """nf4_quantize_dq (quantizer writing the run sums, then one double
+    quantization kernel; above 2048 runs a chunk-sum kernel too) against the
+    oracle's quantize + double quantize, bit for bit, outputs and workspace
+    guarded."""
     if dtype == "wide":
         w_cpu = wide_range_weight(n, 5)
     else:
